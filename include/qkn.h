@@ -1,0 +1,209 @@
+/*
+ * qkn.h — C ABI of libqkn: QK-Normed MLA absorbed latent decode attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method ("QK-Normed MLA: QK normalization without full key caching",
+ * technical summary, Metodología items 1–4 and the decode-logit equation;
+ * arXiv abstract) keeps MLA's latent cache and adds post-projection QK
+ * RMSNorm without ever materialising a key:
+ *   - RMSNorm(z) = z * gamma / S(z) splits into a static weight gamma and a
+ *     dynamic scalar S(z);
+ *   - the static key weight gamma_k (and gamma_q) are folded into the query
+ *     side: q~[i,h] = W^K_{g(h),h} (gamma_q[h] * gamma_k[h] * q[i,h]);
+ *   - the dynamic key statistic becomes one inverse-RMS scalar per token and
+ *     KV group, a_k[t,g] = 1 / S(c_t W^K_g), cached next to the latent c_t;
+ *   - content and RoPE blocks are normalised separately; the RoPE block uses
+ *     ordinary materialised vectors;
+ *   - decode logits are l[i,t,h] = (q~[i,h] . c_t) * a_q[i,h] * a_k[t,g(h)]
+ *     + q^R^[i,h] . k^R^_t, a row/column rescale applied before the softmax;
+ *     the output is the softmax-weighted sum of the latents c_t.
+ *
+ * Conventions shared by every call
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory,
+ *     row-major, densely packed in the order the comments give.  The library
+ *     allocates nothing (the decode workspace is caller-allocated too).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only validates host-side arguments and enqueues kernels; it returns
+ *     before the GPU work runs.
+ *   - Argument errors are found on the host before anything is launched and
+ *     return QKN_ERR_INVALID_ARG or QKN_ERR_UNSUPPORTED; nothing is enqueued
+ *     then.  A failed launch returns QKN_ERR_CUDA.  Problems only the device
+ *     can see (a sequence length out of range, a bounded wait that ran out)
+ *     are recorded in the workspace's status word; read it with
+ *     qkn_read_device_status.
+ *   - dtype QKN_BF16 means activations (c, k^R, q, q^R), the cache, q~, q^R^
+ *     and the output are bf16; QKN_F32 means they are fp32.  Weights, norm
+ *     weights, a_k, a_q and lse are always fp32.
+ */
+#ifndef QKN_H_
+#define QKN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QKN_VERSION 1
+
+#if defined(__GNUC__)
+#define QKN_EXPORT __attribute__((visibility("default")))
+#else
+#define QKN_EXPORT
+#endif
+
+typedef enum {
+  QKN_OK = 0,
+  QKN_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or shape */
+  QKN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. a forced kernel that cannot take these dims) */
+  QKN_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  QKN_ERR_TIMEOUT = 4,       /* device: a bounded wait inside a kernel ran out */
+  QKN_ERR_BOUNDS = 5         /* device: a sequence length or block id outside its stated range */
+} qkn_status;
+
+typedef enum { QKN_F32 = 0, QKN_BF16 = 1 } qkn_dtype;
+
+/* Column scale used by qkn_decode.  QKN_AK_ONE treats every a_k as 1 and does
+ * not read the a_k cache: that is plain absorbed MLA on the same cache, the
+ * baseline for the method's overhead. */
+typedef enum { QKN_AK_CACHE = 0, QKN_AK_ONE = 1 } qkn_ak_mode;
+
+/* Decode kernel choice.  AUTO takes the tcgen05 kernel whenever the dims
+ * allow it and the CUDA-core kernel otherwise. */
+typedef enum { QKN_KERNEL_AUTO = 0, QKN_KERNEL_SIMT = 1, QKN_KERNEL_TCGEN05 = 2 } qkn_kernel;
+
+/* Model dimensions.  num_heads query heads form num_groups KV groups of
+ * n_g = num_heads / num_groups consecutive heads; head h belongs to group
+ * h / n_g and is slot h % n_g inside it.  W^K_g has n_g * d_h output columns,
+ * head h's key slice being columns [(h % n_g) * d_h, (h % n_g + 1) * d_h). */
+typedef struct {
+  int32_t num_heads;
+  int32_t num_groups;
+  int32_t r_kv;          /* latent width r */
+  int32_t d_h;           /* per-head content dimension */
+  int32_t d_rope;        /* RoPE dimension d_R (even) */
+  int32_t block_size;    /* cache page size in tokens; must be 64 */
+  float eps;             /* RMSNorm: S(z) = sqrt(mean(z^2) + eps), all four norms */
+  float softmax_scale;   /* sigma, applied to the whole logit (content + RoPE) */
+  float rope_theta;      /* RoPE base; pairs (i, i + d_R/2), angle pos * theta^(-2i/d_R) */
+  qkn_dtype dtype;
+} qkn_dims;
+
+/* The decode cache (technical summary, Metodología item 3: the latent c_t is
+ * the dominant state plus a small scalar cache of inverse RMS values; no
+ * normalised key is stored).  Caller-allocated device memory:
+ *   latent [num_blocks, block_size, r_kv]   dtype
+ *   k_rope [num_blocks, block_size, d_rope] dtype, RMS-normalised and rotated
+ *   a_k    [num_blocks, block_size, num_groups] fp32
+ * Slot s of the pool is token s % block_size of block s / block_size.
+ * Slots that no qkn_append has written may hold anything; decode never lets
+ * them reach its output. */
+typedef struct {
+  void* latent;
+  void* k_rope;
+  float* a_k;
+  int32_t num_blocks;
+} qkn_cache;
+
+/* Optional decode knobs (pass NULL for defaults). */
+typedef struct {
+  qkn_kernel kernel;       /* default QKN_KERNEL_AUTO */
+  int32_t max_ctas;        /* cap on decode CTAs (split-KV width); 0 = one per SM */
+  int32_t head_tile;       /* tcgen05: query rows per CTA (16, 32 or 64); 0 = automatic */
+  int64_t wait_limit;      /* bounded-wait limit in clock cycles for the mbarrier waits; 0 = default (~2 s) */
+} qkn_decode_opts;
+
+/* qkn_append — write n_tok new tokens into the cache.
+ * For token i with slot s = slot[i] and position p = pos[i]:
+ *   latent[s]  = c_new[i]                                    (copied as is)
+ *   k_rope[s]  = RoPE_p(gamma_kr * k_rope_raw[i] / S(k_rope_raw[i]))
+ *   a_k[s, g]  = 1 / S(c_new[i] W^K_g)   for every group g,
+ * S(z) = sqrt(mean(z^2) + eps) over the full n_g * d_h width of c W^K_g.
+ * This is the dynamic key statistic reduced to one scalar per token and KV
+ * group, computed once at append time (technical summary, Metodología items
+ * 2 and 4).  No key is stored.
+ *   c_new      [n_tok, r_kv]   dtype
+ *   k_rope_raw [n_tok, d_rope] dtype
+ *   slot, pos  [n_tok] int32; every slot in [0, num_blocks * block_size)
+ *   w_k        [num_groups, r_kv, n_g * d_h] fp32
+ *   gamma_kr   [d_rope] fp32 (shared by all heads)
+ * n_tok == 0 is a no-op.  Slots must be distinct within one call. */
+QKN_EXPORT qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache,
+                      const void* c_new, const void* k_rope_raw,
+                      const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                      const float* w_k, const float* gamma_kr, void* stream);
+
+/* qkn_absorb_query — fold the static norm weights into the query
+ * (technical summary, Metodología item 1 and the decode-logit equation).
+ * For query row i and head h (group g = h / n_g, slot m = h % n_g):
+ *   q_tilde[i,h]    = W^K_g[:, m*d_h:(m+1)*d_h] (gamma_q[h] * gamma_k[h] * q[i,h])   in R^r
+ *   a_q[i,h]        = softmax_scale / S(q[i,h])            (row scale, sigma folded in)
+ *   q_rope_hat[i,h] = softmax_scale * RoPE_{pos[i]}(gamma_qr[h] * q_rope[i,h] / S(q_rope[i,h]))
+ *   q          [n_q, H, d_h]    dtype       gamma_q, gamma_k [H, d_h] fp32
+ *   q_rope     [n_q, H, d_rope] dtype       gamma_qr [H, d_rope] fp32
+ *   pos        [n_q] int32 RoPE positions of the query rows
+ *   w_k        [num_groups, r_kv, n_g * d_h] fp32
+ *   q_tilde    [n_q, H, r_kv] dtype (out), a_q [n_q, H] fp32 (out),
+ *   q_rope_hat [n_q, H, d_rope] dtype (out).
+ * n_q == 0 is a no-op. */
+QKN_EXPORT qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_rope,
+                            const int32_t* pos, int32_t n_q, const float* w_k,
+                            const float* gamma_q, const float* gamma_k, const float* gamma_qr,
+                            void* q_tilde, float* a_q, void* q_rope_hat, void* stream);
+
+/* Bytes of decode workspace needed for `batch` sequences of `s_q` query
+ * tokens on a GPU with `num_sms` SMs (0 = ask the current device).  The
+ * workspace holds a status word and the per-split partial results of the
+ * split-KV decode.  Returns QKN_ERR_INVALID_ARG for bad dims. */
+QKN_EXPORT qkn_status qkn_decode_workspace_size(const qkn_dims* dims, int32_t batch, int32_t s_q,
+                                     int32_t num_sms, size_t* bytes);
+
+/* Zero the workspace's status word (once, after allocating the workspace,
+ * and after handling a reported device error).  Enqueued on `stream`. */
+QKN_EXPORT qkn_status qkn_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* qkn_decode — one decode step of QK-Normed MLA attention over the cache.
+ * Query row i = b * s_q + j is query token j of sequence b, at position
+ * L_b - s_q + j; it attends to the tokens t of sequence b with t <= that
+ * position (causal within the step).  For head h in group g:
+ *   l[t]  = a_q[i,h] * a_k[t,g] * (q_tilde[i,h] . c_t) + q_rope_hat[i,h] . k^R^_t
+ *   out[i,h] = sum_t softmax(l)[t] * c_t,   lse[i,h] = log sum_t exp(l[t])
+ * (technical summary, Metodología, decode-logit equation: scalar factors as
+ * a row/column rescale before the softmax).  The context is split across
+ * CTAs (split-KV) and the partial results are merged by a combine kernel.
+ *   q_tilde    [batch*s_q, H, r_kv] dtype; a_q [batch*s_q, H] fp32
+ *   q_rope_hat [batch*s_q, H, d_rope] dtype
+ *   block_table [batch, max_blocks] int32: block j of sequence b holds its
+ *              tokens [64j, 64j+64); only the first ceil(L_b/64) entries of
+ *              a row are read
+ *   seq_lens   [batch] int32 on the device, s_q <= L_b <= max_blocks * 64
+ *   workspace  >= qkn_decode_workspace_size(...) bytes, 256-byte aligned,
+ *              initialised once with qkn_workspace_init
+ *   out        [batch, s_q, H, r_kv] dtype; lse [batch, s_q, H] fp32
+ * A sequence whose length breaks its bound is recorded as QKN_ERR_BOUNDS in
+ * the status word and its rows are written as zeros with lse = -inf. */
+QKN_EXPORT qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode,
+                      const void* q_tilde, const float* a_q, const void* q_rope_hat,
+                      const int32_t* block_table, int32_t max_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t s_q,
+                      void* workspace, size_t ws_bytes, void* out, float* lse,
+                      const qkn_decode_opts* opts, void* stream);
+
+/* Synchronise `stream`, then read the workspace status word into *device_status
+ * (a qkn_status value; QKN_OK if no kernel recorded an error).  The word is
+ * sticky until qkn_workspace_init clears it. */
+QKN_EXPORT qkn_status qkn_read_device_status(const void* workspace, void* stream, int32_t* device_status);
+
+/* Which decode kernel qkn_decode would run for these dims and options
+ * (QKN_KERNEL_SIMT or QKN_KERNEL_TCGEN05), or -1 if none can. */
+QKN_EXPORT int32_t qkn_decode_kernel_for(const qkn_dims* dims, int32_t s_q, const qkn_decode_opts* opts);
+
+QKN_EXPORT const char* qkn_status_string(qkn_status status);
+QKN_EXPORT int32_t qkn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKN_H_ */

@@ -1,0 +1,294 @@
+// The C ABI of libqkn (declared in include/qkn.h): host-side argument checks,
+// kernel selection, the decode workspace layout and kernel launches.  Every
+// entry point validates before it enqueues anything, and none allocates.
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace qkn;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t elem_size(qkn_dtype t) { return t == QKN_BF16 ? 2 : 4; }
+
+qkn_status check_dims(const qkn_dims* d) {
+  if (!d) return QKN_ERR_INVALID_ARG;
+  if (d->dtype != QKN_F32 && d->dtype != QKN_BF16) return QKN_ERR_INVALID_ARG;
+  if (d->num_heads <= 0 || d->num_groups <= 0 || d->num_heads % d->num_groups) return QKN_ERR_INVALID_ARG;
+  if (d->block_size != kBlockSize) return QKN_ERR_INVALID_ARG;
+  if (d->d_h <= 0 || d->d_h > 1024) return QKN_ERR_INVALID_ARG;
+  // 16-byte rows for every token-major array (vector loads, TMA rows).
+  if (d->r_kv <= 0 || d->r_kv > 1024 || (d->r_kv * elem_size(d->dtype)) % 16) return QKN_ERR_INVALID_ARG;
+  if (d->d_rope <= 0 || d->d_rope > 128 || (d->d_rope % 2) ||
+      (d->d_rope * elem_size(d->dtype)) % 16)
+    return QKN_ERR_INVALID_ARG;
+  if (!(d->eps >= 0.f) || !(d->softmax_scale > 0.f) || !(d->rope_theta > 0.f)) return QKN_ERR_INVALID_ARG;
+  const int64_t width = (int64_t)(d->num_heads / d->num_groups) * d->d_h;
+  if (width > (1 << 24)) return QKN_ERR_INVALID_ARG;
+  return QKN_OK;
+}
+
+qkn_status check_cache(const qkn_dims* d, const qkn_cache* c) {
+  if (!c || !c->latent || !c->k_rope || !c->a_k || c->num_blocks <= 0) return QKN_ERR_INVALID_ARG;
+  if (!aligned(c->latent, 16) || !aligned(c->k_rope, 16) || !aligned(c->a_k, 16)) return QKN_ERR_INVALID_ARG;
+  if ((int64_t)c->num_blocks * kBlockSize > INT32_MAX) return QKN_ERR_INVALID_ARG;
+  (void)d;
+  return QKN_OK;
+}
+
+int sm_count(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+    *out = cached[dev];
+    return 0;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  *out = n;
+  return 0;
+}
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Rows per tile for the tcgen05 kernel: the smallest supported tile that
+// covers the per-sequence query rows, capped at 64 (the accumulator of a
+// 64-row tile already fills the tensor memory of one SM).
+int tc_rows(const qkn_dims* d, int s_q, const qkn_decode_opts* o) {
+  if (o && o->head_tile) return o->head_tile;
+  const int qrows = s_q * d->num_heads;
+  if (qrows <= 16) return 16;
+  if (qrows <= 32) return 32;
+  return 64;
+}
+
+int pick_kernel(const qkn_dims* d, int s_q, const qkn_decode_opts* o) {
+  const qkn_kernel want = o ? o->kernel : QKN_KERNEL_AUTO;
+  const bool tc_ok = d->dtype == QKN_BF16 && decode_tc_supported(d->r_kv, d->d_rope, tc_rows(d, s_q, o), d->num_groups);
+  if (want == QKN_KERNEL_SIMT) return QKN_KERNEL_SIMT;
+  if (want == QKN_KERNEL_TCGEN05) return tc_ok ? QKN_KERNEL_TCGEN05 : -1;
+  if (want != QKN_KERNEL_AUTO) return -1;
+  return tc_ok ? QKN_KERNEL_TCGEN05 : QKN_KERNEL_SIMT;
+}
+
+struct WsLayout {
+  size_t lse_off, o_off, total;
+};
+
+WsLayout ws_layout(const qkn_dims* d, int batch, int s_q, int ncta) {
+  // Size for the largest row tile any kernel may use, so that one workspace
+  // serves every kernel choice.
+  int64_t slot_rows = 0;
+  const int qrows = s_q * d->num_heads;
+  for (int rows : {kSimtRows, 16, 32, 64}) {
+    const int64_t ht = ceil_div(qrows, rows);
+    const int64_t sr = sched_slots(batch, ht, ncta) * rows;
+    if (sr > slot_rows) slot_rows = sr;
+  }
+  WsLayout w;
+  w.lse_off = kStatusBytes;
+  const size_t lse_bytes = ((size_t)slot_rows * 4 + 255) / 256 * 256;
+  w.o_off = w.lse_off + lse_bytes;
+  w.total = w.o_off + (size_t)slot_rows * d->r_kv * 4;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qkn_status_string(qkn_status s) {
+  switch (s) {
+    case QKN_OK: return "ok";
+    case QKN_ERR_INVALID_ARG: return "invalid argument";
+    case QKN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QKN_ERR_CUDA: return "CUDA error";
+    case QKN_ERR_TIMEOUT: return "device wait timed out";
+    case QKN_ERR_BOUNDS: return "sequence length or block id out of range";
+  }
+  return "unknown status";
+}
+
+int32_t qkn_version(void) { return QKN_VERSION; }
+
+qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache, const void* c_new,
+                      const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                      const float* w_k, const float* gamma_kr, void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (n_tok < 0) return QKN_ERR_INVALID_ARG;
+  if (n_tok == 0) return QKN_OK;
+  if ((st = check_cache(dims, cache)) != QKN_OK) return st;
+  if (!c_new || !k_rope_raw || !slot || !pos || !w_k || !gamma_kr) return QKN_ERR_INVALID_ARG;
+  if (!aligned(c_new, 16) || !aligned(k_rope_raw, 16)) return QKN_ERR_INVALID_ARG;
+  AppendArgs a;
+  a.latent = cache->latent;
+  a.k_rope = cache->k_rope;
+  a.a_k = cache->a_k;
+  a.c_new = c_new;
+  a.k_rope_raw = k_rope_raw;
+  a.slot = slot;
+  a.pos = pos;
+  a.w_k = w_k;
+  a.gamma_kr = gamma_kr;
+  a.n_tok = n_tok;
+  a.r = dims->r_kv;
+  a.d_rope = dims->d_rope;
+  a.groups = dims->num_groups;
+  a.width = (dims->num_heads / dims->num_groups) * dims->d_h;
+  a.eps = dims->eps;
+  a.rope_theta = dims->rope_theta;
+  cudaError_t e = launch_append(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_rope, const int32_t* pos,
+                            int32_t n_q, const float* w_k, const float* gamma_q, const float* gamma_k,
+                            const float* gamma_qr, void* q_tilde, float* a_q, void* q_rope_hat,
+                            void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (n_q < 0) return QKN_ERR_INVALID_ARG;
+  if (n_q == 0) return QKN_OK;
+  if (!q || !q_rope || !pos || !w_k || !gamma_q || !gamma_k || !gamma_qr || !q_tilde || !a_q || !q_rope_hat)
+    return QKN_ERR_INVALID_ARG;
+  if (dims->d_h > 256) return QKN_ERR_UNSUPPORTED;
+  AbsorbArgs a;
+  a.q = q;
+  a.q_rope = q_rope;
+  a.pos = pos;
+  a.w_k = w_k;
+  a.gamma_q = gamma_q;
+  a.gamma_k = gamma_k;
+  a.gamma_qr = gamma_qr;
+  a.q_tilde = q_tilde;
+  a.a_q = a_q;
+  a.q_rope_hat = q_rope_hat;
+  a.n_q = n_q;
+  a.heads = dims->num_heads;
+  a.groups = dims->num_groups;
+  a.r = dims->r_kv;
+  a.d_h = dims->d_h;
+  a.d_rope = dims->d_rope;
+  a.eps = dims->eps;
+  a.softmax_scale = dims->softmax_scale;
+  a.rope_theta = dims->rope_theta;
+  cudaError_t e = launch_absorb(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+qkn_status qkn_decode_workspace_size(const qkn_dims* dims, int32_t batch, int32_t s_q, int32_t num_sms,
+                                     size_t* bytes) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (!bytes || batch < 0 || s_q < 1 || num_sms < 0) return QKN_ERR_INVALID_ARG;
+  int n = num_sms;
+  if (n == 0 && sm_count(&n) != 0) return QKN_ERR_CUDA;
+  *bytes = ws_layout(dims, batch, s_q, n).total;
+  return QKN_OK;
+}
+
+qkn_status qkn_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || ws_bytes < (size_t)kStatusBytes || !aligned(workspace, 256)) return QKN_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+int32_t qkn_decode_kernel_for(const qkn_dims* dims, int32_t s_q, const qkn_decode_opts* opts) {
+  if (check_dims(dims) != QKN_OK || s_q < 1) return -1;
+  return pick_kernel(dims, s_q, opts);
+}
+
+qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode, const void* q_tilde,
+                      const float* a_q, const void* q_rope_hat, const int32_t* block_table, int32_t max_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t s_q, void* workspace, size_t ws_bytes,
+                      void* out, float* lse, const qkn_decode_opts* opts, void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if ((st = check_cache(dims, cache)) != QKN_OK) return st;
+  if (ak_mode != QKN_AK_CACHE && ak_mode != QKN_AK_ONE) return QKN_ERR_INVALID_ARG;
+  if (batch < 0 || s_q < 1 || max_blocks < 1) return QKN_ERR_INVALID_ARG;
+  if (batch == 0) return QKN_OK;
+  if (!q_tilde || !a_q || !q_rope_hat || !block_table || !seq_lens || !workspace || !out || !lse)
+    return QKN_ERR_INVALID_ARG;
+  if (!aligned(q_tilde, 16) || !aligned(q_rope_hat, 16) || !aligned(workspace, 256)) return QKN_ERR_INVALID_ARG;
+  if (opts && (opts->max_ctas < 0 || opts->wait_limit < 0 ||
+               (opts->head_tile && opts->head_tile != 16 && opts->head_tile != 32 && opts->head_tile != 64)))
+    return QKN_ERR_INVALID_ARG;
+  const int kernel = pick_kernel(dims, s_q, opts);
+  if (kernel < 0) return QKN_ERR_UNSUPPORTED;
+
+  int nsm = 0;
+  if (sm_count(&nsm) != 0) return QKN_ERR_CUDA;
+  const WsLayout w = ws_layout(dims, batch, s_q, nsm);
+  if (ws_bytes < w.total) return QKN_ERR_INVALID_ARG;
+  int ncta = nsm;
+  if (opts && opts->max_ctas > 0 && opts->max_ctas < ncta) ncta = opts->max_ctas;
+
+  char* ws = static_cast<char*>(workspace);
+  DecodeArgs a;
+  a.latent = cache->latent;
+  a.k_rope = cache->k_rope;
+  a.a_k = cache->a_k;
+  a.num_blocks = cache->num_blocks;
+  a.q_tilde = q_tilde;
+  a.a_q = a_q;
+  a.q_rope_hat = q_rope_hat;
+  a.block_table = block_table;
+  a.max_blocks = max_blocks;
+  a.seq_lens = seq_lens;
+  a.batch = batch;
+  a.s_q = s_q;
+  a.heads = dims->num_heads;
+  a.groups = dims->num_groups;
+  a.r = dims->r_kv;
+  a.d_rope = dims->d_rope;
+  a.ak_one = ak_mode == QKN_AK_ONE;
+  a.rows = kernel == QKN_KERNEL_TCGEN05 ? tc_rows(dims, s_q, opts) : kSimtRows;
+  a.ht_count = ceil_div(s_q * dims->num_heads, a.rows);
+  a.ncta = ncta;
+  a.part_lse = reinterpret_cast<float*>(ws + w.lse_off);
+  a.part_o = reinterpret_cast<float*>(ws + w.o_off);
+  a.status = reinterpret_cast<int32_t*>(ws);
+  a.wait_limit = (opts && opts->wait_limit > 0) ? opts->wait_limit : (int64_t)4000000000LL;
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dims->dtype == QKN_BF16;
+  cudaError_t e = kernel == QKN_KERNEL_TCGEN05 ? launch_decode_tc(a, cs) : launch_decode_simt(a, bf16, cs);
+  if (e != cudaSuccess) return QKN_ERR_CUDA;
+
+  CombineArgs c;
+  c.seq_lens = seq_lens;
+  c.batch = batch;
+  c.s_q = s_q;
+  c.heads = dims->num_heads;
+  c.r = dims->r_kv;
+  c.rows = a.rows;
+  c.ht_count = a.ht_count;
+  c.ncta = ncta;
+  c.max_blocks = max_blocks;
+  c.part_o = a.part_o;
+  c.part_lse = a.part_lse;
+  c.out = out;
+  c.lse = lse;
+  c.status = a.status;
+  e = launch_combine(c, bf16, cs);
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+qkn_status qkn_read_device_status(const void* workspace, void* stream, int32_t* device_status) {
+  if (!workspace || !device_status) return QKN_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QKN_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return QKN_ERR_CUDA;
+  *device_status = v;
+  return QKN_OK;
+}
+
+}  // extern "C"

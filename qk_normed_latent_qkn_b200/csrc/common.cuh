@@ -1,0 +1,172 @@
+// Shared device helpers for libqkn: element types, the device status word,
+// and the split-KV work schedule used by the decode and combine kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/qkn.h"
+
+namespace qkn {
+
+constexpr int kBlockSize = 64;          // tokens per cache page
+constexpr int kStatusBytes = 256;       // workspace header holding the status word
+
+// ---------------------------------------------------------------- elements
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------- status word
+// The first int32 of the decode workspace.  Kernels record the first error
+// they see (compare-and-swap from QKN_OK); the host reads it after a sync.
+__device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
+  if (status) atomicCAS(status, (int32_t)QKN_OK, code);
+}
+
+// ---------------------------------------------------------------- schedule
+// The decode work of one step is a list of "units": one cache page (64
+// tokens) of one segment, a segment being (sequence b, query-row tile ht).
+// Segments are ordered (b, ht) and units inside a segment by page, so the
+// units of segment (b, ht) are [HT*P(b) + ht*n(b), ... + n(b)) where n(b) is
+// the page count of sequence b and P(b) the pages of sequences before it.
+// CTA c of `ncta` takes the contiguous unit range [c*Q, (c+1)*Q) with
+// Q = ceil(total / ncta).  The piece of segment s that CTA c works on is an
+// "item"; its partial result goes to workspace slot s + c, which is unique
+// because segments and CTAs advance together.
+struct SchedParams {
+  const int32_t* seq_lens;
+  int32_t batch;
+  int32_t s_q;
+  int32_t max_blocks;
+  int32_t ht_count;     // query-row tiles per sequence
+  int32_t ncta;
+};
+
+__device__ __forceinline__ int32_t pages_of(int32_t L, const SchedParams& p) {
+  if (L < p.s_q || L > p.max_blocks * kBlockSize) return 0;   // rejected length
+  return (L + kBlockSize - 1) / kBlockSize;
+}
+
+// Total units, computed by one full warp (all lanes get the result).
+__device__ __forceinline__ int64_t sched_total_units(const SchedParams& p) {
+  const int lane = threadIdx.x & 31;
+  int64_t acc = 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    int b = b0 + lane;
+    int64_t n = (b < p.batch) ? pages_of(p.seq_lens[b], p) : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    acc += n;
+  }
+  return acc * p.ht_count;
+}
+
+// Pages before sequence b (P(b)), computed by one full warp.
+__device__ __forceinline__ int64_t sched_pages_before(const SchedParams& p, int32_t b_end) {
+  const int lane = threadIdx.x & 31;
+  int64_t acc = 0;
+  for (int b0 = 0; b0 < b_end; b0 += 32) {
+    int b = b0 + lane;
+    int64_t n = (b < b_end) ? pages_of(p.seq_lens[b], p) : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    acc += n;
+  }
+  return acc;
+}
+
+// Cursor over the items of one CTA.  Start it with sched_begin (one full
+// warp), copy it to every role, then step with sched_next (any thread).
+struct Cursor {
+  int64_t begin, end;    // this CTA's unit range
+  int64_t seg_u0;        // first unit of the current segment
+  int32_t b, ht;         // current segment
+  int32_t n;             // pages of sequence b
+  int64_t quota;         // Q
+};
+
+// Item handed to the roles: pages [p0, p1) of sequence b, row tile ht.
+struct Item {
+  int32_t b, ht, p0, p1, L, slot;
+};
+
+__device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta) {
+  Cursor cur;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = sched_total_units(p);
+  const int64_t q = (total + p.ncta - 1) / (p.ncta > 0 ? p.ncta : 1);
+  cur.quota = q;
+  cur.begin = (int64_t)cta * q;
+  cur.end = cur.begin + q < total ? cur.begin + q : total;
+  cur.b = p.batch;
+  cur.ht = 0;
+  cur.n = 0;
+  cur.seg_u0 = total;
+  if (cur.begin >= cur.end) return cur;
+  // Find the sequence holding unit `begin`: scan with a warp prefix sum.
+  int64_t base = 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    int b = b0 + lane;
+    int64_t n = (b < p.batch) ? pages_of(p.seq_lens[b], p) * (int64_t)p.ht_count : 0;
+    int64_t incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int64_t lo = base + incl - n, hi = base + incl;
+    const unsigned hit = __ballot_sync(0xffffffffu, b < p.batch && n > 0 && cur.begin >= lo && cur.begin < hi);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      const int64_t seq_lo = __shfl_sync(0xffffffffu, lo, src);
+      const int32_t bb = b0 + src;
+      const int32_t nn = pages_of(p.seq_lens[bb], p);
+      cur.b = bb;
+      cur.n = nn;
+      cur.ht = (int32_t)((cur.begin - seq_lo) / nn);
+      cur.seg_u0 = seq_lo + (int64_t)cur.ht * nn;
+      return cur;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return cur;
+}
+
+// Returns false when the CTA has no further item.  Any single thread.
+__device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, int32_t cta, Item& it) {
+  while (cur.b < p.batch && cur.seg_u0 < cur.end) {
+    const int64_t s0 = cur.seg_u0, s1 = cur.seg_u0 + cur.n;
+    const bool overlaps = cur.n > 0 && s1 > cur.begin;
+    if (overlaps) {
+      it.b = cur.b;
+      it.ht = cur.ht;
+      it.p0 = (int32_t)((cur.begin > s0 ? cur.begin : s0) - s0);
+      it.p1 = (int32_t)((cur.end < s1 ? cur.end : s1) - s0);
+      it.L = p.seq_lens[cur.b];
+      it.slot = cur.b * p.ht_count + cur.ht + cta;
+    }
+    // advance to the next segment
+    cur.seg_u0 = s1;
+    if (++cur.ht >= p.ht_count || cur.n == 0) {
+      cur.ht = 0;
+      ++cur.b;
+      cur.n = cur.b < p.batch ? pages_of(p.seq_lens[cur.b], p) : 0;
+      if (cur.n == 0) cur.ht = 0;
+    }
+    if (overlaps) return true;
+  }
+  return false;
+}
+
+// Workspace slots needed: one per (segment, CTA) pair that can meet.
+inline int64_t sched_slots(int64_t batch, int64_t ht_count, int64_t ncta) {
+  return batch * ht_count + ncta;
+}
+
+}  // namespace qkn

@@ -1,0 +1,599 @@
+// Split-KV QK-Normed MLA decode on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// What it computes ("QK-Normed MLA: QK normalization without full key
+// caching", technical summary, Metodología, decode-logit equation; the
+// scalar factors are fused into the attention kernel as the summary's
+// caveats ask): for every query row rho of a tile and every cached token t
+//   l[t, rho] = a_q[rho] * a_k[t, g(rho)] * (c_t . q~[rho]) + k^R^_t . q^R^[rho]
+// then an online softmax over the CTA's token range and O = sum_t p * c_t.
+//
+// Orientation ("swap AB"): tokens are the MMA M dimension (128 per tile = two
+// 64-token pages) and query rows are N (R = 16, 32 or 64), so one tile is
+//   S^T[128 x R]  = C[128 x 512] . Q~^T            (K = latent, 32 MMAs)
+//   S_R^T[128 x R] = K^R[128 x 64] . Q^R^T          (K = RoPE,   4 MMAs)
+//   O^T[512 x R] += C^T[512 x 128] . P^T[128 x R]   (4 latent blocks x 8 MMAs)
+// with the latent tile C staged once in shared memory and read by both
+// products (as K-major A for S, as MN-major A for O).  The fp32 accumulator
+// O^T takes 4R TMEM columns, S^T and S_R^T R columns each.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warps 0-3  softmax + epilogue: thread t owns TMEM lane t = token row t of
+//              S^T and latent row t of each O^T block; column (query row)
+//              maxima and sums are reduced across the 128 threads;
+//   warp 4     TMA producer: query tiles per item, then per tile eight 16 KB
+//              latent chunks, the RoPE-key chunk and the a_k rows;
+//   warp 5     TMEM allocator and single-thread MMA issuer.
+// Shared-memory rings: latent chunks (full/empty mbarrier pairs), and a
+// RoPE-key slot that the softmax reuses for P^T once the RoPE MMAs are done.
+// Every mbarrier wait is bounded; a wait that runs out records
+// QKN_ERR_TIMEOUT in the workspace status word and the CTA winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace qkn {
+using namespace sm100;
+
+namespace {
+
+constexpr int kTile = 128;                 // tokens per tile (MMA M)
+constexpr int kRkv = 512;                  // latent width this kernel takes
+constexpr int kChunks = kRkv / 64;         // 64-column (128-byte) chunks of the latent
+constexpr int kDrope = 64;                 // RoPE width this kernel takes
+constexpr int kSlotBytes = kTile * 128;    // one chunk of one tile: 16 KB
+constexpr int kPageChunkBytes = 64 * 128;  // one chunk of one page: 8 KB
+constexpr int kMaxGroups = 8;
+constexpr int kAkSlotBytes = kTile * kMaxGroups * 4;
+constexpr int kThreads = 192;
+constexpr int kSoftThreads = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;       // rescale O only when a column max grows by > 2^8
+constexpr int64_t kDrainLimit = 4000000000LL;
+
+template <int R>
+struct Cfg {
+  static constexpr int NS = (R == 64) ? 8 : 10;              // latent chunk slots (even)
+  static constexpr int NKR = (R == 16) ? 2 : 1;              // RoPE-key / P^T slots
+  static constexpr int TMEM_COLS = (6 * R <= 128) ? 128 : (6 * R <= 256 ? 256 : 512);
+  static constexpr int Q_OFF = 0;                                    // R x 512 bf16, 8 chunks
+  static constexpr int QR_OFF = Q_OFF + R * 1024;                    // R x 64 bf16
+  static constexpr int C_OFF = QR_OFF + ((R * 128 + 1023) / 1024) * 1024;
+  static constexpr int KR_OFF = C_OFF + NS * kSlotBytes;
+  static constexpr int AK_OFF = KR_OFF + NKR * kSlotBytes;
+  static constexpr int MISC_OFF = AK_OFF + NKR * kAkSlotBytes;
+  static constexpr int MISC_BYTES = 4096;
+  static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;          // + alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(4 * R + 2 * R <= TMEM_COLS, "tensor memory budget");
+};
+
+template <int R, int NS, int NKR>
+struct Misc {
+  uint64_t full[NS], empty[NS], krfull[NKR], krempty[NKR];
+  uint64_t q_full, q_empty, s_full, p_full, o_full, o_empty, drain;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+  Cursor cursor;
+  float aq2[R];      // a_q * log2(e) per column (query row)
+  int32_t grp[R];    // KV group per column
+  int32_t qlim[R];   // last visible token position per column (-1: padding column)
+  float mu[R];       // running max (log2 units) used for the exponentials
+  float corr[R];     // rescale factor of the current tile
+  float linv[R];
+  float red[4][R];   // per-warp partial column reductions
+};
+
+}  // namespace
+
+struct TcMaps {
+  CUtensorMap latent;   // [num_blocks*64, 512] bf16, box 64 x 64
+  CUtensorMap krope;    // [num_blocks*64, 64]  bf16, box 64 x 64
+  CUtensorMap qt;       // [n_q*H, 512]         bf16, box 64 x R
+  CUtensorMap qr;       // [n_q*H, 64]          bf16, box 64 x R
+};
+
+// Column reduction across the 32 lanes of a warp: on entry each lane holds R
+// values (one per column); on exit lane L holds the reduction over the warp's
+// 32 rows of columns [L*R/32, (L+1)*R/32) (R >= 32) or of column L*R/32
+// (R < 32; neighbouring lanes hold the same column).  Each step hands half of
+// the remaining columns to the partner lane, so the whole reduction takes
+// R-1 shuffles (plus plain butterflies once one column is left).
+template <int R, bool MAX>
+__device__ __forceinline__ void warp_col_reduce(float (&v)[R], int lane) {
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int len = R >> s;
+    const int bit = 16 >> s;
+    const bool upper = (lane & bit) != 0;
+    if (len >= 2) {
+      const int half = len / 2;
+#pragma unroll
+      for (int c = 0; c < half; ++c) {
+        const float send = upper ? v[c] : v[c + half];
+        const float keep = upper ? v[c + half] : v[c];
+        const float got = __shfl_xor_sync(0xffffffffu, send, bit);
+        v[c] = MAX ? fmaxf(keep, got) : keep + got;
+      }
+    } else {
+      const float got = __shfl_xor_sync(0xffffffffu, v[0], bit);
+      v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
+    }
+  }
+}
+
+// Write the warp-reduced columns of this lane into red[warp][...].
+template <int R>
+__device__ __forceinline__ void store_reduced(float* red_w, const float (&v)[R], int lane) {
+  if constexpr (R >= 32) {
+    constexpr int per = R / 32;
+#pragma unroll
+    for (int i = 0; i < per; ++i) red_w[lane * per + i] = v[i];
+  } else {
+    constexpr int share = 32 / R;
+    if ((lane % share) == 0) red_w[lane / share] = v[0];
+  }
+}
+
+__device__ __forceinline__ bool group_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ bool group_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+template <int R, bool AK_ONE>
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TcMaps maps) {
+  using C = Cfg<R>;
+  constexpr int NS = C::NS, NKR = C::NKR;
+  using MiscT = Misc<R, NS, NKR>;
+  static_assert(sizeof(MiscT) <= C::MISC_BYTES, "misc shared-memory block");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  MiscT& ms = *reinterpret_cast<MiscT*>(smem + C::MISC_OFF);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
+  const int qrows = a.s_q * a.heads;
+  const int G = a.groups;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&ms.full[s]), 1);
+      mbar_init(smem_u32(&ms.empty[s]), 1);
+    }
+    for (int s = 0; s < NKR; ++s) {
+      mbar_init(smem_u32(&ms.krfull[s]), 1);
+      mbar_init(smem_u32(&ms.krempty[s]), 1);
+    }
+    mbar_init(smem_u32(&ms.q_full), 1);
+    mbar_init(smem_u32(&ms.q_empty), 1);
+    mbar_init(smem_u32(&ms.s_full), 1);
+    mbar_init(smem_u32(&ms.p_full), kSoftThreads);
+    mbar_init(smem_u32(&ms.o_full), 1);
+    mbar_init(smem_u32(&ms.o_empty), kSoftThreads);
+    mbar_init(smem_u32(&ms.drain), 1);
+    ms.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&maps.latent);
+    prefetch_tmap(&maps.krope);
+    prefetch_tmap(&maps.qt);
+    prefetch_tmap(&maps.qr);
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&ms.tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0) {
+    Cursor c = sched_begin(sp, blockIdx.x);
+    if (lane == 0) ms.cursor = c;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem_base;
+  Cursor cur = ms.cursor;
+  Item it;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int64_t c_it = 0, k_it = 0;
+      int n_item = 0;
+      bool ok = true;
+      while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+        if (!mbar_wait(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+        const int qrow0 = it.b * qrows + it.ht * R;
+        const uint32_t qf = smem_u32(&ms.q_full);
+        mbar_arrive_expect_tx(qf, R * 1024 + R * 128);
+#pragma unroll
+        for (int k = 0; k < kChunks; ++k) tma_load_2d(sb + C::Q_OFF + k * R * 128, &maps.qt, k * 64, qrow0, qf);
+        tma_load_2d(sb + C::QR_OFF, &maps.qr, 0, qrow0, qf);
+        const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
+        for (int p = it.p0; p < it.p1 && ok; p += 2) {
+          const int np = min(2, it.p1 - p);
+          int32_t blk[2] = {row[p], np > 1 ? row[p + 1] : 0};
+          for (int i = 0; i < np; ++i)
+            if (blk[i] < 0 || blk[i] >= a.num_blocks) {
+              record_status(a.status, QKN_ERR_BOUNDS);
+              blk[i] = 0;
+            }
+          for (int k = 0; k < kChunks; ++k) {
+            const int slot = (int)(c_it % NS);
+            if (!mbar_wait(smem_u32(&ms.empty[slot]), ((c_it / NS) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&ms.full[slot]);
+            mbar_arrive_expect_tx(fb, np * kPageChunkBytes);
+            const uint32_t dst = sb + C::C_OFF + slot * kSlotBytes;
+            for (int i = 0; i < np; ++i) tma_load_2d(dst + i * kPageChunkBytes, &maps.latent, k * 64, blk[i] * 64, fb);
+            ++c_it;
+          }
+          if (!ok) break;
+          const int ks = (int)(k_it % NKR);
+          if (!mbar_wait(smem_u32(&ms.krempty[ks]), ((k_it / NKR) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+          const uint32_t kb = smem_u32(&ms.krfull[ks]);
+          const uint32_t akpage = 64u * (uint32_t)G * 4u;
+          mbar_arrive_expect_tx(kb, np * kPageChunkBytes + (AK_ONE ? 0u : np * akpage));
+          for (int i = 0; i < np; ++i) {
+            tma_load_2d(sb + C::KR_OFF + ks * kSlotBytes + i * kPageChunkBytes, &maps.krope, 0, blk[i] * 64, kb);
+            if (!AK_ONE)
+              bulk_load(sb + C::AK_OFF + ks * kAkSlotBytes + i * akpage, a.a_k + (int64_t)blk[i] * 64 * G, akpage, kb);
+          }
+          ++k_it;
+        }
+        ++n_item;
+      }
+      if (!ok) {
+        record_status(a.status, QKN_ERR_TIMEOUT);
+        ms.abort_flag = 1;
+        // let the copies already in flight land before the CTA's memory is released
+        const int64_t first = c_it > NS ? c_it - NS : 0;
+        for (int64_t i = first; i < c_it; ++i)
+          mbar_wait(smem_u32(&ms.full[i % NS]), (i / NS) & 1, kDrainLimit);
+        const int64_t kfirst = k_it > NKR ? k_it - NKR : 0;
+        for (int64_t i = kfirst; i < k_it; ++i)
+          mbar_wait(smem_u32(&ms.krfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, R, false, false);
+      constexpr uint32_t idPV = idesc_bf16(128, R, true, false);
+      const uint32_t tS = tmem + 4 * R, tSR = tmem + 5 * R;
+      int64_t c_it = 0, k_it = 0, tile_n = 0;
+      int n_item = 0;
+      bool ok = true;
+      while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+        if (!mbar_wait(smem_u32(&ms.q_full), n_item & 1, a.wait_limit)) { ok = false; break; }
+        tc_fence_after();
+        const int ntiles = (it.p1 - it.p0 + 1) / 2;
+        for (int i = 0; i < ntiles && ok; ++i) {
+          const int np = min(2, it.p1 - (it.p0 + 2 * i));
+          const int64_t c_first = c_it;
+          // S^T = C . Q~^T over the 8 latent chunks
+          for (int k = 0; k < kChunks; ++k) {
+            const int slot = (int)(c_it % NS);
+            if (!mbar_wait(smem_u32(&ms.full[slot]), (c_it / NS) & 1, a.wait_limit)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t abase = sb + C::C_OFF + slot * kSlotBytes;
+            const uint32_t bbase = sb + C::Q_OFF + k * R * 128;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tS, smem_desc(abase + kk * 32, 16, 1024), smem_desc(bbase + kk * 32, 16, 1024), idS,
+                       (k | kk) != 0);
+            ++c_it;
+          }
+          if (!ok) break;
+          const int ks = (int)(k_it % NKR);
+          if (!mbar_wait(smem_u32(&ms.krfull[ks]), (k_it / NKR) & 1, a.wait_limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t krbase = sb + C::KR_OFF + ks * kSlotBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tSR, smem_desc(krbase + kk * 32, 16, 1024), smem_desc(sb + C::QR_OFF + kk * 32, 16, 1024),
+                     idS, kk != 0);
+          mma_commit(smem_u32(&ms.s_full));
+          if (i == ntiles - 1) mma_commit(smem_u32(&ms.q_empty));
+          // O^T += C^T . P^T, once the softmax has written P^T into the RoPE-key slot
+          if (i == 0 && !mbar_wait(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&ms.p_full), tile_n & 1, a.wait_limit)) { ok = false; break; }
+          tc_fence_after();
+          const int nkk = np * 4;   // 16-token K steps that hold real pages
+          for (int m = 0; m < 4; ++m) {
+            const int s0 = (int)((c_first + 2 * m) % NS);
+            const uint32_t abase = sb + C::C_OFF + s0 * kSlotBytes;
+            for (int kk = 0; kk < nkk; ++kk) {
+              const uint64_t ad = smem_desc(abase + kk * 2048, kSlotBytes, 1024);
+              const uint64_t bd = smem_desc(krbase + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
+              mma_bf16(tmem + m * R, ad, bd, idPV, (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(smem_u32(&ms.empty[s0]));
+            mma_commit(smem_u32(&ms.empty[s0 + 1]));
+          }
+          mma_commit(smem_u32(&ms.krempty[ks]));
+          ++k_it;
+          ++tile_n;
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&ms.o_full));
+        ++n_item;
+      }
+      if (!ok) {
+        record_status(a.status, QKN_ERR_TIMEOUT);
+        ms.abort_flag = 1;
+      }
+      // every MMA issued so far must finish before the tensor memory is freed
+      mma_commit(smem_u32(&ms.drain));
+      mbar_wait(smem_u32(&ms.drain), 0, kDrainLimit);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = threadIdx.x;                         // token row / TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const int ng = a.heads / G;
+    int64_t c_it = 0, k_it = 0, tile_n = 0;
+    int n_item = 0;
+    bool ok = true;
+    while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+      if (t < R) {
+        const int rho = it.ht * R + t;
+        const bool valid = rho < qrows;
+        const int j = valid ? rho / a.heads : 0;
+        const int h = valid ? rho - j * a.heads : 0;
+        ms.aq2[t] = valid ? a.a_q[(int64_t)it.b * qrows + rho] * kLog2e : 0.f;
+        ms.grp[t] = h / ng;
+        ms.qlim[t] = valid ? it.L - a.s_q + j : -1;
+        ms.mu[t] = -INFINITY;
+      }
+      named_bar_sync(1, kSoftThreads);
+      float lpart[R];
+#pragma unroll
+      for (int c = 0; c < R; ++c) lpart[c] = 0.f;
+      const int ntiles = (it.p1 - it.p0 + 1) / 2;
+      for (int i = 0; i < ntiles; ++i) {
+        const int np = min(2, it.p1 - (it.p0 + 2 * i));
+        const int tok0 = (it.p0 + 2 * i) * 64;
+        const int nvalid = min(np * 64, it.L - tok0);
+        const int ks = (int)(k_it % NKR);
+        bool got = true;
+        if (t == 0) got = mbar_wait(smem_u32(&ms.s_full), tile_n & 1, a.wait_limit);
+        if (!group_all(got)) { ok = false; break; }
+        tc_fence_after();
+        float ak0 = 1.f;
+        const float* akrow = reinterpret_cast<const float*>(smem + C::AK_OFF + ks * kAkSlotBytes) + t * G;
+        if (!AK_ONE) {
+          // the RoPE-key barrier also covers the a_k rows; it completed before S did
+          mbar_wait(smem_u32(&ms.krfull[ks]), (k_it / NKR) & 1, kDrainLimit);
+          ak0 = akrow[0];
+        }
+        const bool row_ok = t < nvalid;
+        const int tpos = tok0 + t;
+        // logit of column c for this token row, in log2 units; -inf when masked
+        auto logit = [&](int c, uint32_t sc, uint32_t sr) {
+          float akc = ak0;
+          if (!AK_ONE && G > 1) akc = akrow[ms.grp[c]];
+          const float v = ms.aq2[c] * akc * __uint_as_float(sc) + kLog2e * __uint_as_float(sr);
+          return (row_ok && tpos <= ms.qlim[c]) ? v : -INFINITY;
+        };
+        // pass 1: column maxima of this tile
+        {
+          float v[R];
+#pragma unroll
+          for (int c0 = 0; c0 < R; c0 += 16) {
+            uint32_t sc[16], sr[16];
+            tmem_ld16(tl + 4 * R + c0, sc);
+            tmem_ld16(tl + 5 * R + c0, sr);
+            tmem_wait_ld(sc, sr);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[c0 + e] = logit(c0 + e, sc[e], sr[e]);
+          }
+          warp_col_reduce<R, true>(v, lane);
+          store_reduced<R>(ms.red[warp], v, lane);
+        }
+        named_bar_sync(1, kSoftThreads);
+        bool mine = false;
+        if (t < R) {
+          const float mt = fmaxf(fmaxf(ms.red[0][t], ms.red[1][t]), fmaxf(ms.red[2][t], ms.red[3][t]));
+          const float mo = ms.mu[t];
+          float cr = 1.f;
+          if (mt > mo + kRescaleLog2) {
+            cr = (mo == -INFINITY) ? 0.f : ex2(mo - mt);
+            ms.mu[t] = mt;
+            mine = true;
+          }
+          ms.corr[t] = cr;
+        }
+        const bool rescale = group_any(mine) && i > 0;
+        // pass 2: probabilities, running column sums, and P^T (K-major, 128-byte
+        // swizzle: row = query row c, element = token t) into the RoPE-key slot
+        uint8_t* pbase = smem + C::KR_OFF + ks * kSlotBytes + (t >> 6) * (R * 128);
+        const int within = t & 63;
+#pragma unroll
+        for (int c0 = 0; c0 < R; c0 += 16) {
+          uint32_t sc[16], sr[16];
+          tmem_ld16(tl + 4 * R + c0, sc);
+          tmem_ld16(tl + 5 * R + c0, sr);
+          tmem_wait_ld(sc, sr);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = c0 + e;
+            const float xc = logit(c, sc[e], sr[e]);
+            const float p = (xc == -INFINITY) ? 0.f : ex2(xc - ms.mu[c]);
+            lpart[c] = lpart[c] * ms.corr[c] + p;
+            const int chunk = (within >> 3) ^ (c & 7);
+            *reinterpret_cast<__nv_bfloat16*>(pbase + c * 128 + (chunk << 4) + ((within & 7) << 1)) =
+                __float2bfloat16_rn(p);
+          }
+        }
+        // rows of real pages past the context: zero them so that 0 * garbage cannot reach O
+        if (!row_ok && t < np * 64) {
+#pragma unroll
+          for (int k = 0; k < kChunks; ++k) {
+            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + ((c_it + k) % NS) * kSlotBytes + t * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) rowp[q] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        if (rescale) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+#pragma unroll
+            for (int c0 = 0; c0 < R; c0 += 16) {
+              uint32_t ov[16];
+              tmem_ld16(tl + m * R + c0, ov);
+              tmem_wait_ld(ov);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[c0 + e]);
+              tmem_st16(tl + m * R + c0, ov);
+              tmem_wait_st();
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ms.p_full));
+        c_it += kChunks;
+        ++k_it;
+        ++tile_n;
+      }
+      if (!ok) break;
+      // ---------------- epilogue: O / l and lse for this item
+      bool got = true;
+      if (t == 0) got = mbar_wait(smem_u32(&ms.o_full), n_item & 1, a.wait_limit);
+      if (!group_all(got)) { ok = false; break; }
+      tc_fence_after();
+      warp_col_reduce<R, false>(lpart, lane);
+      store_reduced<R>(ms.red[warp], lpart, lane);
+      named_bar_sync(1, kSoftThreads);
+      if (t < R) {
+        const float l = ms.red[0][t] + ms.red[1][t] + ms.red[2][t] + ms.red[3][t];
+        ms.linv[t] = l > 0.f ? 1.f / l : 0.f;
+        a.part_lse[(int64_t)it.slot * R + t] = l > 0.f ? (ms.mu[t] + log2f(l)) * kLn2 : -INFINITY;
+      }
+      named_bar_sync(1, kSoftThreads);
+      float* po = a.part_o + (int64_t)it.slot * R * kRkv;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+#pragma unroll
+        for (int c0 = 0; c0 < R; c0 += 16) {
+          uint32_t ov[16];
+          tmem_ld16(tl + m * R + c0, ov);
+          tmem_wait_ld(ov);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            po[(int64_t)(c0 + e) * kRkv + m * 128 + t] = __uint_as_float(ov[e]) * ms.linv[c0 + e];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ms.o_empty));
+      ++n_item;
+    }
+    if (!ok && t == 0) {
+      record_status(a.status, QKN_ERR_TIMEOUT);
+      ms.abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 row-major tensor [rows, inner], 128-byte swizzled boxes [box_rows, box_inner].
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+              uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R, bool AK_ONE>
+cudaError_t launch_tc(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<R, AK_ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<R>::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  decode_tc_kernel<R, AK_ONE><<<a.ncta, kThreads, Cfg<R>::SMEM, st>>>(a, maps);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_tc_supported(int r, int d_rope, int rows, int groups) {
+  return r == kRkv && d_rope == kDrope && (rows == 16 || rows == 32 || rows == 64) && groups >= 1 &&
+         groups <= kMaxGroups;
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
+  if (!decode_tc_supported(a.r, a.d_rope, a.rows, a.groups)) return cudaErrorNotSupported;
+  TcMaps maps;
+  const uint64_t cache_rows = (uint64_t)a.num_blocks * 64;
+  const uint64_t q_rows = (uint64_t)a.batch * a.s_q * a.heads;
+  if (!make_map(&maps.latent, a.latent, kRkv, cache_rows, 64, 64) ||
+      !make_map(&maps.krope, a.k_rope, kDrope, cache_rows, 64, 64) ||
+      !make_map(&maps.qt, a.q_tilde, kRkv, q_rows, 64, a.rows) ||
+      !make_map(&maps.qr, a.q_rope_hat, kDrope, q_rows, 64, a.rows))
+    return cudaErrorInvalidValue;
+  switch (a.rows * 2 + (a.ak_one ? 1 : 0)) {
+    case 32: return launch_tc<16, false>(a, maps, st);
+    case 33: return launch_tc<16, true>(a, maps, st);
+    case 64: return launch_tc<32, false>(a, maps, st);
+    case 65: return launch_tc<32, true>(a, maps, st);
+    case 128: return launch_tc<64, false>(a, maps, st);
+    case 129: return launch_tc<64, true>(a, maps, st);
+  }
+  return cudaErrorNotSupported;
+}
+
+}  // namespace qkn

@@ -1,0 +1,82 @@
+// Host-side launch interfaces between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qkn {
+
+struct AppendArgs {
+  void* latent;            // cache pool
+  void* k_rope;
+  float* a_k;
+  const void* c_new;       // [n_tok, r]
+  const void* k_rope_raw;  // [n_tok, d_rope]
+  const int32_t* slot;
+  const int32_t* pos;
+  const float* w_k;        // [groups, r, width]
+  const float* gamma_kr;   // [d_rope]
+  int32_t n_tok, r, d_rope, groups, width;   // width = n_g * d_h
+  float eps, rope_theta;
+};
+
+struct AbsorbArgs {
+  const void* q;           // [n_q, H, d_h]
+  const void* q_rope;      // [n_q, H, d_rope]
+  const int32_t* pos;      // [n_q]
+  const float* w_k;        // [groups, r, n_g * d_h]
+  const float* gamma_q;    // [H, d_h]
+  const float* gamma_k;    // [H, d_h]
+  const float* gamma_qr;   // [H, d_rope]
+  void* q_tilde;           // [n_q, H, r]
+  float* a_q;              // [n_q, H]
+  void* q_rope_hat;        // [n_q, H, d_rope]
+  int32_t n_q, heads, groups, r, d_h, d_rope;
+  float eps, softmax_scale, rope_theta;
+};
+
+struct DecodeArgs {
+  const void* latent;        // [num_blocks, 64, r]
+  const void* k_rope;        // [num_blocks, 64, d_rope]
+  const float* a_k;          // [num_blocks, 64, groups]
+  int32_t num_blocks;
+  const void* q_tilde;       // [batch*s_q, H, r]
+  const float* a_q;          // [batch*s_q, H]
+  const void* q_rope_hat;    // [batch*s_q, H, d_rope]
+  const int32_t* block_table;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  int32_t batch, s_q, heads, groups, r, d_rope;
+  int32_t ak_one;            // 1: plain MLA (a_k treated as 1)
+  int32_t rows;              // query rows per tile (R)
+  int32_t ht_count;          // tiles per sequence = ceil(s_q*H / R)
+  int32_t ncta;
+  float* part_o;             // [slots, R, r] fp32
+  float* part_lse;           // [slots, R] fp32
+  int32_t* status;           // workspace status word
+  int64_t wait_limit;        // bounded-wait cycles (tcgen05 kernel)
+};
+
+struct CombineArgs {
+  const int32_t* seq_lens;
+  int32_t batch, s_q, heads, r, rows, ht_count, ncta, max_blocks;
+  const float* part_o;
+  const float* part_lse;
+  void* out;                 // [batch, s_q, H, r]
+  float* lse;                // [batch, s_q, H]
+  int32_t* status;           // workspace status word
+};
+
+cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_absorb(const AbsorbArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_decode_simt(const DecodeArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st);
+
+// tcgen05 decode (bf16 only).  Returns cudaErrorNotSupported for dims it
+// cannot take.
+bool decode_tc_supported(int r, int d_rope, int rows, int groups);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
+
+constexpr int kSimtRows = 8;   // query rows per CTA of the CUDA-core decode
+
+}  // namespace qkn

@@ -1,0 +1,111 @@
+"""Device-resident decode state on top of the C ABI.
+
+A ``DecodeSession`` owns a paged cache, the key up-projection and norm
+weights, the absorbed queries and a decode workspace, and forwards to
+``qkn_append``, ``qkn_absorb_query`` and ``qkn_decode``.  It moves host
+arrays to the device and nothing else: all arithmetic runs in libqkn.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, decode, decode_workspace_size,
+               read_device_status, workspace_init)
+
+
+def to_device(x, dtype: torch.dtype, device) -> torch.Tensor:
+    if isinstance(x, torch.Tensor):
+        return x.to(device=device, dtype=dtype).contiguous()
+    return torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dtype).contiguous()
+
+
+class DecodeSession:
+    def __init__(self, dims: Dims, num_blocks: int, device="cuda"):
+        self.dims = dims
+        self.device = torch.device(device)
+        self.cache = Cache(dims, num_blocks, device=self.device)
+        self.w_k = self.gamma_q = self.gamma_k = self.gamma_qr = self.gamma_kr = None
+        self.q_tilde = self.a_q = self.q_rope_hat = None
+        self.workspace: Optional[torch.Tensor] = None
+
+    # ------------------------------------------------------------ weights
+    def load_weights(self, w_k, gamma_q, gamma_k, gamma_qr, gamma_kr) -> None:
+        f32, dev = torch.float32, self.device
+        self.w_k = to_device(w_k, f32, dev)
+        self.gamma_q = to_device(gamma_q, f32, dev)
+        self.gamma_k = to_device(gamma_k, f32, dev)
+        self.gamma_qr = to_device(gamma_qr, f32, dev)
+        self.gamma_kr = to_device(gamma_kr, f32, dev)
+
+    # ------------------------------------------------------------ cache
+    def append(self, c, k_rope_raw, slot, pos, chunk: int = 1 << 16) -> None:
+        """Append tokens (host or device arrays) in chunks of ``chunk`` tokens."""
+        dt, dev = self.dims.torch_dtype, self.device
+        n = int(c.shape[0])
+        for t0 in range(0, n, chunk):
+            sl = slice(t0, min(n, t0 + chunk))
+            append(self.dims, self.cache, to_device(c[sl], dt, dev), to_device(k_rope_raw[sl], dt, dev),
+                   to_device(slot[sl], torch.int32, dev), to_device(pos[sl], torch.int32, dev),
+                   self.w_k, self.gamma_kr)
+
+    # ------------------------------------------------------------ queries
+    def absorb(self, q, q_rope, pos) -> None:
+        """q [n_q, H, d_h], q_rope [n_q, H, d_R], pos [n_q] -> q~, a_q, q^R^ on the device."""
+        d, dt, dev = self.dims, self.dims.torch_dtype, self.device
+        q = to_device(q, dt, dev)
+        q_rope = to_device(q_rope, dt, dev)
+        n_q = q.shape[0]
+        self.q_tilde = torch.empty((n_q, d.num_heads, d.r_kv), dtype=dt, device=dev)
+        self.a_q = torch.empty((n_q, d.num_heads), dtype=torch.float32, device=dev)
+        self.q_rope_hat = torch.empty((n_q, d.num_heads, d.d_rope), dtype=dt, device=dev)
+        absorb_query(d, q, q_rope, to_device(pos, torch.int32, dev), self.w_k, self.gamma_q, self.gamma_k,
+                     self.gamma_qr, self.q_tilde, self.a_q, self.q_rope_hat)
+
+    # ------------------------------------------------------------ decode
+    def ensure_workspace(self, batch: int, s_q: int) -> torch.Tensor:
+        need = decode_workspace_size(self.dims, batch, s_q)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            workspace_init(self.workspace)
+        return self.workspace
+
+    def decode(self, block_table, seq_lens, s_q: int, out=None, lse=None, ak_mode: int = AK_CACHE,
+               kernel: int = KERNEL_AUTO, max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0):
+        d, dev = self.dims, self.device
+        bt = to_device(block_table, torch.int32, dev)
+        sl = to_device(seq_lens, torch.int32, dev)
+        batch = bt.shape[0]
+        ws = self.ensure_workspace(batch, s_q)
+        if out is None:
+            out = torch.empty((batch, s_q, d.num_heads, d.r_kv), dtype=d.torch_dtype, device=dev)
+        if lse is None:
+            lse = torch.empty((batch, s_q, d.num_heads), dtype=torch.float32, device=dev)
+        decode(d, self.cache, self.q_tilde, self.a_q, self.q_rope_hat, bt, sl, s_q, ws, out, lse,
+               ak_mode=ak_mode, kernel=kernel, max_ctas=max_ctas, head_tile=head_tile, wait_limit=wait_limit)
+        return out, lse
+
+    def device_status(self) -> int:
+        return read_device_status(self.workspace)
+
+    def clear_status(self) -> None:
+        workspace_init(self.workspace)
+
+
+def session_from_inputs(inp, device="cuda", dtype=None) -> DecodeSession:
+    """Build a session from a seeded problem (an object with the fields of qkn_inputs.Inputs):
+    weights loaded, every context token appended, queries absorbed."""
+    wl = inp.wl
+    dt = dtype if dtype is not None else (1 if wl.dtype == "bf16" else 0)
+    dims = Dims(num_heads=wl.heads, num_groups=wl.groups, r_kv=wl.r_kv, d_h=wl.d_h, d_rope=wl.d_rope,
+                eps=wl.eps, softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, dtype=dt,
+                block_size=wl.block_size)
+    s = DecodeSession(dims, inp.num_blocks, device=device)
+    s.load_weights(inp.w_k, inp.gamma_q, inp.gamma_k, inp.gamma_qr, inp.gamma_kr)
+    s.append(inp.c, inp.k_rope, inp.token_slots(), inp.token_positions())
+    B, s_q = wl.batch, wl.s_q
+    s.absorb(inp.q.reshape(B * s_q, wl.heads, wl.d_h), inp.q_rope.reshape(B * s_q, wl.heads, wl.d_rope),
+             inp.query_positions().reshape(-1))
+    return s

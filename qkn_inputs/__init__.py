@@ -180,7 +180,8 @@ def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
     nblk = (lens.astype(np.int64) + bs - 1) // bs
     pool = int(nblk.sum())
     max_blocks = int(nblk.max())
-    perm = rng.permutation(pool).astype(np.int32) if wl.paged else np.arange(pool, dtype=np.int32)
+    drawn_perm = rng.permutation(pool).astype(np.int32)      # drawn either way: keeps later draws aligned
+    perm = drawn_perm if wl.paged else np.arange(pool, dtype=np.int32)
     table = np.zeros((B, max_blocks), dtype=np.int32)
     boff = np.concatenate([[0], np.cumsum(nblk)])
     for b in range(B):

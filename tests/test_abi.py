@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every symbol include/qkn.h declares, and
+rejects bad arguments on the host before touching a GPU (CPU only)."""
+import ctypes
+import re
+import os
+
+import pytest
+
+import qk_normed_latent_qkn_b200 as qkn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "qkn.h")).read()
+    return sorted(set(re.findall(r"QKN_EXPORT\s+[\w\s\*]+?\b(qkn_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = qkn.raw_library()
+    names = declared_symbols()
+    assert names, "no declarations found"
+    assert sorted(qkn.EXPORTED) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings():
+    assert qkn.version() == 1
+    for s in range(6):
+        assert qkn.status_string(s)
+    assert qkn.status_string(0) == "ok"
+
+
+DIMS = qkn.Dims(num_heads=16, num_groups=1, r_kv=512, d_h=128, d_rope=64)
+
+
+def _ws(dims, batch=4, s_q=1, sms=148):
+    return qkn.decode_workspace_size(dims, batch, s_q, num_sms=sms)
+
+
+def test_workspace_size_host_only():
+    small = _ws(DIMS, 1)
+    big = _ws(DIMS, 64)
+    assert big > small > 256
+    # enough room for one partial (rows x r fp32) per (segment, CTA) slot
+    assert _ws(DIMS, 16, sms=148) >= (16 + 148) * 16 * 512 * 4
+
+
+@pytest.mark.parametrize("bad", [
+    dict(num_heads=0), dict(num_groups=3), dict(r_kv=12), dict(d_rope=7), dict(d_rope=256),
+    dict(block_size=32), dict(eps=-1.0), dict(softmax_scale=0.0), dict(dtype=7),
+])
+def test_bad_dims_rejected(bad):
+    import dataclasses
+    d = dataclasses.replace(DIMS, **bad)
+    with pytest.raises(qkn.QknError) as e:
+        _ws(d)
+    assert e.value.status == qkn.ERR_INVALID_ARG
+
+
+def test_decode_rejects_null_pointers_before_any_launch():
+    lib = qkn.raw_library()
+    dims = DIMS.c()
+    cache = qkn._Cache(None, None, None, 0)
+    rc = lib.qkn_decode(ctypes.byref(dims), ctypes.byref(cache), 0, None, None, None, None, 1, None, 1, 1,
+                        None, 0, None, None, None, None)
+    assert rc == qkn.ERR_INVALID_ARG
+    # a valid-looking cache but missing queries
+    cache = qkn._Cache(0x1000, 0x2000, 0x3000, 4)
+    rc = lib.qkn_decode(ctypes.byref(dims), ctypes.byref(cache), 0, None, None, None, None, 1, None, 1, 1,
+                        None, 0, None, None, None, None)
+    assert rc == qkn.ERR_INVALID_ARG
+    # misaligned cache base
+    cache = qkn._Cache(0x1001, 0x2000, 0x3000, 4)
+    rc = lib.qkn_decode(ctypes.byref(dims), ctypes.byref(cache), 0, 0x100, 0x100, 0x100, 0x100, 1, 0x100, 1,
+                        1, 0x100, 1 << 20, 0x100, 0x100, None, None)
+    assert rc == qkn.ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_options():
+    lib = qkn.raw_library()
+    dims = DIMS.c()
+    cache = qkn._Cache(0x1000, 0x2000, 0x3000, 4)
+    opts = qkn._Opts(qkn.KERNEL_AUTO, 0, 48, 0)     # head tile must be 16, 32 or 64
+    rc = lib.qkn_decode(ctypes.byref(dims), ctypes.byref(cache), 0, 0x100, 0x100, 0x100, 0x100, 1, 0x100, 1,
+                        1, 0x100, 1 << 30, 0x100, 0x100, ctypes.byref(opts), None)
+    assert rc == qkn.ERR_INVALID_ARG
+    rc = lib.qkn_decode(ctypes.byref(dims), ctypes.byref(cache), 5, 0x100, 0x100, 0x100, 0x100, 1, 0x100, 1,
+                        1, 0x100, 1 << 30, 0x100, 0x100, None, None)
+    assert rc == qkn.ERR_INVALID_ARG
+
+
+def test_append_and_absorb_reject_bad_arguments():
+    lib = qkn.raw_library()
+    dims = DIMS.c()
+    cache = qkn._Cache(0x1000, 0x2000, 0x3000, 4)
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 0, None, None,
+                          None) == qkn.OK          # n_tok == 0 is a no-op
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 3, None, None,
+                          None) == qkn.ERR_INVALID_ARG
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), 0x100, 0x100, 0x100, 0x100, -1, 0x100,
+                          0x100, None) == qkn.ERR_INVALID_ARG
+    assert lib.qkn_absorb_query(ctypes.byref(dims), None, None, None, 0, None, None, None, None, None, None,
+                                None, None) == qkn.OK
+    assert lib.qkn_absorb_query(ctypes.byref(dims), None, None, None, 2, None, None, None, None, None, None,
+                                None, None) == qkn.ERR_INVALID_ARG
+
+
+def test_kernel_choice_is_host_logic():
+    f32 = qkn.Dims(num_heads=4, num_groups=1, r_kv=64, d_h=32, d_rope=16, dtype=qkn.F32)
+    assert qkn.decode_kernel_for(f32, 1) == qkn.KERNEL_SIMT
+    assert qkn.decode_kernel_for(f32, 1, kernel=qkn.KERNEL_TCGEN05) == -1
