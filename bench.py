@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Decode benchmark for QK-Normed MLA on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole decode hot path over one batch: append the
+step's new tokens (latent, RoPE key, a_k), absorb the step's queries, split-KV
+decode and combine.  Inputs are seeded synthetic tensors shaped like the
+named workload (default: small_mla_bf16, 16 sequences x 4096 tokens, 16 heads,
+r = 512, d_R = 64, bf16).  Each rank runs its own replica (its own sequences;
+weak scaling, no collective on the data path); the step time is the max over
+ranks of CUDA-event time.  Every step is a CUDA graph replay; consecutive
+steps read different copies of the cache so that the working set of the timed
+steps is larger than L2.
+
+One JSON line on rank 0 carries the whole-job decode tokens/s, the decode
+kernel's roofline fraction, the overhead against the same kernel with a_k
+fixed to 1 (plain MLA), an end-to-end figure through the public API with
+host buffers, SM clocks sampled while the GPU was under this load, and the
+fp64 oracle's throughput on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s and us/step at 1 B200; % of HBM/tensor roofline; overhead vs MLA"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="small_mla_bf16")
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--soak-seconds", type=float, default=1.0, help="load window around the timed steps for clocks")
+    p.add_argument("--overhead-rounds", type=int, default=5)
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if a.steps < 1:
+        p.error("--steps must be >= 1")
+    return a
+
+
+# ----------------------------------------------------------------- distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_workload(name: str, rank: int):
+    """The workload replica of one rank: same shapes, its own sequences (seed offset by rank)."""
+    from qkn_inputs import WORKLOADS
+    wl = WORKLOADS[name]
+    return wl.with_(seed=wl.seed + rank)
+
+
+def job_throughput(tokens_per_rank: int, world: int, local_ms_total: float, steps: int, device=None):
+    """Whole-job tokens/s and ms per step: every rank's tokens over the slowest rank's time."""
+    step_ms = reduce_max(local_ms_total, device) / steps
+    return world * tokens_per_rank / (step_ms * 1e-3), step_ms
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- CUDA events that survive capture
+class Events:
+    """Raw cudaEvent_t handles recorded with cudaEventRecordExternal, so that a
+    record inside stream capture becomes an event node of the graph."""
+
+    def __init__(self):
+        import torch
+        lib = None
+        for cand in ("libcudart.so.12", "libcudart.so"):
+            try:
+                lib = ctypes.CDLL(cand)
+                break
+            except OSError:
+                continue
+        if lib is None:
+            base = os.path.join(os.path.dirname(os.path.dirname(torch.__file__)), "nvidia", "cuda_runtime", "lib")
+            lib = ctypes.CDLL(os.path.join(base, "libcudart.so.12"))
+        self.lib = lib
+        lib.cudaEventCreate.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+        lib.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        lib.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
+        lib.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+
+    def create(self) -> int:
+        h = ctypes.c_void_p()
+        assert self.lib.cudaEventCreate(ctypes.byref(h)) == 0
+        return h.value
+
+    def record(self, ev: int, stream: int) -> None:
+        assert self.lib.cudaEventRecordWithFlags(ctypes.c_void_p(ev), ctypes.c_void_p(stream), 1) == 0
+
+    def ms(self, a: int, b: int) -> float:
+        out = ctypes.c_float()
+        rc = self.lib.cudaEventElapsedTime(ctypes.byref(out), ctypes.c_void_p(a), ctypes.c_void_p(b))
+        assert rc == 0, rc
+        return float(out.value)
+
+
+# ----------------------------------------------------------------- clocks
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the GPU is loaded."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.period = [], set(), period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            self.h = None
+            if uuid:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(h)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                        self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - no NVML
+            self.nvml, self.error = None, str(e)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for b, name in REASON_BITS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+
+    def summary(self, window_s: float):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "window_s": round(window_s, 2), "source": "nvml"}
+
+
+# ----------------------------------------------------------------- oracle CPU baseline
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_throughput(inp, budget_s: float, max_seqs=None):
+    """Decode tokens/s of the fp64 oracle: whole sequences of the workload until the budget is spent."""
+    import oracle
+    wl = inp.wl
+    done, t0 = 0, time.perf_counter()
+    order = list(range(wl.batch)) if max_seqs is None else list(range(min(wl.batch, max_seqs)))
+    for b in order:
+        oracle.decode_sequence(inp, b)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return done * wl.s_q / el, done, el
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import torch
+    import qk_normed_latent_qkn_b200 as qkn
+    from qk_normed_latent_qkn_b200.roofline import decode_step_cost
+    from qk_normed_latent_qkn_b200.session import DecodeSession, session_from_inputs
+    from qkn_inputs import WORKLOADS, make_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = rank_workload(args.workload, rank)
+    kernel = {"auto": qkn.KERNEL_AUTO, "simt": qkn.KERNEL_SIMT, "tcgen05": qkn.KERNEL_TCGEN05}[args.kernel]
+    inp = make_inputs(wl)
+    B, s_q, H = wl.batch, wl.s_q, wl.heads
+    n_q = B * s_q
+
+    # per-step inputs: the step's new tokens (the last s_q of every sequence) and its queries
+    last = np.concatenate([np.arange(inp.tok_off[b + 1] - s_q, inp.tok_off[b + 1]) for b in range(B)])
+    slots, poss = inp.token_slots()[last], inp.token_positions()[last]
+    host = {
+        "c": inp.c[last], "kr": inp.k_rope[last], "slot": slots, "pos": poss,
+        "q": inp.q.reshape(n_q, H, wl.d_h), "qr": inp.q_rope.reshape(n_q, H, wl.d_rope),
+        "qpos": inp.query_positions().reshape(-1), "bt": inp.block_table, "sl": inp.seq_lens,
+    }
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    types = {"c": dt, "kr": dt, "slot": torch.int32, "pos": torch.int32, "q": dt, "qr": dt,
+             "qpos": torch.int32, "bt": torch.int32, "sl": torch.int32}
+
+    base = session_from_inputs(inp, device=device)
+    cache_bytes = sum(t.numel() * t.element_size() for t in (base.cache.latent, base.cache.k_rope, base.cache.a_k))
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    n_copies = max(1, min(16, math.ceil(3 * l2 / cache_bytes))) if cache_bytes < 2 * l2 else 1
+    sessions = [base]
+    for _ in range(n_copies - 1):
+        s = DecodeSession(base.dims, inp.num_blocks, device=device)
+        s.cache.latent.copy_(base.cache.latent)
+        s.cache.k_rope.copy_(base.cache.k_rope)
+        s.cache.a_k.copy_(base.cache.a_k)
+        s.load_weights(base.w_k, base.gamma_q, base.gamma_k, base.gamma_qr, base.gamma_kr)
+        sessions.append(s)
+    dev_in = [{k: torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=types[k]) for k, v in
+               host.items()} for _ in sessions]
+    outs = [(torch.empty((B, s_q, H, wl.r_kv), dtype=dt, device=device),
+             torch.empty((B, s_q, H), dtype=torch.float32, device=device)) for _ in sessions]
+
+    def step(i, split_event=None, ak_mode=qkn.AK_CACHE):
+        s, d, (o, l) = sessions[i], dev_in[i], outs[i]
+        s.append(d["c"], d["kr"], d["slot"], d["pos"])
+        s.absorb(d["q"], d["qr"], d["qpos"])
+        s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event)
+
+    def decode_only(i, split_event=None, ak_mode=qkn.AK_CACHE):
+        s, d, (o, l) = sessions[i], dev_in[i], outs[i]
+        s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event)
+
+    # eager warm-up: first-call attributes, workspaces, absorbed queries
+    for i in range(len(sessions)):
+        step(i)
+        step(i, ak_mode=qkn.AK_ONE)
+    torch.cuda.synchronize(device)
+    status = [s.device_status() for s in sessions]
+    assert all(v == qkn.OK for v in status), f"device status {status}"
+    kernel_used = qkn.decode_kernel_for(base.dims, s_q, kernel=kernel)
+
+    ev = Events()
+    stream = torch.cuda.Stream(device=device)
+    total = args.warmup + args.steps
+    graphs, marks = [], []
+    with torch.cuda.stream(stream):
+        for k in range(total):
+            i = k % n_copies
+            e = [ev.create() for _ in range(4)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                sid = stream.cuda_stream
+                ev.record(e[0], sid)
+                sessions[i].append(dev_in[i]["c"], dev_in[i]["kr"], dev_in[i]["slot"], dev_in[i]["pos"])
+                sessions[i].absorb(dev_in[i]["q"], dev_in[i]["qr"], dev_in[i]["qpos"])
+                ev.record(e[1], sid)
+                decode_only(i, split_event=e[2])
+                ev.record(e[3], sid)
+            graphs.append(g)
+            marks.append(e)
+        # decode-only graphs, QK-Normed and plain MLA, for the overhead figure
+        over = {}
+        for mode in (qkn.AK_CACHE, qkn.AK_ONE):
+            lst = []
+            for i in range(n_copies):
+                e = [ev.create() for _ in range(2)]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                    ev.record(e[0], stream.cuda_stream)
+                    decode_only(i, split_event=e[1], ak_mode=mode)
+                lst.append((g, e))
+            over[mode] = lst
+    torch.cuda.synchronize(device)
+
+    soak_graphs = graphs[:n_copies] if len(graphs) >= n_copies else graphs
+
+    def soak(seconds):
+        t_end = time.perf_counter() + seconds
+        with torch.cuda.stream(stream):
+            while time.perf_counter() < t_end:
+                for g in soak_graphs:
+                    g.replay()
+                stream.synchronize()
+
+    t_start_ev = torch.cuda.Event(enable_timing=True)
+    t_end_ev = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    w0 = time.perf_counter()
+    with sampler:
+        soak(args.soak_seconds)
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup):
+                graphs[k].replay()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        with torch.cuda.stream(stream):
+            t_start_ev.record(stream)
+            for k in range(args.warmup, total):
+                graphs[k].replay()
+            t_end_ev.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        soak(args.soak_seconds)
+    window = time.perf_counter() - w0
+    local_ms = t_start_ev.elapsed_time(t_end_ev)
+    value, step_ms = job_throughput(B * s_q, world, local_ms, args.steps, device)
+
+    split_ms = [ev.ms(marks[k][1], marks[k][2]) for k in range(args.warmup, total)]
+    combine_ms = [ev.ms(marks[k][2], marks[k][3]) for k in range(args.warmup, total)]
+    prep_ms = [ev.ms(marks[k][0], marks[k][1]) for k in range(args.warmup, total)]
+
+    # overhead vs plain MLA: interleaved rounds of decode-only graphs
+    per_mode = {qkn.AK_CACHE: [], qkn.AK_ONE: []}
+    with torch.cuda.stream(stream):
+        for _ in range(args.overhead_rounds):
+            for mode in (qkn.AK_CACHE, qkn.AK_ONE):
+                for g, _e in over[mode]:
+                    g.replay()
+                stream.synchronize()
+                per_mode[mode] += [ev.ms(e[0], e[1]) for _g, e in over[mode]]
+    t_qkn = statistics.median(per_mode[qkn.AK_CACHE])
+    t_mla = statistics.median(per_mode[qkn.AK_ONE])
+
+    # end to end through the public API, host (pinned) buffers in and out every step
+    pinned_in = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dtype=types[k]).pin_memory() for k, v in host.items()}
+    pinned_out = (torch.empty((B, s_q, H, wl.r_kv), dtype=dt).pin_memory(),
+                  torch.empty((B, s_q, H), dtype=torch.float32).pin_memory())
+    h2d = sum(t.numel() * t.element_size() for t in pinned_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in pinned_out)
+
+    def e2e_step(k):
+        i = k % n_copies
+        d = dev_in[i]
+        for key, t in pinned_in.items():
+            d[key].copy_(t, non_blocking=True)
+        step(i)
+        pinned_out[0].copy_(outs[i][0], non_blocking=True)
+        pinned_out[1].copy_(outs[i][1], non_blocking=True)
+        torch.cuda.current_stream(device).synchronize()
+
+    for k in range(args.warmup):
+        e2e_step(k)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(args.steps):
+        e2e_step(k)
+    e1.record()
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device) / args.steps
+    assert all(s.device_status() == qkn.OK for s in sessions)
+
+    # roofline of the dominant kernel (the split-KV decode)
+    cost = decode_step_cost(inp.seq_lens, s_q, H, wl.groups, wl.r_kv, wl.d_rope,
+                            elem=2 if wl.dtype == "bf16" else 4)
+    peaks, peak_src = load_peaks()
+    split_avg = statistics.mean(split_ms)
+    achieved_gbs = cost.bytes / (split_avg * 1e-3) / 1e9
+    tflops = cost.flops / (split_avg * 1e-3) / 1e12
+    tokens = world * B * s_q
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tps, nseq, el = oracle_throughput(inp, args.cpu_seconds)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{nseq} of {B} sequences of the workload ({nseq * s_q} query tokens, "
+                             f"{int(inp.seq_lens[:nseq].sum())} cached tokens) in {el:.1f} s, fp64 numpy"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_gpu": B, "s_q": s_q, "heads": H, "groups": wl.groups,
+                       "r_kv": wl.r_kv, "d_h": wl.d_h, "d_rope": wl.d_rope,
+                       "context": list(wl.context) if isinstance(wl.context, tuple) else wl.context,
+                       "cached_tokens_per_gpu": int(inp.seq_lens.sum()), "paged": wl.paged,
+                       "kernel": {qkn.KERNEL_TCGEN05: "tcgen05", qkn.KERNEL_SIMT: "simt"}.get(kernel_used),
+                       "l2": f"{n_copies} rotating cache copies, {n_copies * cache_bytes / 2**20:.0f} MiB "
+                             f"(L2 {l2 / 2**20:.0f} MiB)", "step_launch": "CUDA graph per step",
+                       "parallelism": f"replicas x{world}"},
+            "breakdown_us": {"append_absorb": statistics.mean(prep_ms) * 1e3,
+                             "decode_split": split_avg * 1e3, "combine": statistics.mean(combine_ms) * 1e3},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes": cost.bytes, "peak_source": f"{peak_src} HBM copy bandwidth",
+                         "kernel": "decode split (tcgen05)" if kernel_used == qkn.KERNEL_TCGEN05 else "decode split",
+                         "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                    "frac": tflops / peaks["bf16_tflops"], "flops": cost.flops}},
+            "overhead_vs_mla": {"qkn_us": t_qkn * 1e3, "mla_us": t_mla * 1e3, "frac": t_qkn / t_mla - 1.0,
+                                "what": "decode split kernel, a_k cache vs a_k = 1, median of interleaved rounds"},
+            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "what": "DecodeSession append/absorb/decode, eager, pinned host in/out, sync per step"},
+            "gpu_launches": 7 * args.steps,
+            "clocks": sampler.summary(window),
+            "cpu_baseline": cpu,
+        }
+    return line
+
+
+# ----------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    from qkn_inputs import WORKLOADS, make_inputs
+    import oracle
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl)
+    # each step: one whole sequence of the workload through the explicit-key oracle
+    times = []
+    for k in range(args.warmup + args.steps):
+        b = k % wl.batch
+        t0 = time.perf_counter()
+        oracle.decode_sequence(inp, b)
+        if k >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_tok = statistics.mean(times) / wl.s_q
+    v = 1.0 / per_tok
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.heads},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one sequence of {wl.name} per step (explicit keys, fp64 numpy)"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -112,6 +112,8 @@ typedef struct {
   int32_t max_ctas;        /* cap on decode CTAs (split-KV width); 0 = one per SM */
   int32_t head_tile;       /* tcgen05: query rows per CTA (16, 32 or 64); 0 = automatic */
   int64_t wait_limit;      /* bounded-wait limit in clock cycles for the mbarrier waits; 0 = default (~2 s) */
+  void* split_event;       /* optional cudaEvent_t recorded between the split-KV kernel and the combine
+                              kernel (external record, so it also works inside stream capture) */
 } qkn_decode_opts;
 
 /* qkn_append — write n_tok new tokens into the cache.

@@ -262,6 +262,10 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   const bool bf16 = dims->dtype == QKN_BF16;
   cudaError_t e = kernel == QKN_KERNEL_TCGEN05 ? launch_decode_tc(a, cs) : launch_decode_simt(a, bf16, cs);
   if (e != cudaSuccess) return QKN_ERR_CUDA;
+  if (opts && opts->split_event &&
+      cudaEventRecordWithFlags(static_cast<cudaEvent_t>(opts->split_event), cs, cudaEventRecordExternal) !=
+          cudaSuccess)
+    return QKN_ERR_CUDA;
 
   CombineArgs c;
   c.seq_lens = seq_lens;

@@ -53,14 +53,16 @@ class DecodeSession:
 
     # ------------------------------------------------------------ queries
     def absorb(self, q, q_rope, pos) -> None:
-        """q [n_q, H, d_h], q_rope [n_q, H, d_R], pos [n_q] -> q~, a_q, q^R^ on the device."""
+        """q [n_q, H, d_h], q_rope [n_q, H, d_R], pos [n_q] -> q~, a_q, q^R^ on the device.
+        The output buffers are reused while the query count stays the same."""
         d, dt, dev = self.dims, self.dims.torch_dtype, self.device
         q = to_device(q, dt, dev)
         q_rope = to_device(q_rope, dt, dev)
         n_q = q.shape[0]
-        self.q_tilde = torch.empty((n_q, d.num_heads, d.r_kv), dtype=dt, device=dev)
-        self.a_q = torch.empty((n_q, d.num_heads), dtype=torch.float32, device=dev)
-        self.q_rope_hat = torch.empty((n_q, d.num_heads, d.d_rope), dtype=dt, device=dev)
+        if self.q_tilde is None or self.q_tilde.shape[0] != n_q:
+            self.q_tilde = torch.empty((n_q, d.num_heads, d.r_kv), dtype=dt, device=dev)
+            self.a_q = torch.empty((n_q, d.num_heads), dtype=torch.float32, device=dev)
+            self.q_rope_hat = torch.empty((n_q, d.num_heads, d.d_rope), dtype=dt, device=dev)
         absorb_query(d, q, q_rope, to_device(pos, torch.int32, dev), self.w_k, self.gamma_q, self.gamma_k,
                      self.gamma_qr, self.q_tilde, self.a_q, self.q_rope_hat)
 
@@ -73,7 +75,8 @@ class DecodeSession:
         return self.workspace
 
     def decode(self, block_table, seq_lens, s_q: int, out=None, lse=None, ak_mode: int = AK_CACHE,
-               kernel: int = KERNEL_AUTO, max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0):
+               kernel: int = KERNEL_AUTO, max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0,
+               split_event=None):
         d, dev = self.dims, self.device
         bt = to_device(block_table, torch.int32, dev)
         sl = to_device(seq_lens, torch.int32, dev)
@@ -84,7 +87,8 @@ class DecodeSession:
         if lse is None:
             lse = torch.empty((batch, s_q, d.num_heads), dtype=torch.float32, device=dev)
         decode(d, self.cache, self.q_tilde, self.a_q, self.q_rope_hat, bt, sl, s_q, ws, out, lse,
-               ak_mode=ak_mode, kernel=kernel, max_ctas=max_ctas, head_tile=head_tile, wait_limit=wait_limit)
+               ak_mode=ak_mode, kernel=kernel, max_ctas=max_ctas, head_tile=head_tile, wait_limit=wait_limit,
+               split_event=split_event)
         return out, lse
 
     def device_status(self) -> int:
