@@ -1,6 +1,9 @@
 """Build libqkn.so in-tree with nvcc for sm_100a.
 
-    python -m qk_normed_latent_qkn_b200.build [--force]
+    python qk_normed_latent_qkn_b200/build.py [--force] [-v]
+
+(run it as a file: importing the package loads libqkn.so, which is what this
+script produces)
 
 Each ``csrc/*.cu`` compiles to an object under ``_build/`` (git-ignored) and
 the objects link into ``qk_normed_latent_qkn_b200/libqkn.so`` with the CUDA
