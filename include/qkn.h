@@ -192,6 +192,38 @@ QKN_EXPORT qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, q
                       void* workspace, size_t ws_bytes, void* out, float* lse,
                       const qkn_decode_opts* opts, void* stream);
 
+/* Size of the scratch array that qkn_decode_noalloc uses in place of a
+ * caller-allocated workspace.  Every GPU that loads libqkn holds this much
+ * device memory for the scratch until the process exits. */
+#define QKN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* qkn_decode_noalloc — qkn_decode for callers that cannot allocate device
+ * memory (an operator inside another engine that only hands over input and
+ * output pointers, a serving loop whose pool already owns the whole GPU, a
+ * latency-critical loop that must not pay cudaMalloc's implicit
+ * synchronisation).  The paper has no counterpart: this is a deployment
+ * variant of the same decode step.
+ *   Arguments are those of qkn_decode without the workspace.  The split-KV
+ *   partial results go to a fixed QKN_NOALLOC_SCRATCH_BYTES array inside the
+ *   library instead; nothing is allocated and no allocating routine is called.
+ *   device_status: optional DEVICE pointer to one int32; the decode's status
+ *   word (a qkn_status) is copied there on `stream` after the decode.
+ *   Returns QKN_ERR_UNSUPPORTED, before enqueuing anything, when the problem
+ *   needs more scratch than QKN_NOALLOC_SCRATCH_BYTES (that is, when
+ *   qkn_decode_workspace_size for these dims, batch and s_q exceeds it).
+ *   The first call on a device looks up the array's device address on that
+ *   device (the calling thread's current device); make that first call before
+ *   any stream capture.  All calls share the one array: calls whose GPU work
+ *   overlaps (on different streams, or from different threads) race on it and
+ *   must be serialised by the caller.  The status word is cleared at the start
+ *   of every call. */
+QKN_EXPORT qkn_status qkn_decode_noalloc(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode,
+                      const void* q_tilde, const float* a_q, const void* q_rope_hat,
+                      const int32_t* block_table, int32_t max_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t s_q,
+                      void* out, float* lse, int32_t* device_status,
+                      const qkn_decode_opts* opts, void* stream);
+
 /* Synchronise `stream`, then read the workspace status word into *device_status
  * (a qkn_status value; QKN_OK if no kernel recorded an error).  The word is
  * sticky until qkn_workspace_init clears it. */

@@ -26,7 +26,8 @@ KERNEL_AUTO, KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1, 2
 
 EXPORTED = ["qkn_append", "qkn_absorb_query", "qkn_decode_workspace_size", "qkn_workspace_init",
             "qkn_decode", "qkn_read_device_status", "qkn_decode_kernel_for", "qkn_status_string",
-            "qkn_version"]
+            "qkn_version", "qkn_decode_noalloc"]
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class QknError(RuntimeError):
@@ -68,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "qkn_decode_kernel_for": (I32, [PD, I32, PO]),
         "qkn_status_string": (ctypes.c_char_p, [I32]),
         "qkn_version": (I32, []),
+        "qkn_decode_noalloc": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, P, P, PO, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -190,6 +192,19 @@ def decode(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_
                            _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens), batch, s_q,
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
                            ctypes.byref(opts), _stream(stream)), "qkn_decode")
+
+
+def decode_noalloc(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_lens, s_q: int, out, lse,
+                   device_status=None, ak_mode: int = AK_CACHE, kernel: int = KERNEL_AUTO, stream=None) -> None:
+    """qkn_decode_noalloc: the decode step without a workspace, for callers that cannot allocate
+    device memory; its scratch is a fixed array inside the library (see include/qkn.h)."""
+    batch = int(block_table.shape[0])
+    max_blocks = int(block_table.shape[1])
+    opts = _opts(kernel)
+    _check(_lib.qkn_decode_noalloc(ctypes.byref(dims.c()), ctypes.byref(cache.c()), ak_mode, _ptr(q_tilde),
+                                   _ptr(a_q), _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens),
+                                   batch, s_q, _ptr(out), _ptr(lse), _ptr(device_status), ctypes.byref(opts),
+                                   _stream(stream)), "qkn_decode_noalloc")
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
