@@ -1,6 +1,7 @@
 // The C ABI of libqkn (declared in include/qkn.h): host-side argument checks,
 // kernel selection, the decode workspace layout and kernel launches.  Every
 // entry point validates before it enqueues anything, and none allocates.
+#include <math.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -56,6 +57,13 @@ int sm_count(int* out) {
 }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// RoPE pair frequencies theta^(-2i/d_R) in fp64 (constants of the dims).
+RopeFreqs rope_freqs(const qkn_dims* d) {
+  RopeFreqs r;
+  for (int i = 0; i < 64; ++i) r.f[i] = i < d->d_rope / 2 ? pow((double)d->rope_theta, -2.0 * i / d->d_rope) : 0.0;
+  return r;
+}
 
 // Rows per tile for the tcgen05 kernel: the smallest supported tile that
 // covers the per-sequence query rows, capped at 64 (the accumulator of a
@@ -144,6 +152,7 @@ qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache, const void* 
   a.width = (dims->num_heads / dims->num_groups) * dims->d_h;
   a.eps = dims->eps;
   a.rope_theta = dims->rope_theta;
+  a.freq = rope_freqs(dims);
   cudaError_t e = launch_append(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
 }
@@ -158,7 +167,8 @@ qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_r
   if (n_q == 0) return QKN_OK;
   if (!q || !q_rope || !pos || !w_k || !gamma_q || !gamma_k || !gamma_qr || !q_tilde || !a_q || !q_rope_hat)
     return QKN_ERR_INVALID_ARG;
-  if (dims->d_h > 256) return QKN_ERR_UNSUPPORTED;
+  if (dims->d_h > 256 || dims->d_h % 4) return QKN_ERR_UNSUPPORTED;
+  if (!aligned(w_k, 16)) return QKN_ERR_INVALID_ARG;
   AbsorbArgs a;
   a.q = q;
   a.q_rope = q_rope;
@@ -179,6 +189,7 @@ qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_r
   a.eps = dims->eps;
   a.softmax_scale = dims->softmax_scale;
   a.rope_theta = dims->rope_theta;
+  a.freq = rope_freqs(dims);
   cudaError_t e = launch_absorb(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
 }
@@ -217,7 +228,8 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   if (batch == 0) return QKN_OK;
   if (!q_tilde || !a_q || !q_rope_hat || !block_table || !seq_lens || !workspace || !out || !lse)
     return QKN_ERR_INVALID_ARG;
-  if (!aligned(q_tilde, 16) || !aligned(q_rope_hat, 16) || !aligned(workspace, 256)) return QKN_ERR_INVALID_ARG;
+  if (!aligned(q_tilde, 16) || !aligned(q_rope_hat, 16) || !aligned(workspace, 256) || !aligned(out, 16))
+    return QKN_ERR_INVALID_ARG;
   if (opts && (opts->max_ctas < 0 || opts->wait_limit < 0 ||
                (opts->head_tile && opts->head_tile != 16 && opts->head_tile != 32 && opts->head_tile != 64)))
     return QKN_ERR_INVALID_ARG;
@@ -277,6 +289,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   c.ht_count = a.ht_count;
   c.ncta = ncta;
   c.max_blocks = max_blocks;
+  c.max_items = ncta + 1;
   c.part_o = a.part_o;
   c.part_lse = a.part_lse;
   c.out = out;

@@ -6,9 +6,9 @@
 // Three launches on the caller's stream:
 //   1. append_copy:     one warp per token — latent copy, RoPE key
 //                       (RMS-normalise, weight, rotate), a_k slots zeroed;
-//   2. append_keyrms:   z = c W^K_g tiled over (column block, token tile,
-//                       group); each CTA adds sum(z^2) of its columns into
-//                       the token's a_k slot;
+//   2. append_keyrms:   z = c W^K_g tiled over (32-column block, token
+//                       tile, group); each CTA adds sum(z^2) of its columns
+//                       into the token's a_k slot;
 //   3. append_finalize: a_k = 1 / sqrt(sum / (n_g d_h) + eps).
 // The key z is only ever held in registers; it is never written anywhere.
 #include "common.cuh"
@@ -16,30 +16,31 @@
 
 namespace qkn {
 
-// Rotate pairs (i, i + d/2) of x (length d, lanes hold x[lane], x[lane+32], ...)
-// by angle pos * theta^(-2i/d).  Angles are formed in fp64 so that positions in
-// the hundreds of thousands keep full fp32 accuracy after the rotation.
-__device__ __forceinline__ void rope_pair(float& x1, float& x2, int i, int d, int32_t pos, float theta) {
-  const double freq = pow((double)theta, -2.0 * (double)i / (double)d);
-  double s, c;
-  sincos((double)pos * freq, &s, &c);
-  const float cs = (float)c, sn = (float)s;
-  const float a = x1 * cs - x2 * sn;
-  const float b = x2 * cs + x1 * sn;
-  x1 = a;
-  x2 = b;
-}
-
 template <typename T>
-__global__ void __launch_bounds__(256) append_copy_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(256) append_copy_kernel(const __grid_constant__ AppendArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= a.n_tok) return;
   const int64_t slot = a.slot[warp];
   const int32_t pos = a.pos[warp];
-  const T* src = static_cast<const T*>(a.c_new) + (int64_t)warp * a.r;
-  T* dst = static_cast<T*>(a.latent) + slot * a.r;
-  for (int k = lane; k < a.r; k += 32) dst[k] = src[k];
+  // latent row: 16-byte vectors (rows are a multiple of 16 bytes)
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(a.c_new) + (int64_t)warp * a.r);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.latent) + slot * a.r);
+  const int nvec = a.r * (int)sizeof(T) / 16;
+  uint4 cv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int k = lane + 32 * u;
+    if (k < nvec) cv[u] = src[k];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int k = lane + 32 * u;
+    if (k < nvec) dst[k] = cv[u];
+  }
+  for (int k = lane + 128; k < nvec; k += 32) dst[k] = src[k];
 
   // RoPE key: d_R <= 128, so each lane holds at most 4 elements.
   const T* kr = static_cast<const T*>(a.k_rope_raw) + (int64_t)warp * a.d_rope;
@@ -72,71 +73,126 @@ __global__ void __launch_bounds__(256) append_copy_kernel(AppendArgs a) {
   T* kout = static_cast<T*>(a.k_rope) + slot * a.d_rope;
   const int half = a.d_rope / 2;
   for (int i = lane; i < half; i += 32) {
-    float x1 = row[i], x2 = row[i + half];
-    rope_pair(x1, x2, i, a.d_rope, pos, a.rope_theta);
-    kout[i] = from_f32<T>(x1);
-    kout[i + half] = from_f32<T>(x2);
+    const float x1 = row[i], x2 = row[i + half];
+    float sn, cs;
+    rope_sincos(pos, a.freq.f[i], sn, cs);
+    kout[i] = from_f32<T>(x1 * cs - x2 * sn);
+    kout[i + half] = from_f32<T>(x2 * cs + x1 * sn);
   }
   for (int g = lane; g < a.groups; g += 32) a.a_k[slot * a.groups + g] = 0.f;
 }
 
-constexpr int kRmsTok = 32;      // tokens per CTA
-constexpr int kRmsCols = 256;    // key columns per CTA (one per thread)
+// Key statistic sum(z^2), z = c W^K_g.  CTA = (32 key columns, TT tokens,
+// group); its 256 threads are 32 columns x 8 slices of the latent dimension,
+// so every thread issues r/8 independent, coalesced loads of W and reuses
+// each for TT tokens held in shared memory.  Slices are summed in shared
+// memory, squared, reduced over the CTA's 32 columns and added into the
+// token's a_k slot (zeroed by append_copy_kernel).
+constexpr int kRmsCols = 32;
+constexpr int kRmsSlices = 8;
 
-template <typename T>
-__global__ void __launch_bounds__(kRmsCols) append_keyrms_kernel(AppendArgs a) {
+template <typename T, int TT>
+__global__ void __launch_bounds__(kRmsCols * kRmsSlices) append_keyrms_kernel(AppendArgs a) {
   extern __shared__ float4 smem4[];
-  float* cs = reinterpret_cast<float*>(smem4);          // [kRmsTok][r]
-  __shared__ float red[kRmsCols / 32][kRmsTok];
+  float* cs = reinterpret_cast<float*>(smem4);                    // [TT][r]
+  float* zp = cs + TT * a.r;                                      // [kRmsSlices][TT][kRmsCols]
   const int g = blockIdx.z;
-  const int t0 = blockIdx.y * kRmsTok;
-  const int ntok = min(kRmsTok, a.n_tok - t0);
-  const int width = a.width;                            // n_g * d_h
-  const int n = blockIdx.x * kRmsCols + threadIdx.x;
+  const int t0 = blockIdx.y * TT;
+  const int ntok = min(TT, a.n_tok - t0);
+  const int width = a.width;
+  const int col = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int n = blockIdx.x * kRmsCols + col;
+  pdl_trigger();
+  pdl_wait();
 
-  const T* c = static_cast<const T*>(a.c_new);
-  for (int e = threadIdx.x; e < kRmsTok * a.r; e += blockDim.x) {
-    const int t = e / a.r, k = e - t * a.r;
-    cs[e] = t < ntok ? to_f32(c[(int64_t)(t0 + t) * a.r + k]) : 0.f;
-  }
-  __syncthreads();
-
-  float acc[kRmsTok];
+  {   // stage the token tile as fp32, 16 bytes of input per load, loads batched
+    constexpr int kPer = 16 / (int)sizeof(T);          // elements per 16-byte load
+    const uint4* c4 = reinterpret_cast<const uint4*>(static_cast<const T*>(a.c_new) + (int64_t)t0 * a.r);
+    const int nvec = TT * a.r / kPer;
+    for (int e0 = threadIdx.x; e0 < nvec; e0 += 4 * blockDim.x) {
+      uint4 v[4];
 #pragma unroll
-  for (int t = 0; t < kRmsTok; ++t) acc[t] = 0.f;
-  if (n < width) {
-    const float* w = a.w_k + (int64_t)g * a.r * width + n;
-    for (int k = 0; k < a.r; k += 4) {
-      const float w0 = w[(int64_t)(k + 0) * width], w1 = w[(int64_t)(k + 1) * width];
-      const float w2 = w[(int64_t)(k + 2) * width], w3 = w[(int64_t)(k + 3) * width];
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x;
+        v[u] = (e < nvec && (e * kPer) / a.r < ntok) ? c4[e] : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-      for (int t = 0; t < kRmsTok; ++t) {
-        const float4 cv = *reinterpret_cast<const float4*>(cs + t * a.r + k);
-        acc[t] = fmaf(cv.x, w0, acc[t]);
-        acc[t] = fmaf(cv.y, w1, acc[t]);
-        acc[t] = fmaf(cv.z, w2, acc[t]);
-        acc[t] = fmaf(cv.w, w3, acc[t]);
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e < nvec) {
+          const T* x = reinterpret_cast<const T*>(&v[u]);
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) cs[e * kPer + q] = to_f32(x[q]);
+        }
       }
     }
   }
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  __syncthreads();
+
+  float acc[TT];
 #pragma unroll
-  for (int t = 0; t < kRmsTok; ++t) {
-    float v = acc[t] * acc[t];
+  for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+  // latent rows [k0, k1) of this slice
+  const int k0 = (int)((int64_t)slice * a.r / kRmsSlices);
+  const int k1 = (int)((int64_t)(slice + 1) * a.r / kRmsSlices);
+  if (n < width) {
+    const float* w = a.w_k + (int64_t)g * a.r * width + n;
+    int k = k0;
+    // 32 independent W loads in flight per thread, then their FMAs (16-byte token-row reads
+    // need k % 4 == 0, which holds whenever r % 32 == 0)
+    const bool vec_ok = ((k0 | a.r) & 3) == 0;
+    for (; vec_ok && k + 32 <= k1; k += 32) {
+      float wv[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) wv[u] = w[(int64_t)(k + u) * width];
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float4* crow = reinterpret_cast<const float4*>(cs + t * a.r + k);   // r % 4 == 0, k % 32 == k0 % 4 == 0
+#pragma unroll
+        for (int u4 = 0; u4 < 8; ++u4) {
+          const float4 cv = crow[u4];
+          acc[t] = fmaf(cv.x, wv[4 * u4 + 0], acc[t]);
+          acc[t] = fmaf(cv.y, wv[4 * u4 + 1], acc[t]);
+          acc[t] = fmaf(cv.z, wv[4 * u4 + 2], acc[t]);
+          acc[t] = fmaf(cv.w, wv[4 * u4 + 3], acc[t]);
+        }
+      }
+    }
+    for (; k + 8 <= k1; k += 8) {
+      float wv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) wv[u] = w[(int64_t)(k + u) * width];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+#pragma unroll
+        for (int t = 0; t < TT; ++t) acc[t] = fmaf(cs[t * a.r + k + u], wv[u], acc[t]);
+      }
+    }
+    for (; k < k1; ++k) {
+      const float wv = w[(int64_t)k * width];
+#pragma unroll
+      for (int t = 0; t < TT; ++t) acc[t] = fmaf(cs[t * a.r + k], wv, acc[t]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TT; ++t) zp[(slice * TT + t) * kRmsCols + col] = acc[t];
+  __syncthreads();
+  // thread (slice, col) finishes tokens slice, slice + 8, ...: z summed over slices, squared,
+  // then summed over the 32 columns of the warp
+  for (int t = slice; t < ntok; t += kRmsSlices) {
+    float z = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < kRmsSlices; ++sl) z += zp[(sl * TT + t) * kRmsCols + col];
+    float v = (n < width) ? z * z : 0.f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[wid][t] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < ntok) {
-    float s = 0.f;
-#pragma unroll
-    for (int w8 = 0; w8 < kRmsCols / 32; ++w8) s += red[w8][threadIdx.x];
-    atomicAdd(a.a_k + (int64_t)a.slot[t0 + threadIdx.x] * a.groups + g, s);
+    if (col == 0) atomicAdd(a.a_k + (int64_t)a.slot[t0 + t] * a.groups + g, v);
   }
 }
 
 __global__ void append_finalize_kernel(AppendArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n_tok * a.groups) return;
   const int t = i / a.groups, g = i - t * a.groups;
@@ -144,21 +200,29 @@ __global__ void append_finalize_kernel(AppendArgs a) {
   *p = 1.0f / sqrtf(*p / (float)a.width + a.eps);
 }
 
-template <typename T>
-static cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t st) {
-  append_copy_kernel<T><<<(a.n_tok + 7) / 8, 256, 0, st>>>(a);
-  const size_t smem = (size_t)kRmsTok * a.r * sizeof(float);
+template <typename T, int TT>
+static cudaError_t launch_keyrms(const AppendArgs& a, cudaStream_t st) {
+  const size_t smem = ((size_t)TT * a.r + (size_t)kRmsSlices * TT * kRmsCols) * sizeof(float);
   static bool attr_set = false;   // one attribute per instantiation
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(append_keyrms_kernel<T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(append_keyrms_kernel<T, TT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((a.width + kRmsCols - 1) / kRmsCols, (a.n_tok + kRmsTok - 1) / kRmsTok, a.groups);
-  append_keyrms_kernel<T><<<grid, kRmsCols, smem, st>>>(a);
-  append_finalize_kernel<<<(a.n_tok * a.groups + 255) / 256, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  dim3 grid((a.width + kRmsCols - 1) / kRmsCols, (a.n_tok + TT - 1) / TT, a.groups);
+  return launch_chained(append_keyrms_kernel<T, TT>, grid, dim3(kRmsCols * kRmsSlices), smem, st, a);
+}
+
+template <typename T>
+static cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t st) {
+  cudaError_t e0 = launch_chained(append_copy_kernel<T>, dim3((a.n_tok + 7) / 8), dim3(256), 0, st, a);
+  if (e0 != cudaSuccess) return e0;
+  // few tokens (a decode step): small token tiles spread over many CTAs;
+  // many tokens (filling a cache): larger tiles re-read W less often
+  cudaError_t e = a.n_tok <= 256 ? launch_keyrms<T, 16>(a, st) : launch_keyrms<T, 32>(a, st);
+  if (e != cudaSuccess) return e;
+  return launch_chained(append_finalize_kernel, dim3((a.n_tok * a.groups + 255) / 256), dim3(256), 0, st, a);
 }
 
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st) {

@@ -6,7 +6,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/qkn.h"
+#include <utility>
+
+#include "qkn.h"
 
 namespace qkn {
 
@@ -20,6 +22,44 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------- launch chaining
+// Kernels are launched with programmatic stream serialisation: each one lets
+// its successor start launching at once (pdl_trigger) and waits for its
+// predecessor's completion and memory flush (pdl_wait) before it reads
+// anything an earlier launch may have written.  Without a programmatic
+// predecessor pdl_wait returns immediately.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch `kernel` on `st` with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// ---------------------------------------------------------------- RoPE
+// sin and cos of pos * freq.  The angle is formed and reduced to [-pi, pi] in
+// fp64 (one-constant reduction by 2*pi is exact to ~1e-11 here, positions stay
+// below 2^31), so that positions in the hundreds of thousands keep fp32
+// accuracy; the reduced angle then goes through fp32 sincosf.
+__device__ __forceinline__ void rope_sincos(int32_t pos, double freq, float& s, float& c) {
+  const double ang = (double)pos * freq;
+  const double k = rint(ang * 0.15915494309189535);            // 1 / (2 pi)
+  const double red = fma(-k, 6.283185307179586, ang);          // ang - k * 2 pi
+  sincosf((float)red, &s, &c);
 }
 
 // ---------------------------------------------------------------- status word

@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(kSimtRows * 32) decode_simt_kernel(DecodeArgs 
   __shared__ Cursor cur_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
   SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
   if (warp == 0) {
     Cursor c = sched_begin(sp, blockIdx.x);
@@ -160,8 +162,7 @@ static cudaError_t launch_simt_nk(const DecodeArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_simt_kernel<T, NK><<<a.ncta, kSimtRows * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_chained(decode_simt_kernel<T, NK>, dim3(a.ncta), dim3(kSimtRows * 32), smem, st, a);
 }
 
 template <typename T>

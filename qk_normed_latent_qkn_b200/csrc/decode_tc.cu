@@ -43,7 +43,9 @@ constexpr int kTile = 128;                 // tokens per tile (MMA M)
 constexpr int kRkv = 512;                  // latent width this kernel takes
 constexpr int kChunks = kRkv / 64;         // 64-column (128-byte) chunks of the latent
 constexpr int kDrope = 64;                 // RoPE width this kernel takes
-constexpr int kSlotBytes = kTile * 128;    // one chunk of one tile: 16 KB
+constexpr int kChunkBytes = kTile * 128;   // one 64-column chunk of one tile: 16 KB
+constexpr int kSlotBytes = 2 * kChunkBytes; // a ring slot holds two chunks (one 128-row latent block): 32 KB
+constexpr int kSlotsPerTile = kChunks / 2;
 constexpr int kPageChunkBytes = 64 * 128;  // one chunk of one page: 8 KB
 constexpr int kMaxGroups = 8;
 constexpr int kAkSlotBytes = kTile * kMaxGroups * 4;
@@ -53,17 +55,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;       // rescale O only when a column max grows by > 2^8
 constexpr int64_t kDrainLimit = 4000000000LL;
+constexpr int kPrefetchPages = 6;          // pages the L2 prefetch runs ahead of the TMA loads
 
 template <int R>
 struct Cfg {
-  static constexpr int NS = (R == 64) ? 8 : 10;              // latent chunk slots (even)
+  static constexpr int NS = (R == 64) ? 4 : 5;               // latent ring slots (two chunks each)
   static constexpr int NKR = (R == 16) ? 2 : 1;              // RoPE-key / P^T slots
   static constexpr int TMEM_COLS = (6 * R <= 128) ? 128 : (6 * R <= 256 ? 256 : 512);
   static constexpr int Q_OFF = 0;                                    // R x 512 bf16, 8 chunks
   static constexpr int QR_OFF = Q_OFF + R * 1024;                    // R x 64 bf16
   static constexpr int C_OFF = QR_OFF + ((R * 128 + 1023) / 1024) * 1024;
   static constexpr int KR_OFF = C_OFF + NS * kSlotBytes;
-  static constexpr int AK_OFF = KR_OFF + NKR * kSlotBytes;
+  static constexpr int AK_OFF = KR_OFF + NKR * kChunkBytes;
   static constexpr int MISC_OFF = AK_OFF + NKR * kAkSlotBytes;
   static constexpr int MISC_BYTES = 4096;
   static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;          // + alignment slack
@@ -78,13 +81,13 @@ struct Misc {
   uint32_t tmem_base;
   int32_t abort_flag;
   Cursor cursor;
-  float aq2[R];      // a_q * log2(e) per column (query row)
-  int32_t grp[R];    // KV group per column
-  int32_t qlim[R];   // last visible token position per column (-1: padding column)
-  float mu[R];       // running max (log2 units) used for the exponentials
-  float corr[R];     // rescale factor of the current tile
-  float linv[R];
-  float red[4][R];   // per-warp partial column reductions
+  alignas(16) float aq2[R];      // a_q * log2(e) per column (query row)
+  alignas(16) int32_t grp[R];    // KV group per column
+  alignas(16) int32_t qlim[R];   // last visible token position per column (-1: padding column)
+  alignas(16) float mu[R];       // running max (log2 units) used for the exponentials
+  alignas(16) float corr[R];     // rescale factor of the current tile
+  alignas(16) float linv[R];
+  alignas(16) float red[4][R];   // per-warp partial column reductions
 };
 
 }  // namespace
@@ -164,6 +167,42 @@ __device__ __forceinline__ bool group_any(bool v) {
   return r != 0;
 }
 
+// Walks the pages of one CTA's items, in load order, issuing L2 prefetches
+// for the latent, RoPE-key and a_k rows of each page.  The producer keeps it
+// a fixed number of pages ahead of its TMA loads, so that HBM streaming does
+// not wait for shared-memory ring slots to free up.
+struct PrefetchWalker {
+  Cursor cur;
+  Item it;
+  int32_t page;     // next page of `it` to prefetch
+  bool live;        // an item is open
+  bool done;        // no items left
+
+  __device__ __forceinline__ void init(const Cursor& c) {
+    cur = c;
+    live = false;
+    done = false;
+  }
+  template <bool AK_ONE>
+  __device__ __forceinline__ void step(const DecodeArgs& a, const SchedParams& sp, int cta) {
+    if (done) return;
+    if (!live || page >= it.p1) {
+      if (!sched_next(cur, sp, cta, it)) {
+        done = true;
+        return;
+      }
+      live = true;
+      page = it.p0;
+    }
+    const int32_t blk = a.block_table[(int64_t)it.b * a.max_blocks + page];
+    ++page;
+    if (blk < 0 || blk >= a.num_blocks) return;
+    prefetch_l2(static_cast<const __nv_bfloat16*>(a.latent) + (int64_t)blk * 64 * kRkv, 64 * kRkv * 2);
+    prefetch_l2(static_cast<const __nv_bfloat16*>(a.k_rope) + (int64_t)blk * 64 * kDrope, 64 * kDrope * 2);
+    if (!AK_ONE) prefetch_l2(a.a_k + (int64_t)blk * 64 * a.groups, 64u * a.groups * 4u);
+  }
+};
+
 template <int R, bool AK_ONE>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TcMaps maps) {
   using C = Cfg<R>;
@@ -171,7 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
   using MiscT = Misc<R, NS, NKR>;
   static_assert(sizeof(MiscT) <= C::MISC_BYTES, "misc shared-memory block");
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte alignment for the 128-byte swizzle atoms, by pointer arithmetic on the shared
+  // array so that every access below stays a shared-memory (not generic) access
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   MiscT& ms = *reinterpret_cast<MiscT*>(smem + C::MISC_OFF);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -208,6 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     tmem_alloc(smem_u32(&ms.tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
+  // everything above touches only this CTA's own memory; inputs are read after the wait
+  pdl_trigger();
+  pdl_wait();
   if (warp == 0) {
     Cursor c = sched_begin(sp, blockIdx.x);
     if (lane == 0) ms.cursor = c;
@@ -225,6 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       int64_t c_it = 0, k_it = 0;
       int n_item = 0;
       bool ok = true;
+      PrefetchWalker pf;
+      pf.init(cur);
+      for (int i = 0; i < kPrefetchPages; ++i) pf.step<AK_ONE>(a, sp, blockIdx.x);
       while (ok && sched_next(cur, sp, blockIdx.x, it)) {
         if (!mbar_wait(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
         const int qrow0 = it.b * qrows + it.ht * R;
@@ -236,19 +283,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
         for (int p = it.p0; p < it.p1 && ok; p += 2) {
           const int np = min(2, it.p1 - p);
+          for (int i = 0; i < np; ++i) pf.step<AK_ONE>(a, sp, blockIdx.x);
           int32_t blk[2] = {row[p], np > 1 ? row[p + 1] : 0};
           for (int i = 0; i < np; ++i)
             if (blk[i] < 0 || blk[i] >= a.num_blocks) {
               record_status(a.status, QKN_ERR_BOUNDS);
               blk[i] = 0;
             }
-          for (int k = 0; k < kChunks; ++k) {
+          for (int m = 0; m < kSlotsPerTile; ++m) {
             const int slot = (int)(c_it % NS);
             if (!mbar_wait(smem_u32(&ms.empty[slot]), ((c_it / NS) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
             const uint32_t fb = smem_u32(&ms.full[slot]);
-            mbar_arrive_expect_tx(fb, np * kPageChunkBytes);
+            mbar_arrive_expect_tx(fb, 2 * np * kPageChunkBytes);
             const uint32_t dst = sb + C::C_OFF + slot * kSlotBytes;
-            for (int i = 0; i < np; ++i) tma_load_2d(dst + i * kPageChunkBytes, &maps.latent, k * 64, blk[i] * 64, fb);
+            for (int j = 0; j < 2; ++j)
+              for (int i = 0; i < np; ++i)
+                tma_load_2d(dst + j * kChunkBytes + i * kPageChunkBytes, &maps.latent, (2 * m + j) * 64, blk[i] * 64, fb);
             ++c_it;
           }
           if (!ok) break;
@@ -258,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           const uint32_t akpage = 64u * (uint32_t)G * 4u;
           mbar_arrive_expect_tx(kb, np * kPageChunkBytes + (AK_ONE ? 0u : np * akpage));
           for (int i = 0; i < np; ++i) {
-            tma_load_2d(sb + C::KR_OFF + ks * kSlotBytes + i * kPageChunkBytes, &maps.krope, 0, blk[i] * 64, kb);
+            tma_load_2d(sb + C::KR_OFF + ks * kChunkBytes + i * kPageChunkBytes, &maps.krope, 0, blk[i] * 64, kb);
             if (!AK_ONE)
               bulk_load(sb + C::AK_OFF + ks * kAkSlotBytes + i * akpage, a.a_k + (int64_t)blk[i] * 64 * G, akpage, kb);
           }
@@ -282,7 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, R, false, false);
-      constexpr uint32_t idPV = idesc_bf16(128, R, true, false);
+      constexpr uint32_t idPV = idesc_bf16(128, R, true, true);
+      // P^T is stored token-major (MN-major B): rows of 2R bytes, swizzled with the matching width
+      constexpr uint32_t kPswz = (R == 16) ? 6u : (R == 32) ? 4u : 2u;   // 32 / 64 / 128-byte swizzle
       const uint32_t tS = tmem + 4 * R, tSR = tmem + 5 * R;
       int64_t c_it = 0, k_it = 0, tile_n = 0;
       int n_item = 0;
@@ -294,24 +346,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         for (int i = 0; i < ntiles && ok; ++i) {
           const int np = min(2, it.p1 - (it.p0 + 2 * i));
           const int64_t c_first = c_it;
-          // S^T = C . Q~^T over the 8 latent chunks
-          for (int k = 0; k < kChunks; ++k) {
+          // S^T = C . Q~^T over the 8 latent chunks, two chunks per ring slot
+          for (int m = 0; m < kSlotsPerTile; ++m) {
             const int slot = (int)(c_it % NS);
             if (!mbar_wait(smem_u32(&ms.full[slot]), (c_it / NS) & 1, a.wait_limit)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t abase = sb + C::C_OFF + slot * kSlotBytes;
-            const uint32_t bbase = sb + C::Q_OFF + k * R * 128;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tS, smem_desc(abase + kk * 32, 16, 1024), smem_desc(bbase + kk * 32, 16, 1024), idS,
-                       (k | kk) != 0);
+            for (int j = 0; j < 2; ++j) {
+              const int k = 2 * m + j;
+              const uint32_t abase = sb + C::C_OFF + slot * kSlotBytes + j * kChunkBytes;
+              const uint32_t bbase = sb + C::Q_OFF + k * R * 128;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tS, smem_desc(abase + kk * 32, 16, 1024), smem_desc(bbase + kk * 32, 16, 1024), idS,
+                         (k | kk) != 0);
+            }
             ++c_it;
           }
           if (!ok) break;
           const int ks = (int)(k_it % NKR);
           if (!mbar_wait(smem_u32(&ms.krfull[ks]), (k_it / NKR) & 1, a.wait_limit)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t krbase = sb + C::KR_OFF + ks * kSlotBytes;
+          const uint32_t krbase = sb + C::KR_OFF + ks * kChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16(tSR, smem_desc(krbase + kk * 32, 16, 1024), smem_desc(sb + C::QR_OFF + kk * 32, 16, 1024),
@@ -323,16 +379,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           if (!mbar_wait(smem_u32(&ms.p_full), tile_n & 1, a.wait_limit)) { ok = false; break; }
           tc_fence_after();
           const int nkk = np * 4;   // 16-token K steps that hold real pages
-          for (int m = 0; m < 4; ++m) {
-            const int s0 = (int)((c_first + 2 * m) % NS);
+          for (int m = 0; m < kSlotsPerTile; ++m) {
+            const int s0 = (int)((c_first + m) % NS);
             const uint32_t abase = sb + C::C_OFF + s0 * kSlotBytes;
             for (int kk = 0; kk < nkk; ++kk) {
-              const uint64_t ad = smem_desc(abase + kk * 2048, kSlotBytes, 1024);
-              const uint64_t bd = smem_desc(krbase + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
+              // A = C^T of latent block m (MN-major: the two chunks of the slot are LBO apart)
+              const uint64_t ad = smem_desc(abase + kk * 2048, kChunkBytes, 1024);
+              // B = P^T rows 16kk..16kk+15 (MN-major, 2R-byte rows, SBO = eight rows)
+              const uint64_t bd = smem_desc_sw(krbase + kk * 32 * R, 16, 16 * R, kPswz);
               mma_bf16(tmem + m * R, ad, bd, idPV, (i > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(smem_u32(&ms.empty[s0]));
-            mma_commit(smem_u32(&ms.empty[s0 + 1]));
           }
           mma_commit(smem_u32(&ms.krempty[ks]));
           ++k_it;
@@ -392,13 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         }
         const bool row_ok = t < nvalid;
         const int tpos = tok0 + t;
-        // logit of column c for this token row, in log2 units; -inf when masked
-        auto logit = [&](int c, uint32_t sc, uint32_t sr) {
-          float akc = ak0;
-          if (!AK_ONE && G > 1) akc = akrow[ms.grp[c]];
-          const float v = ms.aq2[c] * akc * __uint_as_float(sc) + kLog2e * __uint_as_float(sr);
-          return (row_ok && tpos <= ms.qlim[c]) ? v : -INFINITY;
-        };
         // pass 1: column maxima of this tile
         {
           float v[R];
@@ -407,9 +457,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
             uint32_t sc[16], sr[16];
             tmem_ld16(tl + 4 * R + c0, sc);
             tmem_ld16(tl + 5 * R + c0, sr);
+            float aq[16];
+            int ql[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              *reinterpret_cast<float4*>(aq + 4 * q) = *reinterpret_cast<const float4*>(ms.aq2 + c0 + 4 * q);
+              *reinterpret_cast<int4*>(ql + 4 * q) = *reinterpret_cast<const int4*>(ms.qlim + c0 + 4 * q);
+            }
             tmem_wait_ld(sc, sr);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[c0 + e] = logit(c0 + e, sc[e], sr[e]);
+            for (int e = 0; e < 16; ++e) {
+              const int c = c0 + e;
+              float akc = ak0;
+              if (!AK_ONE && G > 1) akc = akrow[ms.grp[c]];
+              const float x = aq[e] * akc * __uint_as_float(sc[e]) + kLog2e * __uint_as_float(sr[e]);
+              v[c] = (row_ok && tpos <= ql[e]) ? x : -INFINITY;
+            }
           }
           warp_col_reduce<R, true>(v, lane);
           store_reduced<R>(ms.red[warp], v, lane);
@@ -428,32 +491,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           ms.corr[t] = cr;
         }
         const bool rescale = group_any(mine) && i > 0;
-        // pass 2: probabilities, running column sums, and P^T (K-major, 128-byte
-        // swizzle: row = query row c, element = token t) into the RoPE-key slot
-        uint8_t* pbase = smem + C::KR_OFF + ks * kSlotBytes + (t >> 6) * (R * 128);
-        const int within = t & 63;
+        // pass 2: probabilities, running column sums, and P^T into the RoPE-key slot, token-major:
+        // row t holds this token's R probabilities (2R bytes), 16-byte units swizzled by row
+        uint8_t* prow = smem + C::KR_OFF + ks * kChunkBytes + t * (2 * R);
+        const int swz = (R == 16) ? ((t >> 2) & 1) : (R == 32) ? ((t >> 1) & 3) : (t & 7);
 #pragma unroll
         for (int c0 = 0; c0 < R; c0 += 16) {
           uint32_t sc[16], sr[16];
           tmem_ld16(tl + 4 * R + c0, sc);
           tmem_ld16(tl + 5 * R + c0, sr);
-          tmem_wait_ld(sc, sr);
+          float aq[16], mu[16], cr[16];
+          int ql[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = c0 + e;
-            const float xc = logit(c, sc[e], sr[e]);
-            const float p = (xc == -INFINITY) ? 0.f : ex2(xc - ms.mu[c]);
-            lpart[c] = lpart[c] * ms.corr[c] + p;
-            const int chunk = (within >> 3) ^ (c & 7);
-            *reinterpret_cast<__nv_bfloat16*>(pbase + c * 128 + (chunk << 4) + ((within & 7) << 1)) =
-                __float2bfloat16_rn(p);
+          for (int q = 0; q < 4; ++q) {
+            *reinterpret_cast<float4*>(aq + 4 * q) = *reinterpret_cast<const float4*>(ms.aq2 + c0 + 4 * q);
+            *reinterpret_cast<int4*>(ql + 4 * q) = *reinterpret_cast<const int4*>(ms.qlim + c0 + 4 * q);
+            *reinterpret_cast<float4*>(mu + 4 * q) = *reinterpret_cast<const float4*>(ms.mu + c0 + 4 * q);
+            *reinterpret_cast<float4*>(cr + 4 * q) = *reinterpret_cast<const float4*>(ms.corr + c0 + 4 * q);
           }
+          tmem_wait_ld(sc, sr);
+          uint32_t packed[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float pp[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int c = c0 + e + u;
+              float akc = ak0;
+              if (!AK_ONE && G > 1) akc = akrow[ms.grp[c]];
+              const float x = aq[e + u] * akc * __uint_as_float(sc[e + u]) + kLog2e * __uint_as_float(sr[e + u]);
+              const bool vis = row_ok && tpos <= ql[e + u];
+              const float p = vis ? ex2(x - mu[e + u]) : 0.f;
+              lpart[c] = lpart[c] * cr[e + u] + p;
+              pp[u] = p;
+            }
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(pp[0], pp[1]);
+            packed[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          const int u0 = c0 / 8;    // 16-byte units c0/8 and c0/8 + 1 of the row
+          *reinterpret_cast<uint4*>(prow + (((u0 + 0) ^ swz) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ swz) << 4)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
         // rows of real pages past the context: zero them so that 0 * garbage cannot reach O
         if (!row_ok && t < np * 64) {
 #pragma unroll
           for (int k = 0; k < kChunks; ++k) {
-            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + ((c_it + k) % NS) * kSlotBytes + t * 128);
+            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + ((c_it + k / 2) % NS) * kSlotBytes +
+                                                   (k & 1) * kChunkBytes + t * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q) rowp[q] = make_uint4(0, 0, 0, 0);
           }
@@ -476,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(smem_u32(&ms.p_full));
-        c_it += kChunks;
+        c_it += kSlotsPerTile;
         ++k_it;
         ++tile_n;
       }
@@ -564,8 +648,7 @@ cudaError_t launch_tc(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_tc_kernel<R, AK_ONE><<<a.ncta, kThreads, Cfg<R>::SMEM, st>>>(a, maps);
-  return cudaGetLastError();
+  return launch_chained(decode_tc_kernel<R, AK_ONE>, dim3(a.ncta), dim3(kThreads), Cfg<R>::SMEM, st, a, maps);
 }
 
 }  // namespace

@@ -6,6 +6,12 @@
 
 namespace qkn {
 
+// RoPE frequencies theta^(-2i/d_R), i < d_R/2 (d_R <= 128), formed in fp64 on
+// the host from the dims and passed by value with the launch.
+struct RopeFreqs {
+  double f[64];
+};
+
 struct AppendArgs {
   void* latent;            // cache pool
   void* k_rope;
@@ -18,6 +24,7 @@ struct AppendArgs {
   const float* gamma_kr;   // [d_rope]
   int32_t n_tok, r, d_rope, groups, width;   // width = n_g * d_h
   float eps, rope_theta;
+  RopeFreqs freq;
 };
 
 struct AbsorbArgs {
@@ -33,6 +40,7 @@ struct AbsorbArgs {
   void* q_rope_hat;        // [n_q, H, d_rope]
   int32_t n_q, heads, groups, r, d_h, d_rope;
   float eps, softmax_scale, rope_theta;
+  RopeFreqs freq;
 };
 
 struct DecodeArgs {
@@ -60,6 +68,7 @@ struct DecodeArgs {
 struct CombineArgs {
   const int32_t* seq_lens;
   int32_t batch, s_q, heads, r, rows, ht_count, ncta, max_blocks;
+  int32_t max_items;         // upper bound on splits per row (ncta + 1)
   const float* part_o;
   const float* part_lse;
   void* out;                 // [batch, s_q, H, r]

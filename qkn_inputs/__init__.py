@@ -88,9 +88,10 @@ WORKLOAD_ORDER = ["tiny_f32", "small_mla_bf16", "large_mla_bf16", "long_ctx_bf16
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding bf16 values."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = x.view(np.uint32)
+    # finite inputs only: the largest finite pattern 0xFF7FFFFF plus 0x8000 stays below 2^32
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32)
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -110,8 +110,8 @@ def test_identity_table_equals_random_table(kernel):
     _, o1, l1 = run_decode(paged, kernel=KERNELS[kernel])
     _, o2, l2 = run_decode(flat, kernel=KERNELS[kernel])
     # qkn_append accumulates sum(z^2) with fp32 atomics, so the two caches may differ in the
-    # last bit of a_k; the outputs agree to far inside the parity tolerance
-    assert np.abs(o1 - o2).max() <= 1e-3 * np.abs(o1).max()
+    # last bit of a_k, which can move a bf16 output by one unit in the last place (2^-8 relative)
+    assert np.abs(o1 - o2).max() <= 2 ** -7 * np.abs(o1).max()
     assert np.abs(l1 - l2).max() <= 1e-3
 
 
