@@ -14,15 +14,21 @@
 //   O^T[512 x R] += C^T[512 x 128] . P^T[128 x R]   (4 latent blocks x 8 MMAs)
 // with the latent tile C staged once in shared memory and read by both
 // products (as K-major A for S, as MN-major A for O).  The fp32 accumulator
-// O^T takes 4R TMEM columns, S^T and S_R^T R columns each.
+// O^T takes 4R TMEM columns; S^T and S_R^T take R columns each and are double
+// buffered, so that the scores of tile i+1 are computed while the softmax and
+// the output product of tile i run.
 //
-// Warp roles (192 threads, one CTA per SM):
+// Warp roles (224 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue: thread t owns TMEM lane t = token row t of
 //              S^T and latent row t of each O^T block; column (query row)
 //              maxima and sums are reduced across the 128 threads;
 //   warp 4     TMA producer: query tiles per item, then per tile eight 16 KB
 //              latent chunks, the RoPE-key chunk and the a_k rows;
-//   warp 5     TMEM allocator and single-thread MMA issuer.
+//   warp 5     TMEM allocator and issuer of the score MMAs (S^T, S_R^T);
+//   warp 6     issuer of the output MMAs (O^T).
+// A single thread issues tcgen05.mma at a bounded rate, so the two products
+// have one issuing thread each, and every shared-memory descriptor is built
+// once: a K step or a ring slot only moves its start-address field.
 // Shared-memory rings: latent chunks (full/empty mbarrier pairs), and a
 // RoPE-key slot that the softmax reuses for P^T once the RoPE MMAs are done.
 // Every mbarrier wait is bounded; a wait that runs out records
@@ -49,7 +55,7 @@ constexpr int kSlotsPerTile = kChunks / 2;
 constexpr int kPageChunkBytes = 64 * 128;  // one chunk of one page: 8 KB
 constexpr int kMaxGroups = 8;
 constexpr int kAkSlotBytes = kTile * kMaxGroups * 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kSoftThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -61,7 +67,7 @@ template <int R>
 struct Cfg {
   static constexpr int NS = (R == 64) ? 4 : 5;               // latent ring slots (two chunks each)
   static constexpr int NKR = (R == 16) ? 2 : 1;              // RoPE-key / P^T slots
-  static constexpr int TMEM_COLS = (6 * R <= 128) ? 128 : (6 * R <= 256 ? 256 : 512);
+  static constexpr int TMEM_COLS = (8 * R <= 128) ? 128 : (8 * R <= 256 ? 256 : 512);
   static constexpr int Q_OFF = 0;                                    // R x 512 bf16, 8 chunks
   static constexpr int QR_OFF = Q_OFF + R * 1024;                    // R x 64 bf16
   static constexpr int C_OFF = QR_OFF + ((R * 128 + 1023) / 1024) * 1024;
@@ -71,13 +77,14 @@ struct Cfg {
   static constexpr int MISC_BYTES = 4096;
   static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;          // + alignment slack
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(4 * R + 2 * R <= TMEM_COLS, "tensor memory budget");
+  static_assert(4 * R + 2 * 2 * R <= TMEM_COLS, "tensor memory budget");
 };
 
 template <int R, int NS, int NKR>
 struct Misc {
   uint64_t full[NS], empty[NS], krfull[NKR], krempty[NKR];
-  uint64_t q_full, q_empty, s_full, p_full, o_full, o_empty, drain;
+  uint64_t s_full[2], s_empty[2];
+  uint64_t q_full, q_empty, p_full, pv_done, o_empty, drain;
   uint32_t tmem_base;
   int32_t abort_flag;
   Cursor cursor;
@@ -231,11 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     }
     mbar_init(smem_u32(&ms.q_full), 1);
     mbar_init(smem_u32(&ms.q_empty), 1);
-    mbar_init(smem_u32(&ms.s_full), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ms.s_full[b]), 1);
+      mbar_init(smem_u32(&ms.s_empty[b]), kSoftThreads);
+    }
     mbar_init(smem_u32(&ms.p_full), kSoftThreads);
-    mbar_init(smem_u32(&ms.o_full), 1);
+    mbar_init(smem_u32(&ms.pv_done), 1);
     mbar_init(smem_u32(&ms.o_empty), kSoftThreads);
-    mbar_init(smem_u32(&ms.drain), 1);
+    mbar_init(smem_u32(&ms.drain), 2);     // one commit from each MMA issuer
     ms.abort_flag = 0;
     mbar_fence_init();
   }
@@ -329,13 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       }
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, R, false, false);
-      constexpr uint32_t idPV = idesc_bf16(128, R, true, true);
-      // P^T is stored token-major (MN-major B): rows of 2R bytes, swizzled with the matching width
-      constexpr uint32_t kPswz = (R == 16) ? 6u : (R == 32) ? 4u : 2u;   // 32 / 64 / 128-byte swizzle
-      const uint32_t tS = tmem + 4 * R, tSR = tmem + 5 * R;
+      const uint64_t dC = smem_desc(sb + C::C_OFF, 16, 1024);
+      const uint64_t dQ = smem_desc(sb + C::Q_OFF, 16, 1024);
+      const uint64_t dKR = smem_desc(sb + C::KR_OFF, 16, 1024);
+      const uint64_t dQR = smem_desc(sb + C::QR_OFF, 16, 1024);
       int64_t c_it = 0, k_it = 0, tile_n = 0;
       int n_item = 0;
       bool ok = true;
@@ -344,59 +354,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         tc_fence_after();
         const int ntiles = (it.p1 - it.p0 + 1) / 2;
         for (int i = 0; i < ntiles && ok; ++i) {
-          const int np = min(2, it.p1 - (it.p0 + 2 * i));
-          const int64_t c_first = c_it;
+          // S buffer b was last read by the softmax of tile tile_n - 2
+          const int b = (int)(tile_n & 1);
+          if (!mbar_wait(smem_u32(&ms.s_empty[b]), ((tile_n >> 1) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t tS = tmem + 4 * R + b * 2 * R;
           // S^T = C . Q~^T over the 8 latent chunks, two chunks per ring slot
           for (int m = 0; m < kSlotsPerTile; ++m) {
             const int slot = (int)(c_it % NS);
             if (!mbar_wait(smem_u32(&ms.full[slot]), (c_it / NS) & 1, a.wait_limit)) { ok = false; break; }
             tc_fence_after();
+            const uint64_t a0 = dC + (uint64_t)((slot * kSlotBytes) >> 4);
+            const uint64_t b0 = dQ + (uint64_t)((2 * m * R * 128) >> 4);
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int k = 2 * m + j;
-              const uint32_t abase = sb + C::C_OFF + slot * kSlotBytes + j * kChunkBytes;
-              const uint32_t bbase = sb + C::Q_OFF + k * R * 128;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tS, smem_desc(abase + kk * 32, 16, 1024), smem_desc(bbase + kk * 32, 16, 1024), idS,
-                         (k | kk) != 0);
+            for (int u = 0; u < 8; ++u) {   // chunk u / 4 of the slot, K step u % 4 (32 bytes) inside it
+              const uint32_t aoff = (uint32_t)(((u >> 2) * kChunkBytes + (u & 3) * 32) >> 4);
+              const uint32_t boff = (uint32_t)(((u >> 2) * R * 128 + (u & 3) * 32) >> 4);
+              mma_bf16(tS, a0 + aoff, b0 + boff, idS, (m | u) != 0 ? 1u : 0u);
             }
             ++c_it;
           }
           if (!ok) break;
+          // S_R^T = K^R . Q^R^T
           const int ks = (int)(k_it % NKR);
           if (!mbar_wait(smem_u32(&ms.krfull[ks]), (k_it / NKR) & 1, a.wait_limit)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t krbase = sb + C::KR_OFF + ks * kChunkBytes;
+          const uint64_t akr = dKR + (uint64_t)((ks * kChunkBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tSR, smem_desc(krbase + kk * 32, 16, 1024), smem_desc(sb + C::QR_OFF + kk * 32, 16, 1024),
-                     idS, kk != 0);
-          mma_commit(smem_u32(&ms.s_full));
-          if (i == ntiles - 1) mma_commit(smem_u32(&ms.q_empty));
-          // O^T += C^T . P^T, once the softmax has written P^T into the RoPE-key slot
-          if (i == 0 && !mbar_wait(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
-          if (!mbar_wait(smem_u32(&ms.p_full), tile_n & 1, a.wait_limit)) { ok = false; break; }
-          tc_fence_after();
-          const int nkk = np * 4;   // 16-token K steps that hold real pages
-          for (int m = 0; m < kSlotsPerTile; ++m) {
-            const int s0 = (int)((c_first + m) % NS);
-            const uint32_t abase = sb + C::C_OFF + s0 * kSlotBytes;
-            for (int kk = 0; kk < nkk; ++kk) {
-              // A = C^T of latent block m (MN-major: the two chunks of the slot are LBO apart)
-              const uint64_t ad = smem_desc(abase + kk * 2048, kChunkBytes, 1024);
-              // B = P^T rows 16kk..16kk+15 (MN-major, 2R-byte rows, SBO = eight rows)
-              const uint64_t bd = smem_desc_sw(krbase + kk * 32 * R, 16, 16 * R, kPswz);
-              mma_bf16(tmem + m * R, ad, bd, idPV, (i > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(smem_u32(&ms.empty[s0]));
-          }
-          mma_commit(smem_u32(&ms.krempty[ks]));
+          for (int kk = 0; kk < 4; ++kk) mma_bf16(tS + R, akr + 2 * kk, dQR + 2 * kk, idS, kk != 0 ? 1u : 0u);
+          mma_commit(smem_u32(&ms.s_full[b]));
           ++k_it;
           ++tile_n;
         }
         if (!ok) break;
-        mma_commit(smem_u32(&ms.o_full));
+        mma_commit(smem_u32(&ms.q_empty));
         ++n_item;
       }
       if (!ok) {
@@ -404,6 +395,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         ms.abort_flag = 1;
       }
       // every MMA issued so far must finish before the tensor memory is freed
+      mma_commit(smem_u32(&ms.drain));
+      mbar_wait(smem_u32(&ms.drain), 0, kDrainLimit);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ output MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idPV = idesc_bf16(128, R, true, true);
+      // P^T is stored token-major (MN-major B): rows of 2R bytes, swizzled with the matching width
+      constexpr uint32_t kPswz = (R == 16) ? 6u : (R == 32) ? 4u : 2u;   // 32 / 64 / 128-byte swizzle
+      // A = C^T of one latent block (MN-major: the two chunks of a slot are LBO apart)
+      const uint64_t dCt = smem_desc(sb + C::C_OFF, kChunkBytes, 1024);
+      // B = P^T (MN-major, 2R-byte rows, SBO = eight rows)
+      const uint64_t dP = smem_desc_sw(sb + C::KR_OFF, 16, 16 * R, kPswz);
+      int64_t c_it = 0, k_it = 0, tile_n = 0;
+      int n_item = 0;
+      bool ok = true;
+      while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+        const int ntiles = (it.p1 - it.p0 + 1) / 2;
+        for (int i = 0; i < ntiles && ok; ++i) {
+          const int np = min(2, it.p1 - (it.p0 + 2 * i));
+          // O^T of the previous item must have been read out before it is overwritten
+          if (i == 0 && !mbar_wait(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&ms.p_full), tile_n & 1, a.wait_limit)) { ok = false; break; }
+          tc_fence_after();
+          const int ks = (int)(k_it % NKR);
+          const uint64_t bP = dP + (uint64_t)((ks * kChunkBytes) >> 4);
+          const int nkk = np * 4;   // 16-token K steps that hold real pages
+          for (int m = 0; m < kSlotsPerTile; ++m) {
+            const int s0 = (int)(c_it % NS);
+            const uint64_t a0 = dCt + (uint64_t)((s0 * kSlotBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              if (kk < nkk)
+                mma_bf16(tmem + m * R, a0 + (uint64_t)((kk * 2048) >> 4), bP + (uint64_t)((kk * 32 * R) >> 4), idPV,
+                         (i > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(smem_u32(&ms.empty[s0]));
+            ++c_it;
+          }
+          mma_commit(smem_u32(&ms.krempty[ks]));
+          mma_commit(smem_u32(&ms.pv_done));
+          ++k_it;
+          ++tile_n;
+        }
+        if (!ok) break;
+        ++n_item;
+      }
+      if (!ok) {
+        record_status(a.status, QKN_ERR_TIMEOUT);
+        ms.abort_flag = 1;
+      }
       mma_commit(smem_u32(&ms.drain));
       mbar_wait(smem_u32(&ms.drain), 0, kDrainLimit);
     }
@@ -436,8 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const int tok0 = (it.p0 + 2 * i) * 64;
         const int nvalid = min(np * 64, it.L - tok0);
         const int ks = (int)(k_it % NKR);
+        const int sbuf = (int)(tile_n & 1);
+        const uint32_t tSc = tl + 4 * R + sbuf * 2 * R;   // this tile's S^T columns; S_R^T follows at + R
         bool got = true;
-        if (t == 0) got = mbar_wait(smem_u32(&ms.s_full), tile_n & 1, a.wait_limit);
+        if (t == 0) got = mbar_wait(smem_u32(&ms.s_full[sbuf]), (tile_n >> 1) & 1, a.wait_limit);
         if (!group_all(got)) { ok = false; break; }
         tc_fence_after();
         float ak0 = 1.f;
@@ -455,8 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
 #pragma unroll
           for (int c0 = 0; c0 < R; c0 += 16) {
             uint32_t sc[16], sr[16];
-            tmem_ld16(tl + 4 * R + c0, sc);
-            tmem_ld16(tl + 5 * R + c0, sr);
+            tmem_ld16(tSc + c0, sc);
+            tmem_ld16(tSc + R + c0, sr);
             float aq[16];
             int ql[16];
 #pragma unroll
@@ -498,8 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
 #pragma unroll
         for (int c0 = 0; c0 < R; c0 += 16) {
           uint32_t sc[16], sr[16];
-          tmem_ld16(tl + 4 * R + c0, sc);
-          tmem_ld16(tl + 5 * R + c0, sr);
+          tmem_ld16(tSc + c0, sc);
+          tmem_ld16(tSc + R + c0, sr);
           float aq[16], mu[16], cr[16];
           int ql[16];
 #pragma unroll
@@ -532,6 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           *reinterpret_cast<uint4*>(prow + (((u0 + 0) ^ swz) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ swz) << 4)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
+        // the S buffer is free for the tile after next
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ms.s_empty[sbuf]));
         // rows of real pages past the context: zero them so that 0 * garbage cannot reach O
         if (!row_ok && t < np * 64) {
 #pragma unroll
@@ -542,6 +588,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
             for (int q = 0; q < 8; ++q) rowp[q] = make_uint4(0, 0, 0, 0);
           }
         }
+        // the output MMAs of the previous tile must be complete before O^T is rescaled (and,
+        // waited for every tile, this keeps the barrier's phases in step)
+        got = true;
+        if (t == 0 && tile_n > 0) got = mbar_wait(smem_u32(&ms.pv_done), (tile_n - 1) & 1, a.wait_limit);
+        if (!group_all(got)) { ok = false; break; }
+        tc_fence_after();
         if (rescale) {
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
@@ -567,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       if (!ok) break;
       // ---------------- epilogue: O / l and lse for this item
       bool got = true;
-      if (t == 0) got = mbar_wait(smem_u32(&ms.o_full), n_item & 1, a.wait_limit);
+      if (t == 0) got = mbar_wait(smem_u32(&ms.pv_done), (tile_n - 1) & 1, a.wait_limit);
       if (!group_all(got)) { ok = false; break; }
       tc_fence_after();
       warp_col_reduce<R, false>(lpart, lane);
