@@ -7,30 +7,35 @@
 //   l[t, rho] = a_q[rho] * a_k[t, g(rho)] * (c_t . q~[rho]) + k^R^_t . q^R^[rho]
 // then an online softmax over the CTA's token range and O = sum_t p * c_t.
 //
-// Orientation ("swap AB"): tokens are the MMA M dimension (128 per tile = two
-// 64-token pages) and query rows are N (R = 16, 32 or 64), so one tile is
-//   S^T[128 x R]  = C[128 x 512] . Q~^T            (K = latent, 32 MMAs)
-//   S_R^T[128 x R] = K^R[128 x 64] . Q^R^T          (K = RoPE,   4 MMAs)
-//   O^T[512 x R] += C^T[512 x 128] . P^T[128 x R]   (4 latent blocks x 8 MMAs)
-// with the latent tile C staged once in shared memory and read by both
-// products (as K-major A for S, as MN-major A for O).  The fp32 accumulator
-// O^T takes 4R TMEM columns; S^T and S_R^T take R columns each and are double
-// buffered, so that the scores of tile i+1 are computed while the softmax and
-// the output product of tile i run.
+// Orientation ("swap AB"): tokens are the MMA M dimension and query rows are
+// N (R = 16, 32 or 64).  A tile is one 64-token cache page:
+//   S^T[64 x R]   = C[64 x 512] . Q~^T            (K = latent, 32 MMAs, M = 64)
+//   S_R^T[64 x R] = K^R[64 x 64] . Q^R^T          (K = RoPE,   4 MMAs, M = 64)
+//   O^T[512 x R] += C^T[512 x 64] . P^T[64 x R]   (4 latent blocks x 4 MMAs, M = 128)
+// with the page's latent staged once in shared memory and read by both
+// products (as K-major A for S, as MN-major A for O).  One page (72 KB with
+// its RoPE key) is small enough that two to three pages stay resident, so
+// the loads of the next pages run while the softmax and the output product
+// of the current page hold theirs.
+//
+// Tensor memory: O^T takes 4R columns over all 128 lanes; S^T and S_R^T take
+// R columns each in the 64-row layout (token m in lane (m % 16) + 32 (m / 16))
+// and are double buffered, so that the scores of page i+1 are computed while
+// the softmax and the output product of page i run.
 //
 // Warp roles (224 threads, one CTA per SM):
-//   warps 0-3  softmax + epilogue: thread t owns TMEM lane t = token row t of
-//              S^T and latent row t of each O^T block; column (query row)
-//              maxima and sums are reduced across the 128 threads;
-//   warp 4     TMA producer: query tiles per item, then per tile eight 16 KB
-//              latent chunks, the RoPE-key chunk and the a_k rows;
+//   warps 0-3  softmax + epilogue: lane i < 16 of warp w owns token 16w + i
+//              of a page (its TMEM lane); thread t owns latent row t of each
+//              O^T block; column (query row) maxima and sums are reduced
+//              across the 128 threads;
+//   warp 4     TMA producer: query tiles per item, then per page four 16 KB
+//              latent slots, the RoPE-key chunk and the a_k rows; the whole
+//              warp reads the block table 32 entries at a time;
 //   warp 5     TMEM allocator and issuer of the score MMAs (S^T, S_R^T);
 //   warp 6     issuer of the output MMAs (O^T).
 // A single thread issues tcgen05.mma at a bounded rate, so the two products
 // have one issuing thread each, and every shared-memory descriptor is built
 // once: a K step or a ring slot only moves its start-address field.
-// Shared-memory rings: latent chunks (full/empty mbarrier pairs), and a
-// RoPE-key slot that the softmax reuses for P^T once the RoPE MMAs are done.
 // Every mbarrier wait is bounded; a wait that runs out records
 // QKN_ERR_TIMEOUT in the workspace status word and the CTA winds down.
 #include <cuda.h>
@@ -45,37 +50,40 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kTile = 128;                 // tokens per tile (MMA M)
-constexpr int kRkv = 512;                  // latent width this kernel takes
-constexpr int kChunks = kRkv / 64;         // 64-column (128-byte) chunks of the latent
-constexpr int kDrope = 64;                 // RoPE width this kernel takes
-constexpr int kChunkBytes = kTile * 128;   // one 64-column chunk of one tile: 16 KB
-constexpr int kSlotBytes = 2 * kChunkBytes; // a ring slot holds two chunks (one 128-row latent block): 32 KB
+constexpr int kPage = 64;                   // tokens per tile (one cache page; MMA M of the score product)
+constexpr int kRkv = 512;                   // latent width this kernel takes
+constexpr int kChunks = kRkv / 64;          // 64-column (128-byte) chunks of the latent
+constexpr int kDrope = 64;                  // RoPE width this kernel takes
+constexpr int kChunkBytes = kPage * 128;    // one 64-column chunk of one page: 8 KB
+constexpr int kSlotBytes = 2 * kChunkBytes; // a ring slot holds one 128-column latent block of a page: 16 KB
 constexpr int kSlotsPerTile = kChunks / 2;
-constexpr int kPageChunkBytes = 64 * 128;  // one chunk of one page: 8 KB
+constexpr int kKrBytes = kPage * kDrope * 2;            // RoPE keys of one page: 8 KB
 constexpr int kMaxGroups = 8;
-constexpr int kAkSlotBytes = kTile * kMaxGroups * 4;
+constexpr int kAkSlotBytes = kPage * kMaxGroups * 4;    // a_k rows of one page: up to 2 KB
 constexpr int kThreads = 224;
 constexpr int kSoftThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleLog2 = 8.0f;       // rescale O only when a column max grows by > 2^8
+constexpr float kRescaleLog2 = 8.0f;        // rescale O only when a column max grows by > 2^8
 constexpr int64_t kDrainLimit = 4000000000LL;
-constexpr int kPrefetchPages = 6;          // pages the L2 prefetch runs ahead of the TMA loads
+constexpr int kPrefetchPages = 4;          // pages the L2 prefetch runs ahead of the TMA loads
 
 template <int R>
 struct Cfg {
-  static constexpr int NS = (R == 64) ? 4 : 5;               // latent ring slots (two chunks each)
-  static constexpr int NKR = (R == 16) ? 2 : 1;              // RoPE-key / P^T slots
+  static constexpr int NKR = (R == 64) ? 3 : 4;              // RoPE-key / a_k / P^T slots
   static constexpr int TMEM_COLS = (8 * R <= 128) ? 128 : (8 * R <= 256 ? 256 : 512);
   static constexpr int Q_OFF = 0;                                    // R x 512 bf16, 8 chunks
   static constexpr int QR_OFF = Q_OFF + R * 1024;                    // R x 64 bf16
-  static constexpr int C_OFF = QR_OFF + ((R * 128 + 1023) / 1024) * 1024;
-  static constexpr int KR_OFF = C_OFF + NS * kSlotBytes;
-  static constexpr int AK_OFF = KR_OFF + NKR * kChunkBytes;
+  static constexpr int KR_OFF = QR_OFF + ((R * 128 + 1023) / 1024) * 1024;
+  static constexpr int AK_OFF = KR_OFF + NKR * kKrBytes;
   static constexpr int MISC_OFF = AK_OFF + NKR * kAkSlotBytes;
   static constexpr int MISC_BYTES = 4096;
-  static constexpr int SMEM = MISC_OFF + MISC_BYTES + 1024;          // + alignment slack
+  static constexpr int C_OFF = MISC_OFF + MISC_BYTES;                // 1024-aligned: every term above is
+  static constexpr int kBudget = 232448 - 1024;                      // opt-in maximum less alignment slack
+  static constexpr int NS = (kBudget - C_OFF) / kSlotBytes;          // latent ring slots (one block of a page each)
+  static constexpr int SMEM = C_OFF + NS * kSlotBytes + 1024;
+  static_assert(C_OFF % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+  static_assert(NS >= kSlotsPerTile + 2, "the ring must hold more than one page");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(4 * R + 2 * 2 * R <= TMEM_COLS, "tensor memory budget");
 };
@@ -84,7 +92,12 @@ template <int R, int NS, int NKR>
 struct Misc {
   uint64_t full[NS], empty[NS], krfull[NKR], krempty[NKR];
   uint64_t s_full[2], s_empty[2];
-  uint64_t q_full, q_empty, p_full, pv_done, o_empty, drain;
+  // Per-tile handshakes alternate between two barriers by tile parity (tile n: barrier n & 1,
+  // phase n >> 1): the softmax may run two tiles ahead of the output issuer, and a parity wait
+  // needs the barrier to be at most one phase past the phase waited for.
+  uint64_t p_full[2];             // P^T of tile n written
+  uint64_t pv_done[2];            // output MMAs of tile n complete
+  uint64_t q_full, q_empty, o_empty, drain;
   uint32_t tmem_base;
   int32_t abort_flag;
   Cursor cursor;
@@ -174,42 +187,6 @@ __device__ __forceinline__ bool group_any(bool v) {
   return r != 0;
 }
 
-// Walks the pages of one CTA's items, in load order, issuing L2 prefetches
-// for the latent, RoPE-key and a_k rows of each page.  The producer keeps it
-// a fixed number of pages ahead of its TMA loads, so that HBM streaming does
-// not wait for shared-memory ring slots to free up.
-struct PrefetchWalker {
-  Cursor cur;
-  Item it;
-  int32_t page;     // next page of `it` to prefetch
-  bool live;        // an item is open
-  bool done;        // no items left
-
-  __device__ __forceinline__ void init(const Cursor& c) {
-    cur = c;
-    live = false;
-    done = false;
-  }
-  template <bool AK_ONE>
-  __device__ __forceinline__ void step(const DecodeArgs& a, const SchedParams& sp, int cta) {
-    if (done) return;
-    if (!live || page >= it.p1) {
-      if (!sched_next(cur, sp, cta, it)) {
-        done = true;
-        return;
-      }
-      live = true;
-      page = it.p0;
-    }
-    const int32_t blk = a.block_table[(int64_t)it.b * a.max_blocks + page];
-    ++page;
-    if (blk < 0 || blk >= a.num_blocks) return;
-    prefetch_l2(static_cast<const __nv_bfloat16*>(a.latent) + (int64_t)blk * 64 * kRkv, 64 * kRkv * 2);
-    prefetch_l2(static_cast<const __nv_bfloat16*>(a.k_rope) + (int64_t)blk * 64 * kDrope, 64 * kDrope * 2);
-    if (!AK_ONE) prefetch_l2(a.a_k + (int64_t)blk * 64 * a.groups, 64u * a.groups * 4u);
-  }
-};
-
 template <int R, bool AK_ONE>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TcMaps maps) {
   using C = Cfg<R>;
@@ -236,14 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       mbar_init(smem_u32(&ms.krfull[s]), 1);
       mbar_init(smem_u32(&ms.krempty[s]), 1);
     }
-    mbar_init(smem_u32(&ms.q_full), 1);
-    mbar_init(smem_u32(&ms.q_empty), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&ms.s_full[b]), 1);
       mbar_init(smem_u32(&ms.s_empty[b]), kSoftThreads);
+      mbar_init(smem_u32(&ms.pv_done[b]), 1);
+      mbar_init(smem_u32(&ms.p_full[b]), kSoftThreads);
     }
-    mbar_init(smem_u32(&ms.p_full), kSoftThreads);
-    mbar_init(smem_u32(&ms.pv_done), 1);
+    mbar_init(smem_u32(&ms.q_full), 1);
+    mbar_init(smem_u32(&ms.q_empty), 1);
     mbar_init(smem_u32(&ms.o_empty), kSoftThreads);
     mbar_init(smem_u32(&ms.drain), 2);     // one commit from each MMA issuer
     ms.abort_flag = 0;
@@ -274,186 +251,196 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
   Item it;
 
   if (warp == 4) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int64_t c_it = 0, k_it = 0;
-      int n_item = 0;
-      bool ok = true;
-      PrefetchWalker pf;
-      pf.init(cur);
-      for (int i = 0; i < kPrefetchPages; ++i) pf.step<AK_ONE>(a, sp, blockIdx.x);
-      while (ok && sched_next(cur, sp, blockIdx.x, it)) {
-        if (!mbar_wait(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+    // ------------------------------------------------------------ producer (whole warp, elected issue)
+    RingPos<NS> cw;
+    RingPos<NKR> kw;
+    int64_t c_issued = 0, k_issued = 0;
+    int n_item = 0;
+    bool ok = true;
+    const uint32_t akpage = (uint32_t)kPage * (uint32_t)G * 4u;
+    auto prefetch_page = [&](int32_t blk) {
+      prefetch_l2(static_cast<const __nv_bfloat16*>(a.latent) + (int64_t)blk * kPage * kRkv, kPage * kRkv * 2);
+      prefetch_l2(static_cast<const __nv_bfloat16*>(a.k_rope) + (int64_t)blk * kPage * kDrope, kKrBytes);
+      if (!AK_ONE) prefetch_l2(a.a_k + (int64_t)blk * kPage * G, akpage);
+    };
+    while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+      if (!mbar_wait_warp(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+      {
         const int qrow0 = it.b * qrows + it.ht * R;
         const uint32_t qf = smem_u32(&ms.q_full);
-        mbar_arrive_expect_tx(qf, R * 1024 + R * 128);
+        mbar_arrive_expect_tx_elect(qf, R * 1024 + R * 128);
 #pragma unroll
-        for (int k = 0; k < kChunks; ++k) tma_load_2d(sb + C::Q_OFF + k * R * 128, &maps.qt, k * 64, qrow0, qf);
-        tma_load_2d(sb + C::QR_OFF, &maps.qr, 0, qrow0, qf);
-        const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
-        for (int p = it.p0; p < it.p1 && ok; p += 2) {
-          const int np = min(2, it.p1 - p);
-          for (int i = 0; i < np; ++i) pf.step<AK_ONE>(a, sp, blockIdx.x);
-          int32_t blk[2] = {row[p], np > 1 ? row[p + 1] : 0};
-          for (int i = 0; i < np; ++i)
-            if (blk[i] < 0 || blk[i] >= a.num_blocks) {
-              record_status(a.status, QKN_ERR_BOUNDS);
-              blk[i] = 0;
-            }
+        for (int k = 0; k < kChunks; ++k) tma_load_2d_elect(sb + C::Q_OFF + k * R * 128, &maps.qt, k * 64, qrow0, qf);
+        tma_load_2d_elect(sb + C::QR_OFF, &maps.qr, 0, qrow0, qf);
+      }
+      const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
+      for (int pb = it.p0; pb < it.p1 && ok; pb += 32) {
+        // 32 block-table entries per warp-wide load
+        int32_t mine = 0;
+        if (pb + lane < it.p1) {
+          mine = row[pb + lane];
+          if (mine < 0 || mine >= a.num_blocks) {
+            record_status(a.status, QKN_ERR_BOUNDS);
+            mine = 0;
+          }
+        }
+        const int cnt = min(32, it.p1 - pb);
+        // L2 prefetch runs kPrefetchPages ahead of the TMA loads, which wait for ring slots
+        if (lane < min(cnt, kPrefetchPages)) prefetch_page(mine);
+        for (int k = 0; k < cnt && ok; ++k) {
+          const int32_t blk = __shfl_sync(0xffffffffu, mine, k);
+          const int32_t ahead = __shfl_sync(0xffffffffu, mine, min(k + kPrefetchPages, 31));
+          if (lane == 0 && k + kPrefetchPages < cnt) prefetch_page(ahead);
+          __syncwarp();
           for (int m = 0; m < kSlotsPerTile; ++m) {
-            const int slot = (int)(c_it % NS);
-            if (!mbar_wait(smem_u32(&ms.empty[slot]), ((c_it / NS) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
-            const uint32_t fb = smem_u32(&ms.full[slot]);
-            mbar_arrive_expect_tx(fb, 2 * np * kPageChunkBytes);
-            const uint32_t dst = sb + C::C_OFF + slot * kSlotBytes;
-            for (int j = 0; j < 2; ++j)
-              for (int i = 0; i < np; ++i)
-                tma_load_2d(dst + j * kChunkBytes + i * kPageChunkBytes, &maps.latent, (2 * m + j) * 64, blk[i] * 64, fb);
-            ++c_it;
+            if (!mbar_wait_warp(smem_u32(&ms.empty[cw.slot]), cw.phase ^ 1u, a.wait_limit)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&ms.full[cw.slot]);
+            mbar_arrive_expect_tx_elect(fb, kSlotBytes);
+            const uint32_t dst = sb + C::C_OFF + cw.slot * kSlotBytes;
+            tma_load_2d_elect(dst, &maps.latent, (2 * m) * 64, blk * kPage, fb);
+            tma_load_2d_elect(dst + kChunkBytes, &maps.latent, (2 * m + 1) * 64, blk * kPage, fb);
+            cw.next();
+            ++c_issued;
           }
           if (!ok) break;
-          const int ks = (int)(k_it % NKR);
-          if (!mbar_wait(smem_u32(&ms.krempty[ks]), ((k_it / NKR) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
-          const uint32_t kb = smem_u32(&ms.krfull[ks]);
-          const uint32_t akpage = 64u * (uint32_t)G * 4u;
-          mbar_arrive_expect_tx(kb, np * kPageChunkBytes + (AK_ONE ? 0u : np * akpage));
-          for (int i = 0; i < np; ++i) {
-            tma_load_2d(sb + C::KR_OFF + ks * kChunkBytes + i * kPageChunkBytes, &maps.krope, 0, blk[i] * 64, kb);
-            if (!AK_ONE)
-              bulk_load(sb + C::AK_OFF + ks * kAkSlotBytes + i * akpage, a.a_k + (int64_t)blk[i] * 64 * G, akpage, kb);
-          }
-          ++k_it;
+          if (!mbar_wait_warp(smem_u32(&ms.krempty[kw.slot]), kw.phase ^ 1u, a.wait_limit)) { ok = false; break; }
+          const uint32_t kb = smem_u32(&ms.krfull[kw.slot]);
+          mbar_arrive_expect_tx_elect(kb, kKrBytes + (AK_ONE ? 0u : akpage));
+          tma_load_2d_elect(sb + C::KR_OFF + kw.slot * kKrBytes, &maps.krope, 0, blk * kPage, kb);
+          if (!AK_ONE)
+            bulk_load_elect(sb + C::AK_OFF + kw.slot * kAkSlotBytes, a.a_k + (int64_t)blk * kPage * G, akpage, kb);
+          kw.next();
+          ++k_issued;
         }
-        ++n_item;
       }
-      if (!ok) {
-        record_status(a.status, QKN_ERR_TIMEOUT);
-        ms.abort_flag = 1;
-        // let the copies already in flight land before the CTA's memory is released
-        const int64_t first = c_it > NS ? c_it - NS : 0;
-        for (int64_t i = first; i < c_it; ++i)
-          mbar_wait(smem_u32(&ms.full[i % NS]), (i / NS) & 1, kDrainLimit);
-        const int64_t kfirst = k_it > NKR ? k_it - NKR : 0;
-        for (int64_t i = kfirst; i < k_it; ++i)
-          mbar_wait(smem_u32(&ms.krfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
-      }
+      ++n_item;
+    }
+    if (!ok && lane == 0) {
+      record_status(a.status, QKN_ERR_TIMEOUT);
+      ms.abort_flag = 1;
+      // let the copies already in flight land before the CTA's memory is released
+      const int64_t first = c_issued > NS ? c_issued - NS : 0;
+      for (int64_t i = first; i < c_issued; ++i)
+        mbar_wait(smem_u32(&ms.full[i % NS]), (i / NS) & 1, kDrainLimit);
+      const int64_t kfirst = k_issued > NKR ? k_issued - NKR : 0;
+      for (int64_t i = kfirst; i < k_issued; ++i)
+        mbar_wait(smem_u32(&ms.krfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------ score MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, R, false, false);
-      const uint64_t dC = smem_desc(sb + C::C_OFF, 16, 1024);
-      const uint64_t dQ = smem_desc(sb + C::Q_OFF, 16, 1024);
-      const uint64_t dKR = smem_desc(sb + C::KR_OFF, 16, 1024);
-      const uint64_t dQR = smem_desc(sb + C::QR_OFF, 16, 1024);
-      int64_t c_it = 0, k_it = 0, tile_n = 0;
-      int n_item = 0;
-      bool ok = true;
-      while (ok && sched_next(cur, sp, blockIdx.x, it)) {
-        if (!mbar_wait(smem_u32(&ms.q_full), n_item & 1, a.wait_limit)) { ok = false; break; }
+    // ------------------------------------------------------------ score MMA issuer (whole warp)
+    constexpr uint32_t idS = idesc_bf16(kPage, R, false, false);
+    const uint64_t dC = smem_desc(sb + C::C_OFF, 16, 1024);
+    const uint64_t dQ = smem_desc(sb + C::Q_OFF, 16, 1024);
+    const uint64_t dKR = smem_desc(sb + C::KR_OFF, 16, 1024);
+    const uint64_t dQR = smem_desc(sb + C::QR_OFF, 16, 1024);
+    RingPos<NS> cr;
+    RingPos<NKR> kr;
+    RingPos<2> sbuf;          // S buffer of the tile, and the phase of its use
+    int n_item = 0;
+    bool ok = true;
+    while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+      if (!mbar_wait_warp(smem_u32(&ms.q_full), n_item & 1, a.wait_limit)) { ok = false; break; }
+      tc_fence_after();
+      for (int p = it.p0; p < it.p1 && ok; ++p) {
+        // S buffer b was last read by the softmax of the tile two back
+        const int b = sbuf.slot;
+        if (!mbar_wait_warp(smem_u32(&ms.s_empty[b]), sbuf.phase ^ 1u, a.wait_limit)) { ok = false; break; }
         tc_fence_after();
-        const int ntiles = (it.p1 - it.p0 + 1) / 2;
-        for (int i = 0; i < ntiles && ok; ++i) {
-          // S buffer b was last read by the softmax of tile tile_n - 2
-          const int b = (int)(tile_n & 1);
-          if (!mbar_wait(smem_u32(&ms.s_empty[b]), ((tile_n >> 1) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+        const uint32_t tS = tmem + 4 * R + b * 2 * R;
+        // S^T = C . Q~^T over the 8 latent chunks, two chunks per ring slot
+        for (int m = 0; m < kSlotsPerTile; ++m) {
+          if (!mbar_wait_warp(smem_u32(&ms.full[cr.slot]), cr.phase, a.wait_limit)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t tS = tmem + 4 * R + b * 2 * R;
-          // S^T = C . Q~^T over the 8 latent chunks, two chunks per ring slot
-          for (int m = 0; m < kSlotsPerTile; ++m) {
-            const int slot = (int)(c_it % NS);
-            if (!mbar_wait(smem_u32(&ms.full[slot]), (c_it / NS) & 1, a.wait_limit)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t a0 = dC + (uint64_t)((slot * kSlotBytes) >> 4);
-            const uint64_t b0 = dQ + (uint64_t)((2 * m * R * 128) >> 4);
+          const uint64_t a0 = dC + (uint64_t)(cr.slot * (kSlotBytes >> 4));
+          const uint64_t b0 = dQ + (uint64_t)(m * ((2 * R * 128) >> 4));
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {   // chunk u / 4 of the slot, K step u % 4 (32 bytes) inside it
-              const uint32_t aoff = (uint32_t)(((u >> 2) * kChunkBytes + (u & 3) * 32) >> 4);
-              const uint32_t boff = (uint32_t)(((u >> 2) * R * 128 + (u & 3) * 32) >> 4);
-              mma_bf16(tS, a0 + aoff, b0 + boff, idS, (m | u) != 0 ? 1u : 0u);
-            }
-            ++c_it;
+          for (int u = 0; u < 8; ++u) {   // chunk u / 4 of the slot, K step u % 4 (32 bytes) inside it
+            const uint32_t aoff = (uint32_t)(((u >> 2) * kChunkBytes + (u & 3) * 32) >> 4);
+            const uint32_t boff = (uint32_t)(((u >> 2) * R * 128 + (u & 3) * 32) >> 4);
+            mma_bf16_elect(tS, a0 + aoff, b0 + boff, idS, (m | u) != 0 ? 1u : 0u);
           }
-          if (!ok) break;
-          // S_R^T = K^R . Q^R^T
-          const int ks = (int)(k_it % NKR);
-          if (!mbar_wait(smem_u32(&ms.krfull[ks]), (k_it / NKR) & 1, a.wait_limit)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t akr = dKR + (uint64_t)((ks * kChunkBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_bf16(tS + R, akr + 2 * kk, dQR + 2 * kk, idS, kk != 0 ? 1u : 0u);
-          mma_commit(smem_u32(&ms.s_full[b]));
-          ++k_it;
-          ++tile_n;
+          cr.next();
         }
         if (!ok) break;
-        mma_commit(smem_u32(&ms.q_empty));
-        ++n_item;
+        // S_R^T = K^R . Q^R^T
+        if (!mbar_wait_warp(smem_u32(&ms.krfull[kr.slot]), kr.phase, a.wait_limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t akr = dKR + (uint64_t)(kr.slot * (kKrBytes >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_elect(tS + R, akr + 2 * kk, dQR + 2 * kk, idS, kk != 0 ? 1u : 0u);
+        mma_commit_elect(smem_u32(&ms.s_full[b]));
+        kr.next();
+        sbuf.next();
       }
-      if (!ok) {
-        record_status(a.status, QKN_ERR_TIMEOUT);
-        ms.abort_flag = 1;
-      }
-      // every MMA issued so far must finish before the tensor memory is freed
-      mma_commit(smem_u32(&ms.drain));
-      mbar_wait(smem_u32(&ms.drain), 0, kDrainLimit);
+      if (!ok) break;
+      mma_commit_elect(smem_u32(&ms.q_empty));
+      ++n_item;
     }
+    if (!ok && lane == 0) {
+      record_status(a.status, QKN_ERR_TIMEOUT);
+      ms.abort_flag = 1;
+    }
+    // every MMA issued so far must finish before the tensor memory is freed
+    mma_commit_elect(smem_u32(&ms.drain));
+    mbar_wait_warp(smem_u32(&ms.drain), 0, kDrainLimit);
   } else if (warp == 6) {
-    // ------------------------------------------------------------ output MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idPV = idesc_bf16(128, R, true, true);
-      // P^T is stored token-major (MN-major B): rows of 2R bytes, swizzled with the matching width
-      constexpr uint32_t kPswz = (R == 16) ? 6u : (R == 32) ? 4u : 2u;   // 32 / 64 / 128-byte swizzle
-      // A = C^T of one latent block (MN-major: the two chunks of a slot are LBO apart)
-      const uint64_t dCt = smem_desc(sb + C::C_OFF, kChunkBytes, 1024);
-      // B = P^T (MN-major, 2R-byte rows, SBO = eight rows)
-      const uint64_t dP = smem_desc_sw(sb + C::KR_OFF, 16, 16 * R, kPswz);
-      int64_t c_it = 0, k_it = 0, tile_n = 0;
-      int n_item = 0;
-      bool ok = true;
-      while (ok && sched_next(cur, sp, blockIdx.x, it)) {
-        const int ntiles = (it.p1 - it.p0 + 1) / 2;
-        for (int i = 0; i < ntiles && ok; ++i) {
-          const int np = min(2, it.p1 - (it.p0 + 2 * i));
-          // O^T of the previous item must have been read out before it is overwritten
-          if (i == 0 && !mbar_wait(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
-          if (!mbar_wait(smem_u32(&ms.p_full), tile_n & 1, a.wait_limit)) { ok = false; break; }
-          tc_fence_after();
-          const int ks = (int)(k_it % NKR);
-          const uint64_t bP = dP + (uint64_t)((ks * kChunkBytes) >> 4);
-          const int nkk = np * 4;   // 16-token K steps that hold real pages
-          for (int m = 0; m < kSlotsPerTile; ++m) {
-            const int s0 = (int)(c_it % NS);
-            const uint64_t a0 = dCt + (uint64_t)((s0 * kSlotBytes) >> 4);
+    // ------------------------------------------------------------ output MMA issuer (whole warp)
+    constexpr uint32_t idPV = idesc_bf16(128, R, true, true);
+    // P^T is stored token-major (MN-major B): rows of 2R bytes, swizzled with the matching width
+    constexpr uint32_t kPswz = (R == 16) ? 6u : (R == 32) ? 4u : 2u;   // 32 / 64 / 128-byte swizzle
+    // A = C^T of one latent block (MN-major: the two chunks of a slot are LBO apart, 8-token groups SBO apart)
+    const uint64_t dCt = smem_desc(sb + C::C_OFF, kChunkBytes, 1024);
+    // B = P^T (MN-major, 2R-byte rows, SBO = eight rows)
+    const uint64_t dP = smem_desc_sw(sb + C::KR_OFF, 16, 16 * R, kPswz);
+    RingPos<NS> cr;
+    RingPos<NKR> kr;
+    RingPos<2> pb;            // P / output handshake barrier of the tile, and the phase of its use
+    int n_item = 0;
+    bool ok = true;
+    while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+      for (int p = it.p0; p < it.p1 && ok; ++p) {
+        // O^T of the previous item must have been read out before it is overwritten
+        if (p == it.p0 && !mbar_wait_warp(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+        if (!mbar_wait_warp(smem_u32(&ms.p_full[pb.slot]), pb.phase, a.wait_limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t bP = dP + (uint64_t)(kr.slot * (kKrBytes >> 4));
+        const uint32_t acc0 = p > it.p0 ? 1u : 0u;
+        for (int m = 0; m < kSlotsPerTile; ++m) {
+          const uint64_t a0 = dCt + (uint64_t)(cr.slot * (kSlotBytes >> 4));
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              if (kk < nkk)
-                mma_bf16(tmem + m * R, a0 + (uint64_t)((kk * 2048) >> 4), bP + (uint64_t)((kk * 32 * R) >> 4), idPV,
-                         (i > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&ms.empty[s0]));
-            ++c_it;
-          }
-          mma_commit(smem_u32(&ms.krempty[ks]));
-          mma_commit(smem_u32(&ms.pv_done));
-          ++k_it;
-          ++tile_n;
+          for (int kk = 0; kk < kPage / 16; ++kk)
+            mma_bf16_elect(tmem + m * R, a0 + (uint64_t)((kk * 2048) >> 4), bP + (uint64_t)((kk * 32 * R) >> 4), idPV,
+                           kk > 0 ? 1u : acc0);
+          mma_commit_elect(smem_u32(&ms.empty[cr.slot]));
+          cr.next();
         }
-        if (!ok) break;
-        ++n_item;
+        mma_commit_elect(smem_u32(&ms.krempty[kr.slot]));
+        mma_commit_elect(smem_u32(&ms.pv_done[pb.slot]));
+        kr.next();
+        pb.next();
       }
-      if (!ok) {
-        record_status(a.status, QKN_ERR_TIMEOUT);
-        ms.abort_flag = 1;
-      }
-      mma_commit(smem_u32(&ms.drain));
-      mbar_wait(smem_u32(&ms.drain), 0, kDrainLimit);
+      if (!ok) break;
+      ++n_item;
     }
+    if (!ok && lane == 0) {
+      record_status(a.status, QKN_ERR_TIMEOUT);
+      ms.abort_flag = 1;
+    }
+    mma_commit_elect(smem_u32(&ms.drain));
+    mbar_wait_warp(smem_u32(&ms.drain), 0, kDrainLimit);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int t = threadIdx.x;                         // token row / TMEM lane
+    const int t = threadIdx.x;                         // latent row of each O^T block / TMEM lane
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const int tok = warp * 16 + lane;                  // token of the page held in this lane (lane < 16)
+    const bool has_tok = lane < 16;
+    auto pv_wait = [&](int64_t n) {
+      return mbar_wait(smem_u32(&ms.pv_done[n & 1]), (uint32_t)((n >> 1) & 1), a.wait_limit);
+    };
     const int ng = a.heads / G;
-    int64_t c_it = 0, k_it = 0, tile_n = 0;
+    RingPos<NKR> kr;
+    int c_first = 0;          // ring slot of the tile's first latent block
+    int64_t tile_n = 0;
     int n_item = 0;
     bool ok = true;
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
@@ -471,30 +458,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       float lpart[R];
 #pragma unroll
       for (int c = 0; c < R; ++c) lpart[c] = 0.f;
-      const int ntiles = (it.p1 - it.p0 + 1) / 2;
-      for (int i = 0; i < ntiles; ++i) {
-        const int np = min(2, it.p1 - (it.p0 + 2 * i));
-        const int tok0 = (it.p0 + 2 * i) * 64;
-        const int nvalid = min(np * 64, it.L - tok0);
-        const int ks = (int)(k_it % NKR);
+      for (int p = it.p0; p < it.p1; ++p) {
+        const int tok0 = p * kPage;
+        const int nvalid = min(kPage, it.L - tok0);
+        const int ks = kr.slot;
         const int sbuf = (int)(tile_n & 1);
         const uint32_t tSc = tl + 4 * R + sbuf * 2 * R;   // this tile's S^T columns; S_R^T follows at + R
-        bool got = true;
-        if (t == 0) got = mbar_wait(smem_u32(&ms.s_full[sbuf]), (tile_n >> 1) & 1, a.wait_limit);
-        if (!group_all(got)) { ok = false; break; }
+        // every thread waits for the scores itself; the verdicts are pooled at the group vote below
+        bool got = mbar_wait(smem_u32(&ms.s_full[sbuf]), (tile_n >> 1) & 1, a.wait_limit);
+        // output MMAs of two tiles back (normally long complete).  Tile n signals barrier n & 1 in its
+        // phase n >> 1; waiting for every tile two back keeps each barrier at most one phase ahead of
+        // the phase waited for, which a parity wait needs.
+        if (t == 0 && tile_n > 1) got = pv_wait(tile_n - 2) && got;
         tc_fence_after();
+        const bool row_ok = has_tok && tok < nvalid;
+        const int tpos = tok0 + tok;
+        const float* akrow = reinterpret_cast<const float*>(smem + C::AK_OFF + ks * kAkSlotBytes) + (has_tok ? tok : 0) * G;
         float ak0 = 1.f;
-        const float* akrow = reinterpret_cast<const float*>(smem + C::AK_OFF + ks * kAkSlotBytes) + t * G;
         if (!AK_ONE) {
           // the RoPE-key barrier also covers the a_k rows; it completed before S did
-          mbar_wait(smem_u32(&ms.krfull[ks]), (k_it / NKR) & 1, kDrainLimit);
+          got = mbar_wait(smem_u32(&ms.krfull[ks]), kr.phase, a.wait_limit) && got;
           ak0 = akrow[0];
         }
-        const bool row_ok = t < nvalid;
-        const int tpos = tok0 + t;
-        // pass 1: column maxima of this tile
-        {
-          float v[R];
+        // this token's scaled logits in log2 units (-inf where not visible)
+        auto load_logits = [&](float (&x)[R]) {
 #pragma unroll
           for (int c0 = 0; c0 < R; c0 += 16) {
             uint32_t sc[16], sr[16];
@@ -510,49 +497,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
             tmem_wait_ld(sc, sr);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const int c = c0 + e;
               float akc = ak0;
-              if (!AK_ONE && G > 1) akc = akrow[ms.grp[c]];
-              const float x = aq[e] * akc * __uint_as_float(sc[e]) + kLog2e * __uint_as_float(sr[e]);
-              v[c] = (row_ok && tpos <= ql[e]) ? x : -INFINITY;
+              if (!AK_ONE && G > 1) akc = akrow[ms.grp[c0 + e]];
+              const float v = aq[e] * akc * __uint_as_float(sc[e]) + kLog2e * __uint_as_float(sr[e]);
+              x[c0 + e] = (row_ok && tpos <= ql[e]) ? v : -INFINITY;
             }
           }
+        };
+        float x[R];
+        load_logits(x);
+        // Fast path: the exponentials are taken against the running reference mu, which only has
+        // to stay within 2^8 of the true column maximum.  One group vote finds out whether any
+        // logit of the tile passed mu + 8; only then are the column maxima reduced.
+        bool over = false;
+#pragma unroll
+        for (int c0 = 0; c0 < R; c0 += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(ms.mu + c0);
+          over |= (x[c0] > m4.x + kRescaleLog2) | (x[c0 + 1] > m4.y + kRescaleLog2) |
+                  (x[c0 + 2] > m4.z + kRescaleLog2) | (x[c0 + 3] > m4.w + kRescaleLog2);
+        }
+        if (group_any(over || !got)) {
+          if (group_any(!got)) { ok = false; break; }
+          float v[R];
+          load_logits(v);
           warp_col_reduce<R, true>(v, lane);
           store_reduced<R>(ms.red[warp], v, lane);
-        }
-        named_bar_sync(1, kSoftThreads);
-        bool mine = false;
-        if (t < R) {
-          const float mt = fmaxf(fmaxf(ms.red[0][t], ms.red[1][t]), fmaxf(ms.red[2][t], ms.red[3][t]));
-          const float mo = ms.mu[t];
-          float cr = 1.f;
-          if (mt > mo + kRescaleLog2) {
-            cr = (mo == -INFINITY) ? 0.f : ex2(mo - mt);
-            ms.mu[t] = mt;
-            mine = true;
+          named_bar_sync(1, kSoftThreads);
+          bool mine = false;
+          if (t < R) {
+            const float mt = fmaxf(fmaxf(ms.red[0][t], ms.red[1][t]), fmaxf(ms.red[2][t], ms.red[3][t]));
+            const float mo = ms.mu[t];
+            float cr = 1.f;
+            if (mt > mo + kRescaleLog2) {
+              cr = (mo == -INFINITY) ? 0.f : ex2(mo - mt);
+              ms.mu[t] = mt;
+              mine = true;
+            }
+            ms.corr[t] = cr;
           }
-          ms.corr[t] = cr;
+          if (group_any(mine) && p > it.p0) {
+            // O^T holds this item's earlier tiles: rescale it once the previous tile's output
+            // MMAs are complete
+            bool done = true;
+            if (t == 0) done = pv_wait(tile_n - 1);
+            if (!group_all(done)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+#pragma unroll
+              for (int c0 = 0; c0 < R; c0 += 16) {
+                uint32_t ov[16];
+                tmem_ld16(tl + m * R + c0, ov);
+                tmem_wait_ld(ov);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[c0 + e]);
+                tmem_st16(tl + m * R + c0, ov);
+                tmem_wait_st();
+              }
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < R; ++c) lpart[c] *= ms.corr[c];
         }
-        const bool rescale = group_any(mine) && i > 0;
-        // pass 2: probabilities, running column sums, and P^T into the RoPE-key slot, token-major:
-        // row t holds this token's R probabilities (2R bytes), 16-byte units swizzled by row
-        uint8_t* prow = smem + C::KR_OFF + ks * kChunkBytes + t * (2 * R);
-        const int swz = (R == 16) ? ((t >> 2) & 1) : (R == 32) ? ((t >> 1) & 3) : (t & 7);
+        // probabilities, running column sums, and P^T into the RoPE-key slot, token-major:
+        // row `tok` holds this token's R probabilities (2R bytes), 16-byte units swizzled by row
+        uint8_t* prow = smem + C::KR_OFF + ks * kKrBytes + (has_tok ? tok : 0) * (2 * R);
+        const int swz = (R == 16) ? ((tok >> 2) & 1) : (R == 32) ? ((tok >> 1) & 3) : (tok & 7);
 #pragma unroll
         for (int c0 = 0; c0 < R; c0 += 16) {
-          uint32_t sc[16], sr[16];
-          tmem_ld16(tSc + c0, sc);
-          tmem_ld16(tSc + R + c0, sr);
-          float aq[16], mu[16], cr[16];
-          int ql[16];
+          float mu[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            *reinterpret_cast<float4*>(aq + 4 * q) = *reinterpret_cast<const float4*>(ms.aq2 + c0 + 4 * q);
-            *reinterpret_cast<int4*>(ql + 4 * q) = *reinterpret_cast<const int4*>(ms.qlim + c0 + 4 * q);
+          for (int q = 0; q < 4; ++q)
             *reinterpret_cast<float4*>(mu + 4 * q) = *reinterpret_cast<const float4*>(ms.mu + c0 + 4 * q);
-            *reinterpret_cast<float4*>(cr + 4 * q) = *reinterpret_cast<const float4*>(ms.corr + c0 + 4 * q);
-          }
-          tmem_wait_ld(sc, sr);
           uint32_t packed[8];
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
@@ -560,66 +576,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
               const int c = c0 + e + u;
-              float akc = ak0;
-              if (!AK_ONE && G > 1) akc = akrow[ms.grp[c]];
-              const float x = aq[e + u] * akc * __uint_as_float(sc[e + u]) + kLog2e * __uint_as_float(sr[e + u]);
-              const bool vis = row_ok && tpos <= ql[e + u];
-              const float p = vis ? ex2(x - mu[e + u]) : 0.f;
-              lpart[c] = lpart[c] * cr[e + u] + p;
-              pp[u] = p;
+              const float pr = x[c] == -INFINITY ? 0.f : ex2(x[c] - mu[e + u]);
+              lpart[c] += pr;
+              pp[u] = pr;
             }
             __nv_bfloat162 b2 = __floats2bfloat162_rn(pp[0], pp[1]);
             packed[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
           }
-          const int u0 = c0 / 8;    // 16-byte units c0/8 and c0/8 + 1 of the row
-          *reinterpret_cast<uint4*>(prow + (((u0 + 0) ^ swz) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ swz) << 4)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          if (has_tok) {
+            const int u0 = c0 / 8;    // 16-byte units c0/8 and c0/8 + 1 of the row
+            *reinterpret_cast<uint4*>(prow + (((u0 + 0) ^ swz) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ swz) << 4)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          }
         }
         // the S buffer is free for the tile after next
         tc_fence_before();
         mbar_arrive(smem_u32(&ms.s_empty[sbuf]));
-        // rows of real pages past the context: zero them so that 0 * garbage cannot reach O
-        if (!row_ok && t < np * 64) {
+        // rows of the page past the context: zero them so that 0 * garbage cannot reach O
+        if (has_tok && !row_ok) {
 #pragma unroll
           for (int k = 0; k < kChunks; ++k) {
-            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + ((c_it + k / 2) % NS) * kSlotBytes +
-                                                   (k & 1) * kChunkBytes + t * 128);
+            const int sl = c_first + k / 2 < NS ? c_first + k / 2 : c_first + k / 2 - NS;
+            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + sl * kSlotBytes +
+                                                   (k & 1) * kChunkBytes + tok * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q) rowp[q] = make_uint4(0, 0, 0, 0);
           }
         }
-        // the output MMAs of the previous tile must be complete before O^T is rescaled (and,
-        // waited for every tile, this keeps the barrier's phases in step)
-        got = true;
-        if (t == 0 && tile_n > 0) got = mbar_wait(smem_u32(&ms.pv_done), (tile_n - 1) & 1, a.wait_limit);
-        if (!group_all(got)) { ok = false; break; }
-        tc_fence_after();
-        if (rescale) {
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-#pragma unroll
-            for (int c0 = 0; c0 < R; c0 += 16) {
-              uint32_t ov[16];
-              tmem_ld16(tl + m * R + c0, ov);
-              tmem_wait_ld(ov);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[c0 + e]);
-              tmem_st16(tl + m * R + c0, ov);
-              tmem_wait_st();
-            }
-          }
-        }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(smem_u32(&ms.p_full));
-        c_it += kSlotsPerTile;
-        ++k_it;
+        mbar_arrive(smem_u32(&ms.p_full[tile_n & 1]));
+        c_first = c_first + kSlotsPerTile < NS ? c_first + kSlotsPerTile : c_first + kSlotsPerTile - NS;
+        kr.next();
         ++tile_n;
       }
       if (!ok) break;
       // ---------------- epilogue: O / l and lse for this item
       bool got = true;
-      if (t == 0) got = mbar_wait(smem_u32(&ms.pv_done), (tile_n - 1) & 1, a.wait_limit);
+      if (t == 0) {
+        if (tile_n > 1) got = pv_wait(tile_n - 2);
+        got = got && pv_wait(tile_n - 1);
+      }
       if (!group_all(got)) { ok = false; break; }
       tc_fence_after();
       warp_col_reduce<R, false>(lpart, lane);
