@@ -66,7 +66,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;        // rescale O only when a column max grows by > 2^8
 constexpr int64_t kDrainLimit = 4000000000LL;
-constexpr int kPrefetchPages = 4;          // pages the L2 prefetch runs ahead of the TMA loads
 
 template <int R>
 struct Cfg {
@@ -113,7 +112,7 @@ struct Misc {
 }  // namespace
 
 struct TcMaps {
-  CUtensorMap latent;   // [num_blocks*64, 512] bf16, box 64 x 64
+  CUtensorMap latent;   // [8 chunks][num_blocks*64 rows][64] bf16 view of the latent, box 2 x 64 x 64
   CUtensorMap krope;    // [num_blocks*64, 64]  bf16, box 64 x 64
   CUtensorMap qt;       // [n_q*H, 512]         bf16, box 64 x R
   CUtensorMap qr;       // [n_q*H, 64]          bf16, box 64 x R
@@ -258,12 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     int n_item = 0;
     bool ok = true;
     const uint32_t akpage = (uint32_t)kPage * (uint32_t)G * 4u;
-    auto prefetch_page = [&](int32_t blk) {
-      prefetch_l2(static_cast<const __nv_bfloat16*>(a.latent) + (int64_t)blk * kPage * kRkv, kPage * kRkv * 2);
-      prefetch_l2(static_cast<const __nv_bfloat16*>(a.k_rope) + (int64_t)blk * kPage * kDrope, kKrBytes);
-      if (!AK_ONE) prefetch_l2(a.a_k + (int64_t)blk * kPage * G, akpage);
-    };
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+      const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
+      // the first 32 block-table entries of the item are read before the query tile is issued, so
+      // that the two memory latencies overlap
+      int32_t mine = (it.p0 + lane < it.p1) ? row[it.p0 + lane] : 0;
       if (!mbar_wait_warp(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
       {
         const int qrow0 = it.b * qrows + it.ht * R;
@@ -273,32 +271,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         for (int k = 0; k < kChunks; ++k) tma_load_2d_elect(sb + C::Q_OFF + k * R * 128, &maps.qt, k * 64, qrow0, qf);
         tma_load_2d_elect(sb + C::QR_OFF, &maps.qr, 0, qrow0, qf);
       }
-      const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
       for (int pb = it.p0; pb < it.p1 && ok; pb += 32) {
         // 32 block-table entries per warp-wide load
-        int32_t mine = 0;
-        if (pb + lane < it.p1) {
-          mine = row[pb + lane];
-          if (mine < 0 || mine >= a.num_blocks) {
-            record_status(a.status, QKN_ERR_BOUNDS);
-            mine = 0;
-          }
+        if (pb > it.p0) mine = (pb + lane < it.p1) ? row[pb + lane] : 0;
+        if (mine < 0 || mine >= a.num_blocks) {
+          record_status(a.status, QKN_ERR_BOUNDS);
+          mine = 0;
         }
         const int cnt = min(32, it.p1 - pb);
-        // L2 prefetch runs kPrefetchPages ahead of the TMA loads, which wait for ring slots
-        if (lane < min(cnt, kPrefetchPages)) prefetch_page(mine);
         for (int k = 0; k < cnt && ok; ++k) {
           const int32_t blk = __shfl_sync(0xffffffffu, mine, k);
-          const int32_t ahead = __shfl_sync(0xffffffffu, mine, min(k + kPrefetchPages, 31));
-          if (lane == 0 && k + kPrefetchPages < cnt) prefetch_page(ahead);
-          __syncwarp();
           for (int m = 0; m < kSlotsPerTile; ++m) {
             if (!mbar_wait_warp(smem_u32(&ms.empty[cw.slot]), cw.phase ^ 1u, a.wait_limit)) { ok = false; break; }
             const uint32_t fb = smem_u32(&ms.full[cw.slot]);
             mbar_arrive_expect_tx_elect(fb, kSlotBytes);
             const uint32_t dst = sb + C::C_OFF + cw.slot * kSlotBytes;
-            tma_load_2d_elect(dst, &maps.latent, (2 * m) * 64, blk * kPage, fb);
-            tma_load_2d_elect(dst + kChunkBytes, &maps.latent, (2 * m + 1) * 64, blk * kPage, fb);
+            tma_load_3d_elect(dst, &maps.latent, 0, blk * kPage, 2 * m, fb);   // chunks 2m, 2m+1 of the page
             cw.next();
             ++c_issued;
           }
@@ -688,6 +676,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view of the latent cache [rows, 512] as [8 chunks][rows][64]: dimension 0 is the 64 columns
+// of a chunk, dimension 1 the token row (stride 1024 bytes), dimension 2 the chunk (stride 128
+// bytes).  A box of 2 chunks x 64 rows lands as two consecutive 8 KB swizzled chunk tiles.
+bool make_latent_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, 8};
+  cuuint64_t strides[2] = {512 * 2, 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int R, bool AK_ONE>
 cudaError_t launch_tc(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) {
   static bool attr_set = false;
@@ -712,7 +715,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   TcMaps maps;
   const uint64_t cache_rows = (uint64_t)a.num_blocks * 64;
   const uint64_t q_rows = (uint64_t)a.batch * a.s_q * a.heads;
-  if (!make_map(&maps.latent, a.latent, kRkv, cache_rows, 64, 64) ||
+  if (!make_latent_map(&maps.latent, a.latent, cache_rows) ||
       !make_map(&maps.krope, a.k_rope, kDrope, cache_rows, 64, 64) ||
       !make_map(&maps.qt, a.q_tilde, kRkv, q_rows, 64, a.rows) ||
       !make_map(&maps.qr, a.q_rope_hat, kDrope, q_rows, 64, a.rows))
