@@ -148,6 +148,8 @@ QKN_EXPORT qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache,
  *   w_k        [num_groups, r_kv, n_g * d_h] fp32
  *   q_tilde    [n_q, H, r_kv] dtype (out), a_q [n_q, H] fp32 (out),
  *   q_rope_hat [n_q, H, d_rope] dtype (out).
+ * w_k, gamma_q and gamma_k must be 16-byte aligned (QKN_ERR_INVALID_ARG otherwise);
+ * d_h must be a multiple of 4 and at most 256 (QKN_ERR_UNSUPPORTED otherwise).
  * n_q == 0 is a no-op. */
 QKN_EXPORT qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_rope,
                             const int32_t* pos, int32_t n_q, const float* w_k,

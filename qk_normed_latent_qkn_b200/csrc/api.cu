@@ -168,7 +168,7 @@ qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_r
   if (!q || !q_rope || !pos || !w_k || !gamma_q || !gamma_k || !gamma_qr || !q_tilde || !a_q || !q_rope_hat)
     return QKN_ERR_INVALID_ARG;
   if (dims->d_h > 256 || dims->d_h % 4) return QKN_ERR_UNSUPPORTED;
-  if (!aligned(w_k, 16)) return QKN_ERR_INVALID_ARG;
+  if (!aligned(w_k, 16) || !aligned(gamma_q, 16) || !aligned(gamma_k, 16)) return QKN_ERR_INVALID_ARG;
   AbsorbArgs a;
   a.q = q;
   a.q_rope = q_rope;

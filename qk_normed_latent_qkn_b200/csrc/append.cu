@@ -82,14 +82,16 @@ __global__ void __launch_bounds__(256) append_copy_kernel(const __grid_constant_
   for (int g = lane; g < a.groups; g += 32) a.a_k[slot * a.groups + g] = 0.f;
 }
 
-// Key statistic sum(z^2), z = c W^K_g.  CTA = (32 key columns, TT tokens,
-// group); its 256 threads are 32 columns x 8 slices of the latent dimension,
-// so every thread issues r/8 independent, coalesced loads of W and reuses
-// each for TT tokens held in shared memory.  Slices are summed in shared
-// memory, squared, reduced over the CTA's 32 columns and added into the
-// token's a_k slot (zeroed by append_copy_kernel).
-constexpr int kRmsCols = 32;
-constexpr int kRmsSlices = 8;
+// Key statistic sum(z^2), z = c W^K_g.  CTA = (16 key columns, TT tokens,
+// group); its 512 threads are 16 columns x 32 slices of the latent
+// dimension, so a decode step's handful of tokens still spreads over about a
+// hundred CTAs per group.  Every thread loads its slice of one W column in
+// one batch of independent loads and applies it to the TT tokens held in
+// shared memory; slices are summed in shared memory, squared, reduced over
+// the CTA's 16 columns and added into the token's a_k slot (zeroed by
+// append_copy_kernel).
+constexpr int kRmsCols = 16;
+constexpr int kRmsSlices = 32;
 
 template <typename T, int TT>
 __global__ void __launch_bounds__(kRmsCols * kRmsSlices) append_keyrms_kernel(AppendArgs a) {
@@ -100,12 +102,21 @@ __global__ void __launch_bounds__(kRmsCols * kRmsSlices) append_keyrms_kernel(Ap
   const int t0 = blockIdx.y * TT;
   const int ntok = min(TT, a.n_tok - t0);
   const int width = a.width;
-  const int col = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int col = threadIdx.x % kRmsCols, slice = threadIdx.x / kRmsCols;
   const int n = blockIdx.x * kRmsCols + col;
   pdl_trigger();
   pdl_wait();
 
-  {   // stage the token tile as fp32, 16 bytes of input per load, loads batched
+  // latent rows [k0, k1) of this slice; W loads are issued before the token tile is staged
+  const int k0 = (int)((int64_t)slice * a.r / kRmsSlices);
+  const int k1 = (int)((int64_t)(slice + 1) * a.r / kRmsSlices);
+  const float* w = a.w_k + (int64_t)g * a.r * width + min(n, width - 1);
+  constexpr int kBatch = 16;
+  float wv[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) wv[u] = (k0 + u < k1) ? w[(int64_t)(k0 + u) * width] : 0.f;
+
+  {   // stage the token tile as fp32, 16 bytes of input per load
     constexpr int kPer = 16 / (int)sizeof(T);          // elements per 16-byte load
     const uint4* c4 = reinterpret_cast<const uint4*>(static_cast<const T*>(a.c_new) + (int64_t)t0 * a.r);
     const int nvec = TT * a.r / kPer;
@@ -132,24 +143,15 @@ __global__ void __launch_bounds__(kRmsCols * kRmsSlices) append_keyrms_kernel(Ap
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-  // latent rows [k0, k1) of this slice
-  const int k0 = (int)((int64_t)slice * a.r / kRmsSlices);
-  const int k1 = (int)((int64_t)(slice + 1) * a.r / kRmsSlices);
-  if (n < width) {
-    const float* w = a.w_k + (int64_t)g * a.r * width + n;
-    int k = k0;
-    // 32 independent W loads in flight per thread, then their FMAs (16-byte token-row reads
-    // need k % 4 == 0, which holds whenever r % 32 == 0)
-    const bool vec_ok = ((k0 | a.r) & 3) == 0;
-    for (; vec_ok && k + 32 <= k1; k += 32) {
-      float wv[32];
-#pragma unroll
-      for (int u = 0; u < 32; ++u) wv[u] = w[(int64_t)(k + u) * width];
+  for (int kb = k0;; ) {
+    const int nk = min(kBatch, k1 - kb);
+    if (nk == kBatch && (kb & 3) == 0 && (a.r & 3) == 0) {
+      // 16-byte token reads: four FMAs per shared-memory load
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        const float4* crow = reinterpret_cast<const float4*>(cs + t * a.r + k);   // r % 4 == 0, k % 32 == k0 % 4 == 0
+        const float4* crow = reinterpret_cast<const float4*>(cs + t * a.r + kb);
 #pragma unroll
-        for (int u4 = 0; u4 < 8; ++u4) {
+        for (int u4 = 0; u4 < kBatch / 4; ++u4) {
           const float4 cv = crow[u4];
           acc[t] = fmaf(cv.x, wv[4 * u4 + 0], acc[t]);
           acc[t] = fmaf(cv.y, wv[4 * u4 + 1], acc[t]);
@@ -157,36 +159,33 @@ __global__ void __launch_bounds__(kRmsCols * kRmsSlices) append_keyrms_kernel(Ap
           acc[t] = fmaf(cv.w, wv[4 * u4 + 3], acc[t]);
         }
       }
-    }
-    for (; k + 8 <= k1; k += 8) {
-      float wv[8];
+    } else {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) wv[u] = w[(int64_t)(k + u) * width];
+      for (int t = 0; t < TT; ++t) {
+        const float* crow = cs + t * a.r + kb;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-#pragma unroll
-        for (int t = 0; t < TT; ++t) acc[t] = fmaf(cs[t * a.r + k + u], wv[u], acc[t]);
+        for (int u = 0; u < kBatch; ++u)
+          if (u < nk) acc[t] = fmaf(crow[u], wv[u], acc[t]);
       }
     }
-    for (; k < k1; ++k) {
-      const float wv = w[(int64_t)k * width];
+    kb += kBatch;
+    if (kb >= k1) break;
 #pragma unroll
-      for (int t = 0; t < TT; ++t) acc[t] = fmaf(cs[t * a.r + k], wv, acc[t]);
-    }
+    for (int u = 0; u < kBatch; ++u) wv[u] = (kb + u < k1) ? w[(int64_t)(kb + u) * width] : 0.f;
   }
 #pragma unroll
   for (int t = 0; t < TT; ++t) zp[(slice * TT + t) * kRmsCols + col] = acc[t];
   __syncthreads();
-  // thread (slice, col) finishes tokens slice, slice + 8, ...: z summed over slices, squared,
-  // then summed over the 32 columns of the warp
-  for (int t = slice; t < ntok; t += kRmsSlices) {
+  // thread (slice, col) finishes tokens slice, slice + 16, ...: z summed over slices, squared,
+  // then summed over the 16 columns of its half-warp
+  for (int t = slice; t < TT; t += kRmsSlices) {
     float z = 0.f;
 #pragma unroll
     for (int sl = 0; sl < kRmsSlices; ++sl) z += zp[(sl * TT + t) * kRmsCols + col];
     float v = (n < width) ? z * z : 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (col == 0) atomicAdd(a.a_k + (int64_t)a.slot[t0 + t] * a.groups + g, v);
+    for (int o = kRmsCols / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (col == 0 && t < ntok) atomicAdd(a.a_k + (int64_t)a.slot[t0 + t] * a.groups + g, v);
   }
 }
 
