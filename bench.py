@@ -38,6 +38,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "decode tokens/s and us/step at 1 B200; % of HBM/tensor roofline; overhead vs MLA"
+# kernels of libqkn launched per step: append (copy, key RMS, finalize), absorb, split-KV decode, merge
+LAUNCHES_PER_STEP = 6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -295,7 +297,7 @@ def run_ours(args, world, rank, local):
 
     side = torch.cuda.Stream(device=device)
 
-    def step(i, split_event=None, ak_mode=qkn.AK_CACHE, start_event=None):
+    def step(i, split_event=None, ak_mode=qkn.AK_CACHE, start_event=None, end_event=None):
         """Append and absorb are independent: absorb runs on a side stream, joined before decode."""
         s, d, (o, l) = sessions[i], dev_in[i], outs[i]
         main = torch.cuda.current_stream(device)
@@ -307,6 +309,8 @@ def run_ours(args, world, rank, local):
         if start_event is not None:
             ev.record(start_event, main.cuda_stream)
         s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event)
+        if end_event is not None:
+            ev.record(end_event, main.cuda_stream)
 
     def decode_only(i, split_event=None, ak_mode=qkn.AK_CACHE):
         s, d, (o, l) = sessions[i], dev_in[i], outs[i]
@@ -329,11 +333,12 @@ def run_ours(args, world, rank, local):
     with torch.cuda.stream(stream):
         for k in range(total):
             i = k % n_copies
-            # two event nodes per step, around the split-KV kernel: its duration is the roofline's
+            # two event nodes per step, around the decode op (split-KV kernel + merge kernel, chained
+            # by programmatic launch with no node between them): its duration is the roofline's
             e = [ev.create() for _ in range(2)]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-                step(i, split_event=e[1], start_event=e[0])
+                step(i, start_event=e[0], end_event=e[1])
             graphs.append(g)
             marks.append(e)
         # decode-only graphs, QK-Normed and plain MLA, for the overhead figure
@@ -383,7 +388,7 @@ def run_ours(args, world, rank, local):
     local_ms = t_start_ev.elapsed_time(t_end_ev)
     value, step_ms = job_throughput(B * s_q, world, local_ms, args.steps, device)
 
-    split_ms = [ev.ms(marks[k][0], marks[k][1]) for k in range(args.warmup, total)]
+    op_ms = [ev.ms(marks[k][0], marks[k][1]) for k in range(args.warmup, total)]
 
     # breakdown of one step (separate graphs with an event node between every stage; not the timed region)
     bd_graphs = []
@@ -397,13 +402,14 @@ def run_ours(args, world, rank, local):
                 step(i, split_event=e[2], start_event=e[1])
                 ev.record(e[3], sid)
             bd_graphs.append((g, e))
-    prep_ms, combine_ms = [], []
+    prep_ms, split_ms, combine_ms = [], [], []
     with torch.cuda.stream(stream):
         for _ in range(3):
             for g, e in bd_graphs:
                 g.replay()
                 stream.synchronize()
                 prep_ms.append(ev.ms(e[0], e[1]))
+                split_ms.append(ev.ms(e[1], e[2]))
                 combine_ms.append(ev.ms(e[2], e[3]))
 
     # overhead vs plain MLA: interleaved rounds of decode-only graphs
@@ -448,13 +454,13 @@ def run_ours(args, world, rank, local):
     e2e_ms = reduce_max(e0.elapsed_time(e1), device) / args.steps
     assert all(s.device_status() == qkn.OK for s in sessions)
 
-    # roofline of the dominant kernel (the split-KV decode)
+    # roofline of the dominant op (the decode: split-KV kernel + merge kernel)
     cost = decode_step_cost(inp.seq_lens, s_q, H, wl.groups, wl.r_kv, wl.d_rope,
                             elem=2 if wl.dtype == "bf16" else 4)
     peaks, peak_src = load_peaks()
-    split_avg = statistics.mean(split_ms)
-    achieved_gbs = cost.bytes / (split_avg * 1e-3) / 1e9
-    tflops = cost.flops / (split_avg * 1e-3) / 1e12
+    op_avg = statistics.mean(op_ms)
+    achieved_gbs = cost.bytes / (op_avg * 1e-3) / 1e9
+    tflops = cost.flops / (op_avg * 1e-3) / 1e12
     tokens = world * B * s_q
 
     line = None
@@ -479,12 +485,17 @@ def run_ours(args, world, rank, local):
                              f"(L2 {l2 / 2**20:.0f} MiB)", "step_launch": "CUDA graph per step",
                        "parallelism": f"replicas x{world}"},
             "breakdown_us": {"append_absorb": statistics.median(prep_ms) * 1e3,
-                             "decode_split": split_avg * 1e3, "combine": statistics.median(combine_ms) * 1e3,
-                             "what": "append and absorb (side stream) / split-KV kernel / combine; separate graphs"},
+                             "decode_split": statistics.median(split_ms) * 1e3,
+                             "combine": statistics.median(combine_ms) * 1e3, "decode_op_timed": op_avg * 1e3,
+                             "what": "append and absorb (side stream) / split-KV kernel / merge kernel, from "
+                                     "separate graphs with an event between every stage; decode_op_timed is the "
+                                     "split-KV + merge pair inside the timed steps"},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes": cost.bytes, "peak_source": f"{peak_src} HBM copy bandwidth",
-                         "kernel": "decode split (tcgen05)" if kernel_used == qkn.KERNEL_TCGEN05 else "decode split",
+                         "kernel": ("decode op: split-KV kernel (tcgen05) + merge kernel, averaged over the timed "
+                                    "steps" if kernel_used == qkn.KERNEL_TCGEN05 else
+                                    "decode op: split-KV kernel (simt) + merge kernel, averaged over the timed steps"),
                          "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                     "frac": tflops / peaks["bf16_tflops"], "flops": cost.flops}},
             "overhead_vs_mla": {"qkn_us": t_qkn * 1e3, "mla_us": t_mla * 1e3, "frac": t_qkn / t_mla - 1.0,
@@ -492,7 +503,7 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "what": "DecodeSession append/absorb/decode, eager, pinned host in/out, sync per step"},
-            "gpu_launches": 7 * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": sampler.summary(window),
             "cpu_baseline": cpu,
         }

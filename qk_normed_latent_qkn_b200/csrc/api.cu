@@ -86,21 +86,23 @@ int pick_kernel(const qkn_dims* d, int s_q, const qkn_decode_opts* o) {
 }
 
 struct WsLayout {
-  size_t lse_off, o_off, total;
+  size_t desc_off, lse_off, o_off, total;   // status word | segment descriptors | split lse | split outputs
 };
 
 WsLayout ws_layout(const qkn_dims* d, int batch, int s_q, int ncta) {
   // Size for the largest row tile any kernel may use, so that one workspace
   // serves every kernel choice.
-  int64_t slot_rows = 0;
+  int64_t slot_rows = 0, segments = 0;
   const int qrows = s_q * d->num_heads;
   for (int rows : {kSimtRows, 16, 32, 64}) {
     const int64_t ht = ceil_div(qrows, rows);
     const int64_t sr = sched_slots(batch, ht, ncta) * rows;
     if (sr > slot_rows) slot_rows = sr;
+    if (batch * ht > segments) segments = batch * ht;
   }
   WsLayout w;
-  w.lse_off = kStatusBytes;
+  w.desc_off = kStatusBytes;
+  w.lse_off = w.desc_off + ((size_t)segments * 8 + 255) / 256 * 256;
   const size_t lse_bytes = ((size_t)slot_rows * 4 + 255) / 256 * 256;
   w.o_off = w.lse_off + lse_bytes;
   w.total = w.o_off + (size_t)slot_rows * d->r_kv * 4;
@@ -269,6 +271,9 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   a.part_o = reinterpret_cast<float*>(ws + w.o_off);
   a.status = reinterpret_cast<int32_t*>(ws);
   a.wait_limit = (opts && opts->wait_limit > 0) ? opts->wait_limit : (int64_t)4000000000LL;
+  a.out = out;
+  a.lse = lse;
+  a.seg_desc = reinterpret_cast<int2*>(ws + w.desc_off);
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const bool bf16 = dims->dtype == QKN_BF16;
@@ -295,6 +300,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   c.out = out;
   c.lse = lse;
   c.status = a.status;
+  c.seg_desc = kernel == QKN_KERNEL_TCGEN05 ? a.seg_desc : nullptr;
   e = launch_combine(c, bf16, cs);
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
 }

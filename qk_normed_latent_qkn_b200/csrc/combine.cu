@@ -43,17 +43,30 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   const int rho = ht * a.rows + row;
   if (b >= a.batch || rho >= qrows) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (a.seg_desc) {
+    // a sequence with a rejected length has no splits: the tcgen05 kernel wrote its rows itself
+    const int2 d = a.seg_desc[seg];
+    if (d.y <= 0) return;
+  }
   if (warp == 0) {
-    SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
-    const int64_t total = sched_total_units(sp);
-    const int64_t before = sched_pages_before(sp, b);
-    const int32_t n = pages_of(a.seq_lens[b], sp);
-    if (n == 0 && ht == 0 && row == 0 && lane == 0) record_status(a.status, QKN_ERR_BOUNDS);
-    const int64_t q = total > 0 ? (total + a.ncta - 1) / a.ncta : 1;
-    const int64_t u0 = before * a.ht_count + (int64_t)ht * n;
-    const int64_t c0 = u0 / q;
-    const int nitems = n > 0 ? (int)((u0 + n - 1) / q - c0 + 1) : 0;
-    const int64_t first = (int64_t)(seg + c0) * a.rows + row;   // partial row of the first split
+    int64_t first;
+    int nitems;
+    if (a.seg_desc) {
+      const int2 d = a.seg_desc[seg];
+      first = (int64_t)d.x * a.rows + row;
+      nitems = d.y;
+    } else {
+      SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
+      const int64_t total = sched_total_units(sp);
+      const int64_t before = sched_pages_before(sp, b);
+      const int32_t n = pages_of(a.seq_lens[b], sp);
+      if (n == 0 && ht == 0 && row == 0 && lane == 0) record_status(a.status, QKN_ERR_BOUNDS);
+      const int64_t q = total > 0 ? (total + a.ncta - 1) / a.ncta : 1;
+      const int64_t u0 = before * a.ht_count + (int64_t)ht * n;
+      const int64_t c0 = u0 / q;
+      nitems = n > 0 ? (int)((u0 + n - 1) / q - c0 + 1) : 0;
+      first = (int64_t)(seg + c0) * a.rows + row;   // partial row of the first split
+    }
     float mx = -INFINITY;
     for (int c = lane; c < nitems; c += 32) mx = fmaxf(mx, a.part_lse[first + (int64_t)c * a.rows]);
 #pragma unroll

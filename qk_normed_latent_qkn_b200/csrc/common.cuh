@@ -131,9 +131,11 @@ struct Cursor {
   int64_t quota;         // Q
 };
 
-// Item handed to the roles: pages [p0, p1) of sequence b, row tile ht.
+// Item handed to the roles: pages [p0, p1) of sequence b, row tile ht; the
+// segment's units are [seg_u0, seg_u0 + (pages of b)).
 struct Item {
   int32_t b, ht, p0, p1, L, slot;
+  int64_t seg_u0;
 };
 
 __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta) {
@@ -190,6 +192,7 @@ __device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, in
       it.p1 = (int32_t)((cur.end < s1 ? cur.end : s1) - s0);
       it.L = p.seq_lens[cur.b];
       it.slot = cur.b * p.ht_count + cur.ht + cta;
+      it.seg_u0 = s0;
     }
     // advance to the next segment
     cur.seg_u0 = s1;
@@ -202,6 +205,19 @@ __device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, in
     if (overlaps) return true;
   }
   return false;
+}
+
+// The CTAs that share a segment: units [u0, u0 + n) are split over CTAs
+// c0 .. c0 + nitems - 1 (quota q units each), whose partial results sit in
+// workspace slots seg + c0 .. seg + c0 + nitems - 1.
+struct SegSplit {
+  int32_t c0, nitems;
+};
+__device__ __forceinline__ SegSplit seg_split(int64_t u0, int32_t n, int64_t q) {
+  SegSplit s;
+  s.c0 = (int32_t)(u0 / q);
+  s.nitems = (int32_t)((u0 + n - 1) / q) - s.c0 + 1;
+  return s;
 }
 
 // Workspace slots needed: one per (segment, CTA) pair that can meet.

@@ -58,8 +58,7 @@ extern "C" qkn_status qkn_decode_noalloc(const qkn_dims* dims, const qkn_cache* 
   if (!scratch) return QKN_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // The array keeps whatever the previous call left in it; only the status
-  // word has to start from zero (the partial results are written before they
-  // are read).
+  // word has to start from zero (everything else is written before it is read).
   if (cudaMemsetAsync(scratch, 0, qkn::kStatusBytes, cs) != cudaSuccess) return QKN_ERR_CUDA;
   st = qkn_decode(dims, cache, ak_mode, q_tilde, a_q, q_rope_hat, block_table, max_blocks, seq_lens, batch, s_q,
                   scratch, (size_t)QKN_NOALLOC_SCRATCH_BYTES, out, lse, opts, stream);

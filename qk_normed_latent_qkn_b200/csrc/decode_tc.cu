@@ -431,6 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     int64_t tile_n = 0;
     int n_item = 0;
     bool ok = true;
+    // sequences b = blockIdx.x (mod gridDim.x) with a rejected length are this CTA's to report (checked
+    // while the first scores are still being loaded)
+    bool rejected = false;
+    for (int b = blockIdx.x + t * gridDim.x; b < a.batch; b += kSoftThreads * gridDim.x)
+      rejected |= pages_of(a.seq_lens[b], sp) == 0;
+    rejected = group_any(rejected);
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
       if (t < R) {
         const int rho = it.ht * R + t;
@@ -507,7 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         if (group_any(over || !got)) {
           if (group_any(!got)) { ok = false; break; }
           float v[R];
-          load_logits(v);
+#pragma unroll
+          for (int c = 0; c < R; ++c) v[c] = x[c];
           warp_col_reduce<R, true>(v, lane);
           store_reduced<R>(ms.red[warp], v, lane);
           named_bar_sync(1, kSoftThreads);
@@ -631,11 +638,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&ms.o_empty));
+      // the CTA holding a segment's first split tells the merge kernel where its splits are
+      if (t == 0 && it.p0 == 0) {
+        const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota);
+        a.seg_desc[it.b * a.ht_count + it.ht] = make_int2(it.b * a.ht_count + it.ht + sg.c0, sg.nitems);
+      }
       ++n_item;
     }
     if (!ok && t == 0) {
       record_status(a.status, QKN_ERR_TIMEOUT);
       ms.abort_flag = 1;
+    }
+    // A sequence whose length was rejected (outside [s_q, max_blocks * 64]) has no units: its rows
+    // are written as zero with lse = -inf, and the status records QKN_ERR_BOUNDS.
+    for (int b = blockIdx.x; rejected && b < a.batch; b += gridDim.x) {
+      if (pages_of(a.seq_lens[b], sp) != 0) continue;
+      if (t == 0) record_status(a.status, QKN_ERR_BOUNDS);
+      for (int ht = t; ht < a.ht_count; ht += kSoftThreads) a.seg_desc[b * a.ht_count + ht] = make_int2(0, 0);
+      uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * qrows * kRkv);
+      for (int64_t e = t; e < (int64_t)qrows * kRkv / 8; e += kSoftThreads) ob[e] = make_uint4(0, 0, 0, 0);
+      for (int e = t; e < qrows; e += kSoftThreads) a.lse[(int64_t)b * qrows + e] = -INFINITY;
     }
   }
 

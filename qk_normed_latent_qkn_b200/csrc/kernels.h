@@ -2,7 +2,10 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
+
+#include "qkn.h"
 
 namespace qkn {
 
@@ -63,6 +66,11 @@ struct DecodeArgs {
   float* part_lse;           // [slots, R] fp32
   int32_t* status;           // workspace status word
   int64_t wait_limit;        // bounded-wait cycles (tcgen05 kernel)
+  // tcgen05 kernel only: a segment finished by one CTA is written to out / lse directly, and
+  // seg_desc[segment] = (first split slot, number of splits) tells the merge kernel the rest
+  void* out;                 // [batch, s_q, H, r] bf16
+  float* lse;                // [batch, s_q, H]
+  int2* seg_desc;            // [batch * ht_count]
 };
 
 struct CombineArgs {
@@ -74,6 +82,7 @@ struct CombineArgs {
   void* out;                 // [batch, s_q, H, r]
   float* lse;                // [batch, s_q, H]
   int32_t* status;           // workspace status word
+  const int2* seg_desc;      // per-segment (first slot, splits) from the tcgen05 kernel, or null
 };
 
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);
