@@ -424,31 +424,28 @@ def run_ours(args, world, rank, local):
     t_qkn = statistics.median(per_mode[qkn.AK_CACHE])
     t_mla = statistics.median(per_mode[qkn.AK_ONE])
 
-    # end to end through the public API, host (pinned) buffers in and out every step
-    pinned_in = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dtype=types[k]).pin_memory() for k, v in host.items()}
-    pinned_out = (torch.empty((B, s_q, H, wl.r_kv), dtype=dt).pin_memory(),
-                  torch.empty((B, s_q, H), dtype=torch.float32).pin_memory())
-    h2d = sum(t.numel() * t.element_size() for t in pinned_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in pinned_out)
-
-    def e2e_step(k):
-        i = k % n_copies
-        d = dev_in[i]
-        for key, t in pinned_in.items():
-            d[key].copy_(t, non_blocking=True)
-        step(i)
-        pinned_out[0].copy_(outs[i][0], non_blocking=True)
-        pinned_out[1].copy_(outs[i][1], non_blocking=True)
-        torch.cuda.current_stream(device).synchronize()
+    # end to end through the public API: DecodeStep replays copy-in, append || absorb, decode and
+    # copy-out as one graph per step, from and to pinned host buffers, with a synchronize per step
+    from qk_normed_latent_qkn_b200.step import DecodeStep
+    names = {"c": "c", "kr": "k_rope", "slot": "slot", "pos": "pos", "q": "q", "qr": "q_rope", "qpos": "qpos",
+             "bt": "block_table", "sl": "seq_lens"}
+    steps = []
+    for i in range(n_copies):
+        st = DecodeStep(sessions[i], B, s_q, inp.block_table.shape[1], len(last), kernel=kernel)
+        for key, name in names.items():
+            st.host_in[name].copy_(torch.from_numpy(np.ascontiguousarray(host[key])).to(st.host_in[name].dtype))
+        st.capture()
+        steps.append(st)
+    h2d, d2h = steps[0].h2d_bytes, steps[0].d2h_bytes
 
     for k in range(args.warmup):
-        e2e_step(k)
+        steps[k % n_copies].run()
     barrier(device)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for k in range(args.steps):
-        e2e_step(k)
+        steps[k % n_copies].run()
     e1.record()
     torch.cuda.synchronize(device)
     e2e_ms = reduce_max(e0.elapsed_time(e1), device) / args.steps
@@ -502,7 +499,8 @@ def run_ours(args, world, rank, local):
                                 "what": "decode split kernel, a_k cache vs a_k = 1, median of interleaved rounds"},
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "what": "DecodeSession append/absorb/decode, eager, pinned host in/out, sync per step"},
+                    "what": "DecodeStep.run(): one graph per step with copy-in from pinned host buffers, "
+                            "append || absorb, decode, copy-out to pinned host buffers; synchronize per step"},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": sampler.summary(window),
             "cpu_baseline": cpu,

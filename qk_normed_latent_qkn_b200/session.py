@@ -58,13 +58,17 @@ class DecodeSession:
         d, dt, dev = self.dims, self.dims.torch_dtype, self.device
         q = to_device(q, dt, dev)
         q_rope = to_device(q_rope, dt, dev)
-        n_q = q.shape[0]
+        self.ensure_query_buffers(q.shape[0])
+        absorb_query(d, q, q_rope, to_device(pos, torch.int32, dev), self.w_k, self.gamma_q, self.gamma_k,
+                     self.gamma_qr, self.q_tilde, self.a_q, self.q_rope_hat)
+
+    def ensure_query_buffers(self, n_q: int) -> None:
+        """Device buffers for q~, a_q and q^R^ of n_q query rows (kept while n_q stays the same)."""
+        d, dt, dev = self.dims, self.dims.torch_dtype, self.device
         if self.q_tilde is None or self.q_tilde.shape[0] != n_q:
             self.q_tilde = torch.empty((n_q, d.num_heads, d.r_kv), dtype=dt, device=dev)
             self.a_q = torch.empty((n_q, d.num_heads), dtype=torch.float32, device=dev)
             self.q_rope_hat = torch.empty((n_q, d.num_heads, d.d_rope), dtype=dt, device=dev)
-        absorb_query(d, q, q_rope, to_device(pos, torch.int32, dev), self.w_k, self.gamma_q, self.gamma_k,
-                     self.gamma_qr, self.q_tilde, self.a_q, self.q_rope_hat)
 
     # ------------------------------------------------------------ decode
     def ensure_workspace(self, batch: int, s_q: int) -> torch.Tensor:
