@@ -114,6 +114,23 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------- CUDA events that survive capture
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the split-KV kernel from the committed ncu capture, if that capture
+    was taken on this workload with the kernel source as it is now; else None."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        with open(os.path.join(here, "profiles", "decode_tc_traffic.json")) as f:
+            rec = json.load(f)
+        with open(os.path.join(here, rec["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload or rec.get("source_sha256") != sha:
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
 class Events:
     """Raw cudaEvent_t handles recorded with cudaEventRecordExternal, so that a
     record inside stream capture becomes an event node of the graph."""
@@ -459,6 +476,7 @@ def run_ours(args, world, rank, local):
     achieved_gbs = cost.bytes / (op_avg * 1e-3) / 1e9
     tflops = cost.flops / (op_avg * 1e-3) / 1e12
     tokens = world * B * s_q
+    traffic = load_traffic(wl.name) if kernel_used == qkn.KERNEL_TCGEN05 else None
 
     line = None
     if rank == 0:
@@ -488,7 +506,10 @@ def run_ours(args, world, rank, local):
                                      "separate graphs with an event between every stage; decode_op_timed is the "
                                      "split-KV + merge pair inside the timed steps"},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                         "traffic_what": ("DRAM read + write bytes of one split-KV kernel launch from the "
+                                          "committed ncu capture (profiles/); null when the kernel source "
+                                          "or the workload differs from the capture's"),
                          "algorithmic_bytes": cost.bytes, "peak_source": f"{peak_src} HBM copy bandwidth",
                          "kernel": ("decode op: split-KV kernel (tcgen05) + merge kernel, averaged over the timed "
                                     "steps" if kernel_used == qkn.KERNEL_TCGEN05 else
