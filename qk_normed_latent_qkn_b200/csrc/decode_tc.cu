@@ -418,12 +418,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     mbar_wait_warp(smem_u32(&ms.drain), 0, kDrainLimit);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int t = threadIdx.x;                         // latent row of each O^T block / TMEM lane
+    // Thread t of the 128: in the 64-row score layout it holds token `tok` of the page (TMEM lane
+    // tok % 16 of warp tok / 16) and the columns of parity `par`: column 2j + par in its slot j.
+    // In the 128-row O^T layout it holds latent row t of each block.
+    const int t = threadIdx.x;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int tok = warp * 16 + lane;                  // token of the page held in this lane (lane < 16)
-    const bool has_tok = lane < 16;
+    const int tok = warp * 16 + (lane >> 2) + 8 * (lane & 1);
+    const int par = (lane >> 1) & 1;
+    constexpr int NJ = R / 2;                          // columns per thread
+    // per-column values are stored parity-major: column c at pm(c)
+    auto pm = [](int c) { return (c & 1) * NJ + (c >> 1); };
+    const float* aq_p = ms.aq2 + par * NJ;
+    const int32_t* ql_p = ms.qlim + par * NJ;
+    const int32_t* grp_p = ms.grp + par * NJ;
+    float* mu_p = ms.mu + par * NJ;
+    const float* corr_p = ms.corr + par * NJ;
     auto pv_wait = [&](int64_t n) {
       return mbar_wait(smem_u32(&ms.pv_done[n & 1]), (uint32_t)((n >> 1) & 1), a.wait_limit);
+    };
+    // maximum (MAX) or sum over the 16 threads of the warp that hold the same columns (lane bits
+    // 0, 2, 3, 4 vary); threads with lane 0 / 2 then store their parity's columns into red[warp]
+    auto reduce_store = [&](float (&v)[NJ], bool is_max) {
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+        for (int o : {1, 4, 8, 16}) {
+          const float u = __shfl_xor_sync(0xffffffffu, v[j], o);
+          v[j] = is_max ? fmaxf(v[j], u) : v[j] + u;
+        }
+      }
+      if ((lane & ~2) == 0) {
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) ms.red[warp][par * NJ + j] = v[j];
+      }
     };
     const int ng = a.heads / G;
     RingPos<NKR> kr;
@@ -443,15 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const bool valid = rho < qrows;
         const int j = valid ? rho / a.heads : 0;
         const int h = valid ? rho - j * a.heads : 0;
-        ms.aq2[t] = valid ? a.a_q[(int64_t)it.b * qrows + rho] * kLog2e : 0.f;
-        ms.grp[t] = h / ng;
-        ms.qlim[t] = valid ? it.L - a.s_q + j : -1;
-        ms.mu[t] = -INFINITY;
+        ms.aq2[pm(t)] = valid ? a.a_q[(int64_t)it.b * qrows + rho] * kLog2e : 0.f;
+        ms.grp[pm(t)] = h / ng;
+        ms.qlim[pm(t)] = valid ? it.L - a.s_q + j : -1;
+        ms.mu[pm(t)] = -INFINITY;
       }
       named_bar_sync(1, kSoftThreads);
-      float lpart[R];
+      float lpart[NJ];
 #pragma unroll
-      for (int c = 0; c < R; ++c) lpart[c] = 0.f;
+      for (int j = 0; j < NJ; ++j) lpart[j] = 0.f;
       for (int p = it.p0; p < it.p1; ++p) {
         const int tok0 = p * kPage;
         const int nvalid = min(kPage, it.L - tok0);
@@ -465,61 +492,68 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         // the phase waited for, which a parity wait needs.
         if (t == 0 && tile_n > 1) got = pv_wait(tile_n - 2) && got;
         tc_fence_after();
-        const bool row_ok = has_tok && tok < nvalid;
+        const bool row_ok = tok < nvalid;
         const int tpos = tok0 + tok;
-        const float* akrow = reinterpret_cast<const float*>(smem + C::AK_OFF + ks * kAkSlotBytes) + (has_tok ? tok : 0) * G;
+        const float* akrow = reinterpret_cast<const float*>(smem + C::AK_OFF + ks * kAkSlotBytes) + tok * G;
         float ak0 = 1.f;
         if (!AK_ONE) {
           // the RoPE-key barrier also covers the a_k rows; it completed before S did
           got = mbar_wait(smem_u32(&ms.krfull[ks]), kr.phase, a.wait_limit) && got;
           ak0 = akrow[0];
         }
-        // this token's scaled logits in log2 units (-inf where not visible)
-        auto load_logits = [&](float (&x)[R]) {
+        // this token's scaled logits, log2 units, of this thread's columns (-inf where not visible)
+        float x[NJ];
+        {
+          constexpr int NL = NJ < 16 ? NJ : 16;        // registers per 16x64b load
 #pragma unroll
-          for (int c0 = 0; c0 < R; c0 += 16) {
-            uint32_t sc[16], sr[16];
-            tmem_ld16(tSc + c0, sc);
-            tmem_ld16(tSc + R + c0, sr);
-            float aq[16];
-            int ql[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              *reinterpret_cast<float4*>(aq + 4 * q) = *reinterpret_cast<const float4*>(ms.aq2 + c0 + 4 * q);
-              *reinterpret_cast<int4*>(ql + 4 * q) = *reinterpret_cast<const int4*>(ms.qlim + c0 + 4 * q);
+          for (int b0 = 0; b0 < NJ; b0 += NL) {
+            uint32_t sc[NL], sr[NL];
+            if constexpr (NL == 8) {
+              tmem_ld16x64_x8(tSc + 2 * b0, sc);
+              tmem_ld16x64_x8(tSc + R + 2 * b0, sr);
+            } else {
+              tmem_ld16x64_x16(tSc + 2 * b0, sc);
+              tmem_ld16x64_x16(tSc + R + 2 * b0, sr);
             }
-            tmem_wait_ld(sc, sr);
+            tmem_wait_ld();
+            reg_tie(sc);
+            reg_tie(sr);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float akc = ak0;
-              if (!AK_ONE && G > 1) akc = akrow[ms.grp[c0 + e]];
-              const float v = aq[e] * akc * __uint_as_float(sc[e]) + kLog2e * __uint_as_float(sr[e]);
-              x[c0 + e] = (row_ok && tpos <= ql[e]) ? v : -INFINITY;
+            for (int q = 0; q < NL; q += 4) {
+              const float4 aq4 = *reinterpret_cast<const float4*>(aq_p + b0 + q);
+              const int4 ql4 = *reinterpret_cast<const int4*>(ql_p + b0 + q);
+              const float aqv[4] = {aq4.x, aq4.y, aq4.z, aq4.w};
+              const int qlv[4] = {ql4.x, ql4.y, ql4.z, ql4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float akc = ak0;
+                if (!AK_ONE && G > 1) akc = akrow[grp_p[b0 + q + e]];
+                const float v = aqv[e] * akc * __uint_as_float(sc[q + e]) + kLog2e * __uint_as_float(sr[q + e]);
+                x[b0 + q + e] = (row_ok && tpos <= qlv[e]) ? v : -INFINITY;
+              }
             }
           }
-        };
-        float x[R];
-        load_logits(x);
+        }
         // Fast path: the exponentials are taken against the running reference mu, which only has
         // to stay within 2^8 of the true column maximum.  One group vote finds out whether any
         // logit of the tile passed mu + 8; only then are the column maxima reduced.
         bool over = false;
 #pragma unroll
-        for (int c0 = 0; c0 < R; c0 += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(ms.mu + c0);
-          over |= (x[c0] > m4.x + kRescaleLog2) | (x[c0 + 1] > m4.y + kRescaleLog2) |
-                  (x[c0 + 2] > m4.z + kRescaleLog2) | (x[c0 + 3] > m4.w + kRescaleLog2);
+        for (int j = 0; j < NJ; j += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(mu_p + j);
+          over |= (x[j] > m4.x + kRescaleLog2) | (x[j + 1] > m4.y + kRescaleLog2) |
+                  (x[j + 2] > m4.z + kRescaleLog2) | (x[j + 3] > m4.w + kRescaleLog2);
         }
         if (group_any(over || !got)) {
           if (group_any(!got)) { ok = false; break; }
-          float v[R];
+          float v[NJ];
 #pragma unroll
-          for (int c = 0; c < R; ++c) v[c] = x[c];
-          warp_col_reduce<R, true>(v, lane);
-          store_reduced<R>(ms.red[warp], v, lane);
+          for (int j = 0; j < NJ; ++j) v[j] = x[j];
+          reduce_store(v, true);
           named_bar_sync(1, kSoftThreads);
           bool mine = false;
           if (t < R) {
+            // thread t < R updates column slot t (parity-major order)
             const float mt = fmaxf(fmaxf(ms.red[0][t], ms.red[1][t]), fmaxf(ms.red[2][t], ms.red[3][t]));
             const float mo = ms.mu[t];
             float cr = 1.f;
@@ -545,55 +579,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
                 tmem_ld16(tl + m * R + c0, ov);
                 tmem_wait_ld(ov);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[c0 + e]);
+                for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[pm(c0 + e)]);
                 tmem_st16(tl + m * R + c0, ov);
                 tmem_wait_st();
               }
             }
           }
 #pragma unroll
-          for (int c = 0; c < R; ++c) lpart[c] *= ms.corr[c];
+          for (int j = 0; j < NJ; ++j) lpart[j] *= corr_p[j];
         }
-        // probabilities, running column sums, and P^T into the RoPE-key slot, token-major:
-        // row `tok` holds this token's R probabilities (2R bytes), 16-byte units swizzled by row
-        uint8_t* prow = smem + C::KR_OFF + ks * kKrBytes + (has_tok ? tok : 0) * (2 * R);
-        const int swz = (R == 16) ? ((tok >> 2) & 1) : (R == 32) ? ((tok >> 1) & 3) : (tok & 7);
+        // probabilities, running column sums, and P^T into the RoPE-key slot, token-major: row `tok`
+        // holds the token's R probabilities (2R bytes), 16-byte units swizzled by row.  The two threads
+        // of a token swap a quarter of their values (shuffle with lane ^ 2), so that each holds complete
+        // column pairs: parity 0 columns 0 .. R/2 - 1, parity 1 columns R/2 .. R - 1.
+        {
+          float pr[NJ];
 #pragma unroll
-        for (int c0 = 0; c0 < R; c0 += 16) {
-          float mu[16];
+          for (int j = 0; j < NJ; j += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(mu_p + j);
+            const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<float4*>(mu + 4 * q) = *reinterpret_cast<const float4*>(ms.mu + c0 + 4 * q);
-          uint32_t packed[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float pp[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int c = c0 + e + u;
-              const float pr = x[c] == -INFINITY ? 0.f : ex2(x[c] - mu[e + u]);
-              lpart[c] += pr;
-              pp[u] = pr;
+            for (int e = 0; e < 4; ++e) {
+              pr[j + e] = x[j + e] == -INFINITY ? 0.f : ex2(x[j + e] - mv[e]);
+              lpart[j + e] += pr[j + e];
             }
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(pp[0], pp[1]);
-            packed[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
           }
-          if (has_tok) {
-            const int u0 = c0 / 8;    // 16-byte units c0/8 and c0/8 + 1 of the row
-            *reinterpret_cast<uint4*>(prow + (((u0 + 0) ^ swz) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            *reinterpret_cast<uint4*>(prow + (((u0 + 1) ^ swz) << 4)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          constexpr int NP = NJ / 2;                     // column pairs each thread writes
+          uint32_t words[NP];
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            const float send = par == 0 ? pr[j + NP] : pr[j];
+            const float got2 = __shfl_xor_sync(0xffffffffu, send, 2);
+            // parity 0: columns (2j, 2j + 1) = (mine, partner's); parity 1: columns
+            // (2(j + NP), 2(j + NP) + 1) = (partner's, mine)
+            const __nv_bfloat162 b2 = par == 0 ? __floats2bfloat162_rn(pr[j], got2)
+                                               : __floats2bfloat162_rn(got2, pr[j + NP]);
+            words[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint8_t* prow = smem + C::KR_OFF + ks * kKrBytes + tok * (2 * R);
+          const int swz = (R == 16) ? ((tok >> 2) & 1) : (R == 32) ? ((tok >> 1) & 3) : (tok & 7);
+#pragma unroll
+          for (int u = 0; u < NP / 4; ++u) {
+            const int unit = par * (NP / 4) + u;         // 16-byte unit of the row
+            *reinterpret_cast<uint4*>(prow + ((unit ^ swz) << 4)) =
+                make_uint4(words[4 * u], words[4 * u + 1], words[4 * u + 2], words[4 * u + 3]);
           }
         }
         // the S buffer is free for the tile after next
         tc_fence_before();
         mbar_arrive(smem_u32(&ms.s_empty[sbuf]));
-        // rows of the page past the context: zero them so that 0 * garbage cannot reach O
-        if (has_tok && !row_ok) {
+        // rows of the page past the context: zero them so that 0 * garbage cannot reach O (the two
+        // threads of a token take four of its eight chunks each)
+        if (!row_ok) {
 #pragma unroll
-          for (int k = 0; k < kChunks; ++k) {
+          for (int k = par * 4; k < par * 4 + 4; ++k) {
             const int sl = c_first + k / 2 < NS ? c_first + k / 2 : c_first + k / 2 - NS;
-            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + sl * kSlotBytes +
-                                                   (k & 1) * kChunkBytes + tok * 128);
+            uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + sl * kSlotBytes + (k & 1) * kChunkBytes + tok * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q) rowp[q] = make_uint4(0, 0, 0, 0);
           }
@@ -614,13 +655,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       }
       if (!group_all(got)) { ok = false; break; }
       tc_fence_after();
-      warp_col_reduce<R, false>(lpart, lane);
-      store_reduced<R>(ms.red[warp], lpart, lane);
+      reduce_store(lpart, false);
       named_bar_sync(1, kSoftThreads);
       if (t < R) {
-        const float l = ms.red[0][t] + ms.red[1][t] + ms.red[2][t] + ms.red[3][t];
+        const int c = pm(t);
+        const float l = ms.red[0][c] + ms.red[1][c] + ms.red[2][c] + ms.red[3][c];
         ms.linv[t] = l > 0.f ? 1.f / l : 0.f;
-        a.part_lse[(int64_t)it.slot * R + t] = l > 0.f ? (ms.mu[t] + log2f(l)) * kLn2 : -INFINITY;
+        a.part_lse[(int64_t)it.slot * R + t] = l > 0.f ? (ms.mu[c] + log2f(l)) * kLn2 : -INFINITY;
       }
       named_bar_sync(1, kSoftThreads);
       float* po = a.part_o + (int64_t)it.slot * R * kRkv;
