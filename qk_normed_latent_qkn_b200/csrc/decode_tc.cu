@@ -69,7 +69,9 @@ constexpr int64_t kDrainLimit = 4000000000LL;
 
 template <int R>
 struct Cfg {
-  static constexpr int NKR = (R == 64) ? 3 : 4;              // RoPE-key / a_k / P^T slots
+  // RoPE-key / a_k / P^T slots: a page holds one from its load until its output MMAs finish; at R = 64
+  // two suffice (the latent ring holds two pages), which leaves room for an eighth latent slot
+  static constexpr int NKR = (R == 64) ? 2 : 4;
   static constexpr int TMEM_COLS = (8 * R <= 128) ? 128 : (8 * R <= 256 ? 256 : 512);
   static constexpr int Q_OFF = 0;                                    // R x 512 bf16, 8 chunks
   static constexpr int QR_OFF = Q_OFF + R * 1024;                    // R x 64 bf16
