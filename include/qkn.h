@@ -98,12 +98,20 @@ typedef struct {
  *   a_k    [num_blocks, block_size, num_groups] fp32
  * Slot s of the pool is token s % block_size of block s / block_size.
  * Slots that no qkn_append has written may hold anything; decode never lets
- * them reach its output. */
+ * them reach its output.
+ *   ak_scratch [num_blocks, block_size, num_groups, 2] 32-bit words, optional:
+ *     zero when allocated (e.g. cudaMemset); every qkn_append that completes
+ *     leaves it zero again.  With it, qkn_append runs as one launch (a key
+ *     statistic accumulator and an arrival count per slot and group); with
+ *     NULL it runs as three.  After an append that did not complete (a
+ *     sticky CUDA error), clear it again before the next append.  Decode
+ *     does not read it. */
 typedef struct {
   void* latent;
   void* k_rope;
   float* a_k;
   int32_t num_blocks;
+  uint32_t* ak_scratch;
 } qkn_cache;
 
 /* Optional decode knobs (pass NULL for defaults). */

@@ -45,7 +45,7 @@ class _Dims(ctypes.Structure):
 
 class _Cache(ctypes.Structure):
     _fields_ = [("latent", ctypes.c_void_p), ("k_rope", ctypes.c_void_p), ("a_k", ctypes.c_void_p),
-                ("num_blocks", ctypes.c_int32)]
+                ("num_blocks", ctypes.c_int32), ("ak_scratch", ctypes.c_void_p)]
 
 
 class _Opts(ctypes.Structure):
@@ -127,9 +127,12 @@ class Cache:
         self.latent = torch.empty((num_blocks, bs, dims.r_kv), dtype=dims.torch_dtype, device=device)
         self.k_rope = torch.empty((num_blocks, bs, dims.d_rope), dtype=dims.torch_dtype, device=device)
         self.a_k = torch.empty((num_blocks, bs, dims.num_groups), dtype=torch.float32, device=device)
+        # append's per-slot accumulator and arrival count; zero now, left zero by every append
+        self.ak_scratch = torch.zeros((num_blocks, bs, dims.num_groups, 2), dtype=torch.int32, device=device)
 
     def c(self) -> _Cache:
-        return _Cache(self.latent.data_ptr(), self.k_rope.data_ptr(), self.a_k.data_ptr(), self.num_blocks)
+        return _Cache(self.latent.data_ptr(), self.k_rope.data_ptr(), self.a_k.data_ptr(), self.num_blocks,
+                      self.ak_scratch.data_ptr())
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

@@ -35,7 +35,8 @@ qkn_status check_dims(const qkn_dims* d) {
 
 qkn_status check_cache(const qkn_dims* d, const qkn_cache* c) {
   if (!c || !c->latent || !c->k_rope || !c->a_k || c->num_blocks <= 0) return QKN_ERR_INVALID_ARG;
-  if (!aligned(c->latent, 16) || !aligned(c->k_rope, 16) || !aligned(c->a_k, 16)) return QKN_ERR_INVALID_ARG;
+  if (!aligned(c->latent, 16) || !aligned(c->k_rope, 16) || !aligned(c->a_k, 16) || !aligned(c->ak_scratch, 8))
+    return QKN_ERR_INVALID_ARG;
   if ((int64_t)c->num_blocks * kBlockSize > INT32_MAX) return QKN_ERR_INVALID_ARG;
   (void)d;
   return QKN_OK;
@@ -141,6 +142,7 @@ qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache, const void* 
   a.latent = cache->latent;
   a.k_rope = cache->k_rope;
   a.a_k = cache->a_k;
+  a.ak_scratch = cache->ak_scratch;
   a.c_new = c_new;
   a.k_rope_raw = k_rope_raw;
   a.slot = slot;

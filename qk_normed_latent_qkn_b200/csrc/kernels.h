@@ -19,6 +19,7 @@ struct AppendArgs {
   void* latent;            // cache pool
   void* k_rope;
   float* a_k;
+  uint32_t* ak_scratch;    // [slots, groups, 2]: key statistic accumulator, arrival count; or null
   const void* c_new;       // [n_tok, r]
   const void* k_rope_raw;  // [n_tok, d_rope]
   const int32_t* slot;
