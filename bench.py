@@ -38,8 +38,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "decode tokens/s and us/step at 1 B200; % of HBM/tensor roofline; overhead vs MLA"
-# kernels of libqkn launched per step: append (copy, key RMS, finalize), absorb, split-KV decode, merge
-LAUNCHES_PER_STEP = 6
+# kernels of libqkn launched per step: append + absorb (one launch), split-KV decode, merge
+LAUNCHES_PER_STEP = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -312,22 +312,23 @@ def run_ours(args, world, rank, local):
     outs = [(torch.empty((B, s_q, H, wl.r_kv), dtype=dt, device=device),
              torch.empty((B, s_q, H), dtype=torch.float32, device=device)) for _ in sessions]
 
-    side = torch.cuda.Stream(device=device)
+    evs = torch.cuda.Stream(device=device)
 
     def step(i, split_event=None, ak_mode=qkn.AK_CACHE, start_event=None, end_event=None):
-        """Append and absorb are independent: absorb runs on a side stream, joined before decode."""
+        """Append and absorb in one launch, then the split-KV decode and its merge, all on one stream.
+        The start event is recorded on a branch that joins only at the end of the step, so that no
+        graph node sits between the preparation and the decode."""
         s, d, (o, l) = sessions[i], dev_in[i], outs[i]
         main = torch.cuda.current_stream(device)
-        side.wait_stream(main)
-        with torch.cuda.stream(side):
-            s.absorb(d["q"], d["qr"], d["qpos"])
-        s.append(d["c"], d["kr"], d["slot"], d["pos"])
-        main.wait_stream(side)
+        s.prepare(d["c"], d["kr"], d["slot"], d["pos"], d["q"], d["qr"], d["qpos"])
         if start_event is not None:
-            ev.record(start_event, main.cuda_stream)
+            evs.wait_stream(main)
+            ev.record(start_event, evs.cuda_stream)
         s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event)
         if end_event is not None:
             ev.record(end_event, main.cuda_stream)
+        if start_event is not None:
+            main.wait_stream(evs)
 
     def decode_only(i, split_event=None, ak_mode=qkn.AK_CACHE):
         s, d, (o, l) = sessions[i], dev_in[i], outs[i]

@@ -164,6 +164,25 @@ QKN_EXPORT qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, cons
                             const float* gamma_q, const float* gamma_k, const float* gamma_qr,
                             void* q_tilde, float* a_q, void* q_rope_hat, void* stream);
 
+/* qkn_append_absorb — qkn_append followed by qkn_absorb_query, in one launch
+ * where possible.  The two steps are independent (technical summary,
+ * Metodología items 1-4): the append writes the cache's new tokens and their
+ * key statistic, the absorption folds the norm weights into the step's
+ * queries; neither reads what the other writes.  Arguments are those of the
+ * two calls (qpos are the query rows' RoPE positions; w_k is shared), with
+ * the same layouts, validation and results.  One launch is used when the
+ * cache carries ak_scratch, 0 < n_tok <= 256 and n_q > 0; otherwise the two
+ * steps run as their own launches, in this order, on `stream`.  It exists so
+ * that a decode step can prepare its inputs without forking two streams;
+ * the pages have no counterpart. */
+QKN_EXPORT qkn_status qkn_append_absorb(const qkn_dims* dims, const qkn_cache* cache,
+                      const void* c_new, const void* k_rope_raw,
+                      const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                      const void* q, const void* q_rope, const int32_t* qpos, int32_t n_q,
+                      const float* w_k, const float* gamma_q, const float* gamma_k,
+                      const float* gamma_qr, const float* gamma_kr,
+                      void* q_tilde, float* a_q, void* q_rope_hat, void* stream);
+
 /* Bytes of decode workspace needed for `batch` sequences of `s_q` query
  * tokens on a GPU with `num_sms` SMs (0 = ask the current device).  The
  * workspace holds a status word and the per-split partial results of the

@@ -26,7 +26,7 @@ KERNEL_AUTO, KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1, 2
 
 EXPORTED = ["qkn_append", "qkn_absorb_query", "qkn_decode_workspace_size", "qkn_workspace_init",
             "qkn_decode", "qkn_read_device_status", "qkn_decode_kernel_for", "qkn_status_string",
-            "qkn_version", "qkn_decode_noalloc"]
+            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "qkn_status_string": (ctypes.c_char_p, [I32]),
         "qkn_version": (I32, []),
         "qkn_decode_noalloc": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, P, P, PO, P]),
+        "qkn_append_absorb": (I32, [PD, PC, P, P, P, P, I32, P, P, P, I32, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -132,7 +133,7 @@ class Cache:
 
     def c(self) -> _Cache:
         return _Cache(self.latent.data_ptr(), self.k_rope.data_ptr(), self.a_k.data_ptr(), self.num_blocks,
-                      self.ak_scratch.data_ptr())
+                      None if self.ak_scratch is None else self.ak_scratch.data_ptr())
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -165,6 +166,16 @@ def absorb_query(dims: Dims, q, q_rope, pos, w_k, gamma_q, gamma_k, gamma_qr, q_
     _check(_lib.qkn_absorb_query(ctypes.byref(dims.c()), _ptr(q), _ptr(q_rope), _ptr(pos), n_q, _ptr(w_k),
                                  _ptr(gamma_q), _ptr(gamma_k), _ptr(gamma_qr), _ptr(q_tilde), _ptr(a_q),
                                  _ptr(q_rope_hat), _stream(stream)), "qkn_absorb_query")
+
+
+def append_absorb(dims: Dims, cache: Cache, c_new, k_rope_raw, slot, pos, q, q_rope, qpos, w_k, gamma_q, gamma_k,
+                  gamma_qr, gamma_kr, q_tilde, a_q, q_rope_hat, stream=None) -> None:
+    """qkn_append followed by qkn_absorb_query, in one launch where possible (see qkn_append_absorb)."""
+    _check(_lib.qkn_append_absorb(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(c_new), _ptr(k_rope_raw),
+                                  _ptr(slot), _ptr(pos), int(c_new.shape[0]), _ptr(q), _ptr(q_rope), _ptr(qpos),
+                                  int(q.shape[0]), _ptr(w_k), _ptr(gamma_q), _ptr(gamma_k), _ptr(gamma_qr),
+                                  _ptr(gamma_kr), _ptr(q_tilde), _ptr(a_q), _ptr(q_rope_hat), _stream(stream)),
+           "qkn_append_absorb")
 
 
 def decode_workspace_size(dims: Dims, batch: int, s_q: int, num_sms: int = 0) -> int:

@@ -128,35 +128,90 @@ const char* qkn_status_string(qkn_status s) {
 
 int32_t qkn_version(void) { return QKN_VERSION; }
 
-qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache, const void* c_new,
-                      const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
-                      const float* w_k, const float* gamma_kr, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validated launch arguments of an append (n_tok > 0) or QKN_OK with *empty for n_tok == 0.
+qkn_status append_args(const qkn_dims* dims, const qkn_cache* cache, const void* c_new, const void* k_rope_raw,
+                       const int32_t* slot, const int32_t* pos, int32_t n_tok, const float* w_k,
+                       const float* gamma_kr, AppendArgs* a, bool* empty) {
   qkn_status st = check_dims(dims);
   if (st != QKN_OK) return st;
   if (n_tok < 0) return QKN_ERR_INVALID_ARG;
-  if (n_tok == 0) return QKN_OK;
+  *empty = n_tok == 0;
+  if (*empty) return QKN_OK;
   if ((st = check_cache(dims, cache)) != QKN_OK) return st;
   if (!c_new || !k_rope_raw || !slot || !pos || !w_k || !gamma_kr) return QKN_ERR_INVALID_ARG;
   if (!aligned(c_new, 16) || !aligned(k_rope_raw, 16)) return QKN_ERR_INVALID_ARG;
+  a->latent = cache->latent;
+  a->k_rope = cache->k_rope;
+  a->a_k = cache->a_k;
+  a->ak_scratch = cache->ak_scratch;
+  a->c_new = c_new;
+  a->k_rope_raw = k_rope_raw;
+  a->slot = slot;
+  a->pos = pos;
+  a->w_k = w_k;
+  a->gamma_kr = gamma_kr;
+  a->n_tok = n_tok;
+  a->r = dims->r_kv;
+  a->d_rope = dims->d_rope;
+  a->groups = dims->num_groups;
+  a->width = (dims->num_heads / dims->num_groups) * dims->d_h;
+  a->eps = dims->eps;
+  a->rope_theta = dims->rope_theta;
+  a->freq = rope_freqs(dims);
+  return QKN_OK;
+}
+
+// Validated launch arguments of a query absorption (n_q > 0) or QKN_OK with *empty for n_q == 0.
+qkn_status absorb_args(const qkn_dims* dims, const void* q, const void* q_rope, const int32_t* pos, int32_t n_q,
+                       const float* w_k, const float* gamma_q, const float* gamma_k, const float* gamma_qr,
+                       void* q_tilde, float* a_q, void* q_rope_hat, AbsorbArgs* a, bool* empty) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (n_q < 0) return QKN_ERR_INVALID_ARG;
+  *empty = n_q == 0;
+  if (*empty) return QKN_OK;
+  if (!q || !q_rope || !pos || !w_k || !gamma_q || !gamma_k || !gamma_qr || !q_tilde || !a_q || !q_rope_hat)
+    return QKN_ERR_INVALID_ARG;
+  if (dims->d_h > 256 || dims->d_h % 4) return QKN_ERR_UNSUPPORTED;
+  if (!aligned(w_k, 16) || !aligned(gamma_q, 16) || !aligned(gamma_k, 16)) return QKN_ERR_INVALID_ARG;
+  a->q = q;
+  a->q_rope = q_rope;
+  a->pos = pos;
+  a->w_k = w_k;
+  a->gamma_q = gamma_q;
+  a->gamma_k = gamma_k;
+  a->gamma_qr = gamma_qr;
+  a->q_tilde = q_tilde;
+  a->a_q = a_q;
+  a->q_rope_hat = q_rope_hat;
+  a->n_q = n_q;
+  a->heads = dims->num_heads;
+  a->groups = dims->num_groups;
+  a->r = dims->r_kv;
+  a->d_h = dims->d_h;
+  a->d_rope = dims->d_rope;
+  a->eps = dims->eps;
+  a->softmax_scale = dims->softmax_scale;
+  a->rope_theta = dims->rope_theta;
+  a->freq = rope_freqs(dims);
+  return QKN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache, const void* c_new,
+                      const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                      const float* w_k, const float* gamma_kr, void* stream) {
   AppendArgs a;
-  a.latent = cache->latent;
-  a.k_rope = cache->k_rope;
-  a.a_k = cache->a_k;
-  a.ak_scratch = cache->ak_scratch;
-  a.c_new = c_new;
-  a.k_rope_raw = k_rope_raw;
-  a.slot = slot;
-  a.pos = pos;
-  a.w_k = w_k;
-  a.gamma_kr = gamma_kr;
-  a.n_tok = n_tok;
-  a.r = dims->r_kv;
-  a.d_rope = dims->d_rope;
-  a.groups = dims->num_groups;
-  a.width = (dims->num_heads / dims->num_groups) * dims->d_h;
-  a.eps = dims->eps;
-  a.rope_theta = dims->rope_theta;
-  a.freq = rope_freqs(dims);
+  bool empty = false;
+  qkn_status st = append_args(dims, cache, c_new, k_rope_raw, slot, pos, n_tok, w_k, gamma_kr, &a, &empty);
+  if (st != QKN_OK || empty) return st;
   cudaError_t e = launch_append(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
 }
@@ -165,36 +220,37 @@ qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_r
                             int32_t n_q, const float* w_k, const float* gamma_q, const float* gamma_k,
                             const float* gamma_qr, void* q_tilde, float* a_q, void* q_rope_hat,
                             void* stream) {
-  qkn_status st = check_dims(dims);
-  if (st != QKN_OK) return st;
-  if (n_q < 0) return QKN_ERR_INVALID_ARG;
-  if (n_q == 0) return QKN_OK;
-  if (!q || !q_rope || !pos || !w_k || !gamma_q || !gamma_k || !gamma_qr || !q_tilde || !a_q || !q_rope_hat)
-    return QKN_ERR_INVALID_ARG;
-  if (dims->d_h > 256 || dims->d_h % 4) return QKN_ERR_UNSUPPORTED;
-  if (!aligned(w_k, 16) || !aligned(gamma_q, 16) || !aligned(gamma_k, 16)) return QKN_ERR_INVALID_ARG;
   AbsorbArgs a;
-  a.q = q;
-  a.q_rope = q_rope;
-  a.pos = pos;
-  a.w_k = w_k;
-  a.gamma_q = gamma_q;
-  a.gamma_k = gamma_k;
-  a.gamma_qr = gamma_qr;
-  a.q_tilde = q_tilde;
-  a.a_q = a_q;
-  a.q_rope_hat = q_rope_hat;
-  a.n_q = n_q;
-  a.heads = dims->num_heads;
-  a.groups = dims->num_groups;
-  a.r = dims->r_kv;
-  a.d_h = dims->d_h;
-  a.d_rope = dims->d_rope;
-  a.eps = dims->eps;
-  a.softmax_scale = dims->softmax_scale;
-  a.rope_theta = dims->rope_theta;
-  a.freq = rope_freqs(dims);
+  bool empty = false;
+  qkn_status st = absorb_args(dims, q, q_rope, pos, n_q, w_k, gamma_q, gamma_k, gamma_qr, q_tilde, a_q,
+                              q_rope_hat, &a, &empty);
+  if (st != QKN_OK || empty) return st;
   cudaError_t e = launch_absorb(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+qkn_status qkn_append_absorb(const qkn_dims* dims, const qkn_cache* cache, const void* c_new,
+                             const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                             const void* q, const void* q_rope, const int32_t* qpos, int32_t n_q,
+                             const float* w_k, const float* gamma_q, const float* gamma_k, const float* gamma_qr,
+                             const float* gamma_kr, void* q_tilde, float* a_q, void* q_rope_hat, void* stream) {
+  AppendArgs ap;
+  AbsorbArgs ab;
+  bool no_append = false, no_absorb = false;
+  qkn_status st = append_args(dims, cache, c_new, k_rope_raw, slot, pos, n_tok, w_k, gamma_kr, &ap, &no_append);
+  if (st != QKN_OK) return st;
+  st = absorb_args(dims, q, q_rope, qpos, n_q, w_k, gamma_q, gamma_k, gamma_qr, q_tilde, a_q, q_rope_hat, &ab,
+                   &no_absorb);
+  if (st != QKN_OK) return st;
+  const bool bf16 = dims->dtype == QKN_BF16;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (!no_append && !no_absorb && prep_fusable(ap, ab)) {
+    e = launch_prep(ap, ab, bf16, cs);
+  } else {
+    if (!no_append) e = launch_append(ap, bf16, cs);
+    if (e == cudaSuccess && !no_absorb) e = launch_absorb(ab, bf16, cs);
+  }
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
 }
 

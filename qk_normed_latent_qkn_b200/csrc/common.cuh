@@ -50,6 +50,17 @@ inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 bloc
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Opt a kernel into large dynamic shared memory and ask for the largest
+// shared-memory carveout, so that several of its CTAs fit on one SM (the
+// default carveout can hold the SM to one CTA of a kernel that uses 64 KB).
+template <typename... KArgs>
+inline cudaError_t set_smem_attrs(void (*kernel)(KArgs...), int max_dynamic_bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dynamic_bytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
+}
+
 // ---------------------------------------------------------------- RoPE
 // sin and cos of pos * freq.  The angle is formed and reduced to [-pi, pi] in
 // fp64 (one-constant reduction by 2*pi is exact to ~1e-11 here, positions stay

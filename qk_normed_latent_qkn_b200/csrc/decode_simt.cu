@@ -157,8 +157,7 @@ static cudaError_t launch_simt_nk(const DecodeArgs& a, cudaStream_t st) {
                       (size_t)kBlockSize * a.groups * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_simt_kernel<T, NK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaError_t e = set_smem_attrs(decode_simt_kernel<T, NK>, 200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }

@@ -87,6 +87,9 @@ struct CombineArgs {
 };
 
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);
+// One launch for both (prep.cu) when the append can run as one launch and is a decode step's size.
+bool prep_fusable(const AppendArgs& ap, const AbsorbArgs& ab);
+cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, cudaStream_t st);
 cudaError_t launch_absorb(const AbsorbArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_decode_simt(const DecodeArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st);

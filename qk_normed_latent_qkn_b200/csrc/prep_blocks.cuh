@@ -1,0 +1,388 @@
+// Device-side building blocks of the append and query-absorption kernels,
+// shared by their own launches (append.cu, absorb.cu) and by the one-launch
+// step preparation (prep.cu).  The functions take the CTA's block
+// coordinates and shared memory as arguments, so that one kernel can host
+// CTAs of both kinds.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qkn {
+
+// Token i of the call, by one warp: the latent row copied, the RoPE key
+// RMS-normalised, weighted and rotated.  `row` is the warp's 128-float
+// shared-memory buffer (d_R <= 128).
+template <typename T>
+__device__ __forceinline__ void append_token(const AppendArgs& a, int i, int lane, float* row) {
+  const int64_t slot = a.slot[i];
+  const int32_t pos = a.pos[i];
+  // latent row: 16-byte vectors (rows are a multiple of 16 bytes)
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(a.c_new) + (int64_t)i * a.r);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.latent) + slot * a.r);
+  const int nvec = a.r * (int)sizeof(T) / 16;
+  uint4 cv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int k = lane + 32 * u;
+    if (k < nvec) cv[u] = src[k];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int k = lane + 32 * u;
+    if (k < nvec) dst[k] = cv[u];
+  }
+  for (int k = lane + 128; k < nvec; k += 32) dst[k] = src[k];
+
+  // RoPE key: d_R <= 128, so each lane holds at most 4 elements.
+  const T* kr = static_cast<const T*>(a.k_rope_raw) + (int64_t)i * a.d_rope;
+  float x[4];
+  float ss = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k = lane + 32 * q;
+    x[q] = k < a.d_rope ? to_f32(kr[k]) : 0.f;
+    ss += x[q] * x[q];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / (float)a.d_rope + a.eps);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k = lane + 32 * q;
+    if (k < a.d_rope) x[q] = x[q] * inv * a.gamma_kr[k];
+  }
+  // Pair element k (< d/2) with k + d/2, which sits in lane (k + d/2) % 32 of
+  // slot (k + d/2) / 32.  Gather the partner through the warp's shared buffer.
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k = lane + 32 * q;
+    if (k < a.d_rope) row[k] = x[q];
+  }
+  __syncwarp();
+  T* kout = static_cast<T*>(a.k_rope) + slot * a.d_rope;
+  const int half = a.d_rope / 2;
+  for (int k = lane; k < half; k += 32) {
+    const float x1 = row[k], x2 = row[k + half];
+    float sn, cs;
+    rope_sincos(pos, a.freq.f[k], sn, cs);
+    kout[k] = from_f32<T>(x1 * cs - x2 * sn);
+    kout[k + half] = from_f32<T>(x2 * cs + x1 * sn);
+  }
+  __syncwarp();
+}
+
+// Key statistic sum(z^2), z = c W^K_g.  CTA = (16 key columns, TT tokens,
+// group); its 512 threads are 16 columns x 32 slices of the latent
+// dimension, so a decode step's handful of tokens still spreads over about a
+// hundred CTAs per group.  Every thread loads its slice of one W column in
+// one batch of independent loads and applies it to the TT tokens held in
+// shared memory; slices are summed in shared memory, squared, reduced over
+// the CTA's 16 columns and added into the token's a_k slot (zeroed by
+// append_copy_kernel).
+constexpr int kRmsCols = 16;
+constexpr int kRmsSlices = 32;
+
+// FUSED (the cache has ak_scratch): the whole append in this one launch.  One
+// more CTA column (block x == number of column blocks) copies the tile's
+// latents and RoPE keys; the column CTAs add their sums into the slot's
+// accumulator in ak_scratch and count themselves in, and the CTA whose count
+// completes a token writes a_k = 1 / sqrt(sum / width + eps) and returns the
+// accumulator and the count to zero.
+template <typename T, int TT, bool FUSED>
+__device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by, int bz, float* smem) {
+  float* cs = smem;                                               // [TT][r]
+  float* zp = cs + TT * a.r;                                      // [kRmsSlices][TT][kRmsCols]
+  const int g = bz;
+  const int t0 = by * TT;
+  const int ntok = min(TT, a.n_tok - t0);
+  const int width = a.width;
+  const int col = threadIdx.x % kRmsCols, slice = threadIdx.x / kRmsCols;
+  const int n = bx * kRmsCols + col;
+  const int nblk = (width + kRmsCols - 1) / kRmsCols;
+  if constexpr (FUSED) {
+    if (bx == nblk) {
+      __shared__ float rows[kRmsCols * kRmsSlices / 32][128];
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+      if (bz == 0)
+        for (int i = warp; i < ntok; i += kRmsCols * kRmsSlices / 32) append_token<T>(a, t0 + i, lane, rows[warp]);
+      return;
+    }
+  }
+
+  // latent rows [k0, k1) of this slice; W loads are issued before the token tile is staged
+  const int k0 = (int)((int64_t)slice * a.r / kRmsSlices);
+  const int k1 = (int)((int64_t)(slice + 1) * a.r / kRmsSlices);
+  const float* w = a.w_k + (int64_t)g * a.r * width + min(n, width - 1);
+  constexpr int kBatch = 16;
+  float wv[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) wv[u] = (k0 + u < k1) ? w[(int64_t)(k0 + u) * width] : 0.f;
+
+  {   // stage the token tile as fp32, 16 bytes of input per load
+    constexpr int kPer = 16 / (int)sizeof(T);          // elements per 16-byte load
+    const uint4* c4 = reinterpret_cast<const uint4*>(static_cast<const T*>(a.c_new) + (int64_t)t0 * a.r);
+    const int nvec = TT * a.r / kPer;
+    for (int e0 = threadIdx.x; e0 < nvec; e0 += 4 * kRmsCols * kRmsSlices) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * kRmsCols * kRmsSlices;
+        v[u] = (e < nvec && (e * kPer) / a.r < ntok) ? c4[e] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * kRmsCols * kRmsSlices;
+        if (e < nvec) {
+          const T* x = reinterpret_cast<const T*>(&v[u]);
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) cs[e * kPer + q] = to_f32(x[q]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+  for (int kb = k0;; ) {
+    const int nk = min(kBatch, k1 - kb);
+    if (nk == kBatch && (kb & 3) == 0 && (a.r & 3) == 0) {
+      // 16-byte token reads: four FMAs per shared-memory load
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float4* crow = reinterpret_cast<const float4*>(cs + t * a.r + kb);
+#pragma unroll
+        for (int u4 = 0; u4 < kBatch / 4; ++u4) {
+          const float4 cv = crow[u4];
+          acc[t] = fmaf(cv.x, wv[4 * u4 + 0], acc[t]);
+          acc[t] = fmaf(cv.y, wv[4 * u4 + 1], acc[t]);
+          acc[t] = fmaf(cv.z, wv[4 * u4 + 2], acc[t]);
+          acc[t] = fmaf(cv.w, wv[4 * u4 + 3], acc[t]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float* crow = cs + t * a.r + kb;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (u < nk) acc[t] = fmaf(crow[u], wv[u], acc[t]);
+      }
+    }
+    kb += kBatch;
+    if (kb >= k1) break;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) wv[u] = (kb + u < k1) ? w[(int64_t)(kb + u) * width] : 0.f;
+  }
+#pragma unroll
+  for (int t = 0; t < TT; ++t) zp[(slice * TT + t) * kRmsCols + col] = acc[t];
+  __syncthreads();
+  // thread (slice, col) finishes tokens slice, slice + 16, ...: z summed over slices, squared,
+  // then summed over the 16 columns of its half-warp
+  for (int t = slice; t < TT; t += kRmsSlices) {
+    float z = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < kRmsSlices; ++sl) z += zp[(sl * TT + t) * kRmsCols + col];
+    float v = (n < width) ? z * z : 0.f;
+#pragma unroll
+    for (int o = kRmsCols / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (col == 0 && t < ntok) {
+      const int64_t i = (int64_t)a.slot[t0 + t] * a.groups + g;
+      if constexpr (FUSED) {
+        float* acc = reinterpret_cast<float*>(a.ak_scratch + 2 * i);
+        unsigned int* cnt = a.ak_scratch + 2 * i + 1;
+        atomicAdd(acc, v);
+        __threadfence();
+        if (atomicAdd(cnt, 1u) == (unsigned int)(nblk - 1)) {
+          __threadfence();
+          const float total = atomicExch(acc, 0.f);
+          a.a_k[i] = 1.0f / sqrtf(total / (float)width + a.eps);
+          atomicExch(cnt, 0u);
+        }
+      } else {
+        atomicAdd(a.a_k + i, v);
+      }
+    }
+  }
+}
+
+// a_q[i,h] and the rotated RoPE query of one (query row i, head h), by one warp.
+template <typename T>
+__device__ __forceinline__ void absorb_row(const AbsorbArgs& a, int i, int h, float* row, int lane) {
+  const int64_t wid = (int64_t)i * a.heads + h;
+  const T* q = static_cast<const T*>(a.q) + wid * a.d_h;
+  float ss = 0.f;
+  for (int d = lane; d < a.d_h; d += 32) {
+    const float v = to_f32(q[d]);
+    ss += v * v;
+  }
+  const T* qr = static_cast<const T*>(a.q_rope) + wid * a.d_rope;
+  float sr = 0.f;
+  for (int d = lane; d < a.d_rope; d += 32) {
+    const float v = to_f32(qr[d]);
+    row[d] = v;
+    sr += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    sr += __shfl_xor_sync(0xffffffffu, sr, o);
+  }
+  if (lane == 0) a.a_q[wid] = a.softmax_scale / sqrtf(ss / (float)a.d_h + a.eps);
+  const float inv = a.softmax_scale / sqrtf(sr / (float)a.d_rope + a.eps);
+  __syncwarp();
+  const int half = a.d_rope / 2;
+  const int32_t pos = a.pos[i];
+  T* out = static_cast<T*>(a.q_rope_hat) + wid * a.d_rope;
+  for (int d = lane; d < half; d += 32) {
+    const float x1 = row[d] * inv * a.gamma_qr[h * a.d_rope + d];
+    const float x2 = row[d + half] * inv * a.gamma_qr[h * a.d_rope + d + half];
+    float sn, cs;
+    rope_sincos(pos, a.freq.f[d], sn, cs);
+    out[d] = from_f32<T>(x1 * cs - x2 * sn);
+    out[d + half] = from_f32<T>(x2 * cs + x1 * sn);
+  }
+  __syncwarp();
+}
+
+constexpr int kAbsK = 64;        // latent rows of W^K_{g,h} per CTA (two per lane)
+constexpr int kAbsQ = 32;        // query rows per pass
+
+// CTA (h, y < last) of the absorption grid (H, ceil(r / kAbsK) + 1), NW warps:
+// stages its kAbsK x d_h slice of W^K_{g,h} once, with gamma_q * gamma_k folded
+// into its columns, and computes q~[i, h, k] for its latent rows k and every
+// query row i: lane l holds rows l and l + 32, warp w the query rows w, w + NW,
+// ... of a pass, so a warp's W reads hit 32 banks and its query reads are
+// broadcasts.  The slice, the gamma product and the first pass's queries are
+// loaded in one round.  The CTA with y == last produces a_q and the RoPE query
+// of head h.
+template <typename T, int NW>
+__device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by, float* smem) {
+  constexpr int kThreadsAbs = NW * 32;
+  constexpr int kJ = kAbsQ / NW;                           // query rows per warp per pass
+  // row pitch d_h + 4: 16-byte aligned rows, and the eight lanes of a quarter-warp read distinct banks
+  const int pitch = a.d_h + 4;
+  float* wc = smem;                                        // [kAbsK][d_h + 4]
+  float* sv = wc + kAbsK * pitch;                          // [kAbsQ][d_h]
+  float* g2 = sv + kAbsQ * a.d_h;                          // [d_h] gamma_q * gamma_k of head h
+  const int h = bx;
+  const int nkb = (a.r + kAbsK - 1) / kAbsK;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (by == nkb) {
+    __shared__ float rowbuf[NW][128];
+    for (int i = warp; i < a.n_q; i += NW) absorb_row<T>(a, i, h, rowbuf[warp], lane);
+    return;
+  }
+  const int kbase = by * kAbsK;
+  const int ng = a.heads / a.groups;
+  const int g = h / ng, m = h - g * ng;
+  const int width = ng * a.d_h;
+  const float* w = a.w_k + (int64_t)g * a.r * width + (int64_t)m * a.d_h;
+  const int dq = a.d_h / 4;
+  const T* q = static_cast<const T*>(a.q);
+  T* out = static_cast<T*>(a.q_tilde);
+  constexpr int kB = 4;                                    // 16-byte loads per thread per batch
+  // stage query rows [i0, i0 + nq) of head h as fp32, batch by batch (loads, then stores)
+  auto stage_q = [&](int i0, int nq) {
+    for (int e0 = threadIdx.x; e0 < kAbsQ * dq; e0 += kB * kThreadsAbs) {
+      float4 v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int e = e0 + u * kThreadsAbs;
+        const int qi = e / dq, d4 = e - qi * dq;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < kAbsQ * dq && qi < nq) {
+          const T* src = q + ((int64_t)(i0 + qi) * a.heads + h) * a.d_h + d4 * 4;
+          v[u] = make_float4(to_f32(src[0]), to_f32(src[1]), to_f32(src[2]), to_f32(src[3]));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int e = e0 + u * kThreadsAbs;
+        if (e < kAbsQ * dq) reinterpret_cast<float4*>(sv)[e] = v[u];
+      }
+    }
+  };
+  // the slice times the gamma product, batch by batch; the first batch's loads go out with the
+  // gamma and first-pass query loads
+  auto load_w = [&](int e0, float4 (&v)[kB]) {
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int e = e0 + u * kThreadsAbs;
+      const int rr = e / dq, d4 = e - rr * dq;
+      v[u] = (e < kAbsK * dq && kbase + rr < a.r)
+                 ? *reinterpret_cast<const float4*>(w + (int64_t)(kbase + rr) * width + d4 * 4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store_w = [&](int e0, const float4 (&v)[kB]) {
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int e = e0 + u * kThreadsAbs;
+      if (e < kAbsK * dq) {
+        const int rr = e / dq, d4 = e - rr * dq;
+        const float4 gg = reinterpret_cast<const float4*>(g2)[d4];
+        *reinterpret_cast<float4*>(wc + rr * pitch + d4 * 4) =
+            make_float4(v[u].x * gg.x, v[u].y * gg.y, v[u].z * gg.z, v[u].w * gg.w);
+      }
+    }
+  };
+  {
+    float4 wv[kB];
+    load_w(threadIdx.x, wv);
+    float4 gq = make_float4(0.f, 0.f, 0.f, 0.f), gk = gq;
+    if ((int)threadIdx.x < dq) {
+      gq = *reinterpret_cast<const float4*>(a.gamma_q + h * a.d_h + threadIdx.x * 4);
+      gk = *reinterpret_cast<const float4*>(a.gamma_k + h * a.d_h + threadIdx.x * 4);
+    }
+    stage_q(0, min(kAbsQ, a.n_q));
+    if ((int)threadIdx.x < dq)
+      reinterpret_cast<float4*>(g2)[threadIdx.x] = make_float4(gq.x * gk.x, gq.y * gk.y, gq.z * gk.z, gq.w * gk.w);
+    __syncthreads();
+    store_w(threadIdx.x, wv);
+    for (int e0 = threadIdx.x + kB * kThreadsAbs; e0 < kAbsK * dq; e0 += kB * kThreadsAbs) {
+      load_w(e0, wv);
+      store_w(e0, wv);
+    }
+  }
+  const float* wrow0 = wc + lane * pitch;
+  const float* wrow1 = wc + (lane + 32) * pitch;
+  for (int i0 = 0; i0 < a.n_q; i0 += kAbsQ) {
+    const int nq = min(kAbsQ, a.n_q - i0);
+    if (i0 > 0) {
+      __syncthreads();                                     // the previous pass is done with sv
+      stage_q(i0, nq);
+    }
+    __syncthreads();
+    float acc0[kJ], acc1[kJ];
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) acc0[j] = acc1[j] = 0.f;
+    // query rows warp, warp + NW, ... of the pass that exist (warp-uniform)
+    const int nj = (nq - warp + NW - 1) / NW;
+    for (int d = 0; d < a.d_h; d += 4) {
+      const float4 w0 = *reinterpret_cast<const float4*>(wrow0 + d);
+      const float4 w1 = *reinterpret_cast<const float4*>(wrow1 + d);
+#pragma unroll
+      for (int j = 0; j < kJ; ++j) {
+        if (j < nj) {
+          const float4 sq = *reinterpret_cast<const float4*>(sv + (warp + NW * j) * a.d_h + d);
+          acc0[j] = fmaf(w0.x, sq.x, fmaf(w0.y, sq.y, fmaf(w0.z, sq.z, fmaf(w0.w, sq.w, acc0[j]))));
+          acc1[j] = fmaf(w1.x, sq.x, fmaf(w1.y, sq.y, fmaf(w1.z, sq.z, fmaf(w1.w, sq.w, acc1[j]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+      const int qi = warp + NW * j;
+      if (qi < nq) {
+        T* o = out + ((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase;
+        if (kbase + lane < a.r) o[lane] = from_f32<T>(acc0[j]);
+        if (kbase + lane + 32 < a.r) o[lane + 32] = from_f32<T>(acc1[j]);
+      }
+    }
+  }
+}
+
+}  // namespace qkn

@@ -12,8 +12,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, decode, decode_workspace_size,
-               read_device_status, workspace_init)
+from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, append_absorb, decode,
+               decode_workspace_size, read_device_status, workspace_init)
 
 
 def to_device(x, dtype: torch.dtype, device) -> torch.Tensor:
@@ -61,6 +61,16 @@ class DecodeSession:
         self.ensure_query_buffers(q.shape[0])
         absorb_query(d, q, q_rope, to_device(pos, torch.int32, dev), self.w_k, self.gamma_q, self.gamma_k,
                      self.gamma_qr, self.q_tilde, self.a_q, self.q_rope_hat)
+
+    def prepare(self, c, k_rope_raw, slot, pos, q, q_rope, qpos) -> None:
+        """A decode step's append and query absorption, in one launch where possible."""
+        d, dt, dev = self.dims, self.dims.torch_dtype, self.device
+        q = to_device(q, dt, dev)
+        self.ensure_query_buffers(q.shape[0])
+        append_absorb(d, self.cache, to_device(c, dt, dev), to_device(k_rope_raw, dt, dev),
+                      to_device(slot, torch.int32, dev), to_device(pos, torch.int32, dev), q,
+                      to_device(q_rope, dt, dev), to_device(qpos, torch.int32, dev), self.w_k, self.gamma_q,
+                      self.gamma_k, self.gamma_qr, self.gamma_kr, self.q_tilde, self.a_q, self.q_rope_hat)
 
     def ensure_query_buffers(self, n_q: int) -> None:
         """Device buffers for q~, a_q and q^R^ of n_q query rows (kept while n_q stays the same)."""

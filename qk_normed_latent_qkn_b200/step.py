@@ -5,9 +5,9 @@ tokens and queries in, append the tokens to the cache, absorb the queries,
 decode, copy the result out.  ``DecodeStep`` captures that sequence once over
 fixed buffers (pinned host buffers for the inputs and outputs, device buffers
 for everything else) and replays it, so a step costs one graph launch instead
-of a dozen API calls and copies.  Append and query absorption are independent
-and run on two streams inside the graph; the split-KV decode and its merge
-follow both.  All arithmetic runs in libqkn.
+of a dozen API calls and copies.  Append and query absorption run as one
+launch (qkn_append_absorb); the split-KV decode and its merge follow on the
+same stream.  All arithmetic runs in libqkn.
 
 Usage::
 
@@ -19,7 +19,7 @@ from __future__ import annotations
 
 import torch
 
-from . import AK_CACHE, KERNEL_AUTO, absorb_query, append, decode
+from . import AK_CACHE, KERNEL_AUTO, append_absorb, decode
 
 
 class DecodeStep:
@@ -56,7 +56,6 @@ class DecodeStep:
         self.host_out = (hv["out"], hv["lse"])
         session.ensure_query_buffers(n_q)
         self.workspace = session.ensure_workspace(batch, s_q)
-        self.side = torch.cuda.Stream(device=dev)
         self.graph = None
         self.h2d_bytes = in_bytes
         self.d2h_bytes = out_bytes
@@ -81,14 +80,9 @@ class DecodeStep:
 
     def _body(self) -> None:
         s, d, di = self.session, self.session.dims, self.dev_in
-        main = torch.cuda.current_stream(s.device)
         self._dev_in_buf.copy_(self._host_in_buf, non_blocking=True)
-        self.side.wait_stream(main)
-        with torch.cuda.stream(self.side):
-            absorb_query(d, di["q"], di["q_rope"], di["qpos"], s.w_k, s.gamma_q, s.gamma_k, s.gamma_qr,
-                         s.q_tilde, s.a_q, s.q_rope_hat)
-        append(d, s.cache, di["c"], di["k_rope"], di["slot"], di["pos"], s.w_k, s.gamma_kr)
-        main.wait_stream(self.side)
+        append_absorb(d, s.cache, di["c"], di["k_rope"], di["slot"], di["pos"], di["q"], di["q_rope"], di["qpos"],
+                      s.w_k, s.gamma_q, s.gamma_k, s.gamma_qr, s.gamma_kr, s.q_tilde, s.a_q, s.q_rope_hat)
         decode(d, s.cache, s.q_tilde, s.a_q, s.q_rope_hat, di["block_table"], di["seq_lens"], self.s_q,
                self.workspace, self.out, self.lse, ak_mode=self.ak_mode, kernel=self.kernel)
         self._host_out_buf.copy_(self._dev_out_buf, non_blocking=True)
