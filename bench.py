@@ -324,7 +324,8 @@ def run_ours(args, world, rank, local):
         if start_event is not None:
             evs.wait_stream(main)
             ev.record(start_event, evs.cuda_stream)
-        s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event)
+        s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event,
+                 step_writes_only=True)
         if end_event is not None:
             ev.record(end_event, main.cuda_stream)
         if start_event is not None:

@@ -122,6 +122,16 @@ typedef struct {
   int64_t wait_limit;      /* bounded-wait limit in clock cycles for the mbarrier waits; 0 = default (~2 s) */
   void* split_event;       /* optional cudaEvent_t recorded between the split-KV kernel and the combine
                               kernel (external record, so it also works inside stream capture) */
+  int32_t step_writes_only;/* 1: the caller guarantees that the work enqueued on `stream` since the
+                              previous decode of these sequences wrote, of everything the decode reads,
+                              only the queries (q_tilde, a_q, q_rope_hat) and the cache slots of each
+                              sequence's last s_q tokens, and that it is complete or is one launch of
+                              qkn_append_absorb or qkn_append made just before the decode (as in a
+                              decode step; those kernels let the decode launch only once everything
+                              enqueued before them is complete).  The tcgen05 decode then reads the lengths and the block
+                              table and streams the other cache pages while that kernel is still
+                              running, and waits for it only before the queries and the pages that hold
+                              new tokens.  0 (default): it waits before reading anything. */
 } qkn_decode_opts;
 
 /* qkn_append — write n_tok new tokens into the cache.

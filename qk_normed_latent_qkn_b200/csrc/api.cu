@@ -332,6 +332,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   a.out = out;
   a.lse = lse;
   a.seg_desc = reinterpret_cast<int2*>(ws + w.desc_off);
+  a.step_writes_only = (opts && opts->step_writes_only) ? 1 : 0;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const bool bf16 = dims->dtype == QKN_BF16;

@@ -36,8 +36,9 @@ __global__ void __launch_bounds__(256) append_copy_kernel(const __grid_constant_
 template <typename T, int TT, bool FUSED>
 __global__ void __launch_bounds__(kRmsCols * kRmsSlices, 2) append_keyrms_kernel(AppendArgs a) {
   extern __shared__ float4 smem4[];
-  pdl_trigger();
+  // dependents may launch only once everything before this kernel is complete (see prep.cu)
   pdl_wait();
+  pdl_trigger();
   keyrms_block<T, TT, FUSED>(a, blockIdx.x, blockIdx.y, blockIdx.z, reinterpret_cast<float*>(smem4));
 }
 

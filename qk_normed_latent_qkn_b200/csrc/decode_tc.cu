@@ -66,6 +66,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;        // rescale O only when a column max grows by > 2^8
 constexpr int64_t kDrainLimit = 4000000000LL;
+constexpr int kEarlyPages = 2;            // pages the producer may issue before the query tile (ring holds >= 2)
 
 template <int R>
 struct Cfg {
@@ -237,9 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     tmem_alloc(smem_u32(&ms.tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
-  // everything above touches only this CTA's own memory; inputs are read after the wait
+  // everything above touches only this CTA's own memory.  By default every input is read after the
+  // wait for the preceding kernel; with step_writes_only the lengths, the block table and the cache
+  // pages without new tokens are not written by it, so the schedule and the producer start at once
+  // and only the query tile, the pages with new tokens and the softmax (a_q) wait.
   pdl_trigger();
-  pdl_wait();
+  if (!a.step_writes_only) pdl_wait();
   if (warp == 0) {
     Cursor c = sched_begin(sp, blockIdx.x);
     if (lane == 0) ms.cursor = c;
@@ -259,20 +263,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     int n_item = 0;
     bool ok = true;
     const uint32_t akpage = (uint32_t)kPage * (uint32_t)G * 4u;
+    bool waited = !a.step_writes_only;
+    int early_pages = 0;                  // pages issued before the first query tile
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
       const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
       // the first 32 block-table entries of the item are read before the query tile is issued, so
       // that the two memory latencies overlap
       int32_t mine = (it.p0 + lane < it.p1) ? row[it.p0 + lane] : 0;
-      if (!mbar_wait_warp(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
-      {
+      // The query tile is issued at once unless the first pages may stream before the wait: then it
+      // goes out before the first page with new tokens or once the ring holds kEarlyPages pages
+      // (the score MMAs, which free the ring, need it).
+      bool q_pending = true;
+      auto issue_q = [&]() -> bool {
+        if (!waited) {
+          pdl_wait();
+          waited = true;
+        }
+        if (!mbar_wait_warp(smem_u32(&ms.q_empty), (n_item & 1) ^ 1, a.wait_limit)) return false;
         const int qrow0 = it.b * qrows + it.ht * R;
         const uint32_t qf = smem_u32(&ms.q_full);
         mbar_arrive_expect_tx_elect(qf, R * 1024 + R * 128);
 #pragma unroll
         for (int k = 0; k < kChunks; ++k) tma_load_2d_elect(sb + C::Q_OFF + k * R * 128, &maps.qt, k * 64, qrow0, qf);
         tma_load_2d_elect(sb + C::QR_OFF, &maps.qr, 0, qrow0, qf);
-      }
+        q_pending = false;
+        return true;
+      };
+      if (waited && !issue_q()) { ok = false; break; }
+      const int first_new_page = (it.L - a.s_q) / kPage;   // pages from here on hold this step's tokens
       for (int pb = it.p0; pb < it.p1 && ok; pb += 32) {
         // 32 block-table entries per warp-wide load
         if (pb > it.p0) mine = (pb + lane < it.p1) ? row[pb + lane] : 0;
@@ -283,6 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const int cnt = min(32, it.p1 - pb);
         for (int k = 0; k < cnt && ok; ++k) {
           const int32_t blk = __shfl_sync(0xffffffffu, mine, k);
+          if (q_pending && (pb + k >= first_new_page || early_pages >= kEarlyPages)) {
+            if (!issue_q()) { ok = false; break; }
+          }
+          if (q_pending) ++early_pages;
           for (int m = 0; m < kSlotsPerTile; ++m) {
             if (!mbar_wait_warp(smem_u32(&ms.empty[cw.slot]), cw.phase ^ 1u, a.wait_limit)) { ok = false; break; }
             const uint32_t fb = smem_u32(&ms.full[cw.slot]);
@@ -303,8 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           ++k_issued;
         }
       }
+      if (ok && q_pending && !issue_q()) ok = false;
       ++n_item;
     }
+    if (!waited) pdl_wait();
     if (!ok && lane == 0) {
       record_status(a.status, QKN_ERR_TIMEOUT);
       ms.abort_flag = 1;
@@ -454,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         for (int j = 0; j < NJ; ++j) ms.red[warp][par * NJ + j] = v[j];
       }
     };
+    if (a.step_writes_only) pdl_wait();                // a_q is written by the preceding kernel
     const int ng = a.heads / G;
     RingPos<NKR> kr;
     int c_first = 0;          // ring slot of the tile's first latent block

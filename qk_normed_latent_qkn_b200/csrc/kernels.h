@@ -72,6 +72,7 @@ struct DecodeArgs {
   void* out;                 // [batch, s_q, H, r] bf16
   float* lse;                // [batch, s_q, H]
   int2* seg_desc;            // [batch * ht_count]
+  int32_t step_writes_only;  // qkn_decode_opts.step_writes_only: read inputs and old pages before the wait
 };
 
 struct CombineArgs {

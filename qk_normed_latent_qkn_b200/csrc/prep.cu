@@ -26,8 +26,10 @@ template <typename T>
 __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(const __grid_constant__ PrepArgs p) {
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
-  pdl_trigger();
+  // dependents may launch only once everything before this kernel is complete: a decode that
+  // streams old cache pages before its own wait (step_writes_only) relies on it
   pdl_wait();
+  pdl_trigger();
   int bid = blockIdx.x;
   if (bid < p.append_ctas) {
     const int x = bid % p.append_x;
