@@ -23,16 +23,20 @@
 // and are double buffered, so that the scores of page i+1 are computed while
 // the softmax and the output product of page i run.
 //
-// Warp roles (224 threads, one CTA per SM):
-//   warps 0-3  softmax + epilogue: lane i < 16 of warp w owns token 16w + i
-//              of a page (its TMEM lane); thread t owns latent row t of each
-//              O^T block; column (query row) maxima and sums are reduced
-//              across the 128 threads;
-//   warp 4     TMA producer: query tiles per item, then per page four 16 KB
+// Warp roles (352 threads, one CTA per SM):
+//   warps 0-7  softmax + epilogue, two groups of four warps that split the
+//              query rows of the tile: group h takes columns [hR/2, (h+1)R/2)
+//              of S^T and O^T.  Within a group, warp w (mod 4) reads TMEM lanes
+//              32w..32w+31, so lane i < 16 of it owns token 16w + i of a page
+//              and thread t owns latent row t of each O^T block; column maxima
+//              and sums are reduced across the group's 128 threads.  A column
+//              never leaves its group, so the groups synchronise only through
+//              the tile barriers;
+//   warp 8     TMA producer: query tiles per item, then per page four 16 KB
 //              latent slots, the RoPE-key chunk and the a_k rows; the whole
 //              warp reads the block table 32 entries at a time;
-//   warp 5     TMEM allocator and issuer of the score MMAs (S^T, S_R^T);
-//   warp 6     issuer of the output MMAs (O^T).
+//   warp 9     TMEM allocator and issuer of the score MMAs (S^T, S_R^T);
+//   warp 10    issuer of the output MMAs (O^T).
 // A single thread issues tcgen05.mma at a bounded rate, so the two products
 // have one issuing thread each, and every shared-memory descriptor is built
 // once: a K step or a ring slot only moves its start-address field.
@@ -60,8 +64,13 @@ constexpr int kSlotsPerTile = kChunks / 2;
 constexpr int kKrBytes = kPage * kDrope * 2;            // RoPE keys of one page: 8 KB
 constexpr int kMaxGroups = 8;
 constexpr int kAkSlotBytes = kPage * kMaxGroups * 4;    // a_k rows of one page: up to 2 KB
-constexpr int kThreads = 224;
-constexpr int kSoftThreads = 128;
+constexpr int kSoftWarps = 8;               // two groups of four
+constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr int kGroupThreads = 128;
+constexpr int kProducerWarp = kSoftWarps;   // then the two MMA issuers
+constexpr int kScoreWarp = kSoftWarps + 1;
+constexpr int kOutWarp = kSoftWarps + 2;
+constexpr int kThreads = (kSoftWarps + 3) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;        // rescale O only when a column max grows by > 2^8
@@ -109,7 +118,7 @@ struct Misc {
   alignas(16) float mu[R];       // running max (log2 units) used for the exponentials
   alignas(16) float corr[R];     // rescale factor of the current tile
   alignas(16) float linv[R];
-  alignas(16) float red[4][R];   // per-warp partial column reductions
+  alignas(16) float red[4][R];   // partial column reductions of the four warps of each group
 };
 
 }  // namespace
@@ -163,28 +172,29 @@ __device__ __forceinline__ void store_reduced(float* red_w, const float (&v)[R],
   }
 }
 
-__device__ __forceinline__ bool group_all(bool ok) {
+// Votes over the 128 threads that share named barrier `bar` (one barrier per softmax group).
+__device__ __forceinline__ bool group_all(bool ok, uint32_t bar) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)ok)
+      : "r"((uint32_t)ok), "r"(bar)
       : "memory");
   return r != 0;
 }
 
-__device__ __forceinline__ bool group_any(bool v) {
+__device__ __forceinline__ bool group_any(bool v, uint32_t bar) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "r"(bar)
       : "memory");
   return r != 0;
 }
@@ -228,13 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     ms.abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&maps.latent);
     prefetch_tmap(&maps.krope);
     prefetch_tmap(&maps.qt);
     prefetch_tmap(&maps.qr);
   }
-  if (warp == 5) {
+  if (warp == kScoreWarp) {
     tmem_alloc(smem_u32(&ms.tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -255,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
   Cursor cur = ms.cursor;
   Item it;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer (whole warp, elected issue)
     RingPos<NS> cw;
     RingPos<NKR> kw;
@@ -340,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       for (int64_t i = kfirst; i < k_issued; ++i)
         mbar_wait(smem_u32(&ms.krfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
     }
-  } else if (warp == 5) {
+  } else if (warp == kScoreWarp) {
     // ------------------------------------------------------------ score MMA issuer (whole warp)
     constexpr uint32_t idS = idesc_bf16(kPage, R, false, false);
     const uint64_t dC = smem_desc(sb + C::C_OFF, 16, 1024);
@@ -397,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     // every MMA issued so far must finish before the tensor memory is freed
     mma_commit_elect(smem_u32(&ms.drain));
     mbar_wait_warp(smem_u32(&ms.drain), 0, kDrainLimit);
-  } else if (warp == 6) {
+  } else if (warp == kOutWarp) {
     // ------------------------------------------------------------ output MMA issuer (whole warp)
     constexpr uint32_t idPV = idesc_bf16(128, R, true, true);
     // P^T is stored token-major (MN-major B): rows of 2R bytes, swizzled with the matching width
@@ -444,26 +454,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     mbar_wait_warp(smem_u32(&ms.drain), 0, kDrainLimit);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // Thread t of the 128: in the 64-row score layout it holds token `tok` of the page (TMEM lane
-    // tok % 16 of warp tok / 16) and the columns of parity `par`: column 2j + par in its slot j.
-    // In the 128-row O^T layout it holds latent row t of each block.
-    const int t = threadIdx.x;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int tok = warp * 16 + (lane >> 2) + 8 * (lane & 1);
+    // Group hg (warps 4hg .. 4hg + 3) owns the NH = R / 2 columns [hg NH, (hg + 1) NH) of the tile.
+    // Thread t of the group's 128: in the 64-row score layout it holds token `tok` of the page (TMEM
+    // lane tok % 16 of warp tok / 16 of the group) and the group's columns of parity `par`: local
+    // column 2j + par in its slot j.  In the 128-row O^T layout it holds latent row t of each block.
+    const int hg = warp >> 2;
+    const int wq = warp & 3;
+    const int t = threadIdx.x & (kGroupThreads - 1);
+    const uint32_t gbar = 1u + (uint32_t)hg;           // the group's named barrier
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    const int tok = wq * 16 + (lane >> 2) + 8 * (lane & 1);
     const int par = (lane >> 1) & 1;
-    constexpr int NJ = R / 2;                          // columns per thread
-    // per-column values are stored parity-major: column c at pm(c)
+    constexpr int NH = R / 2;                          // columns per group
+    constexpr int NJ = R / 4;                          // columns per thread
+    const int cb = hg * NH;                            // the group's first column
+    // per-column values are stored group by group, parity-major inside a group: local column c of
+    // group hg at cb + pm(c)
     auto pm = [](int c) { return (c & 1) * NJ + (c >> 1); };
-    const float* aq_p = ms.aq2 + par * NJ;
-    const int32_t* ql_p = ms.qlim + par * NJ;
-    const int32_t* grp_p = ms.grp + par * NJ;
-    float* mu_p = ms.mu + par * NJ;
-    const float* corr_p = ms.corr + par * NJ;
+    const float* aq_p = ms.aq2 + cb + par * NJ;
+    const int32_t* ql_p = ms.qlim + cb + par * NJ;
+    const int32_t* grp_p = ms.grp + cb + par * NJ;
+    float* mu_p = ms.mu + cb + par * NJ;
+    const float* corr_p = ms.corr + cb + par * NJ;
+    // O^T columns per TMEM access in the rescale and the epilogue
+    constexpr int kOcols = NH < 16 ? 8 : 16;
+    auto tmem_ld_o = [](uint32_t addr, uint32_t (&v)[kOcols]) {
+      if constexpr (kOcols == 8) tmem_ld8(addr, v); else tmem_ld16(addr, v);
+    };
+    auto tmem_st_o = [](uint32_t addr, const uint32_t (&v)[kOcols]) {
+      if constexpr (kOcols == 8) tmem_st8(addr, v); else tmem_st16(addr, v);
+    };
     auto pv_wait = [&](int64_t n) {
       return mbar_wait(smem_u32(&ms.pv_done[n & 1]), (uint32_t)((n >> 1) & 1), a.wait_limit);
     };
     // maximum (MAX) or sum over the 16 threads of the warp that hold the same columns (lane bits
-    // 0, 2, 3, 4 vary); threads with lane 0 / 2 then store their parity's columns into red[warp]
+    // 0, 2, 3, 4 vary); threads with lane 0 / 2 then store their parity's columns into red[wq]
     auto reduce_store = [&](float (&v)[NJ], bool is_max) {
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
@@ -475,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       }
       if ((lane & ~2) == 0) {
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) ms.red[warp][par * NJ + j] = v[j];
+        for (int j = 0; j < NJ; ++j) ms.red[wq][cb + par * NJ + j] = v[j];
       }
     };
     if (a.step_writes_only) pdl_wait();                // a_q is written by the preceding kernel
@@ -488,21 +513,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     // sequences b = blockIdx.x (mod gridDim.x) with a rejected length are this CTA's to report (checked
     // while the first scores are still being loaded)
     bool rejected = false;
-    for (int b = blockIdx.x + t * gridDim.x; b < a.batch; b += kSoftThreads * gridDim.x)
+    for (int b = blockIdx.x + t * gridDim.x; b < a.batch; b += kGroupThreads * gridDim.x)
       rejected |= pages_of(a.seq_lens[b], sp) == 0;
-    rejected = group_any(rejected);
+    rejected = group_any(rejected, gbar);
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
-      if (t < R) {
-        const int rho = it.ht * R + t;
+      if (t < NH) {
+        const int rho = it.ht * R + cb + t;
         const bool valid = rho < qrows;
         const int j = valid ? rho / a.heads : 0;
         const int h = valid ? rho - j * a.heads : 0;
-        ms.aq2[pm(t)] = valid ? a.a_q[(int64_t)it.b * qrows + rho] * kLog2e : 0.f;
-        ms.grp[pm(t)] = h / ng;
-        ms.qlim[pm(t)] = valid ? it.L - a.s_q + j : -1;
-        ms.mu[pm(t)] = -INFINITY;
+        const int sl = cb + pm(t);
+        ms.aq2[sl] = valid ? a.a_q[(int64_t)it.b * qrows + rho] * kLog2e : 0.f;
+        ms.grp[sl] = h / ng;
+        ms.qlim[sl] = valid ? it.L - a.s_q + j : -1;
+        ms.mu[sl] = -INFINITY;
       }
-      named_bar_sync(1, kSoftThreads);
+      named_bar_sync(gbar, kGroupThreads);
       float lpart[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) lpart[j] = 0.f;
@@ -535,12 +561,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
 #pragma unroll
           for (int b0 = 0; b0 < NJ; b0 += NL) {
             uint32_t sc[NL], sr[NL];
-            if constexpr (NL == 8) {
-              tmem_ld16x64_x8(tSc + 2 * b0, sc);
-              tmem_ld16x64_x8(tSc + R + 2 * b0, sr);
+            if constexpr (NL == 4) {
+              tmem_ld16x64_x4(tSc + cb + 2 * b0, sc);
+              tmem_ld16x64_x4(tSc + R + cb + 2 * b0, sr);
+            } else if constexpr (NL == 8) {
+              tmem_ld16x64_x8(tSc + cb + 2 * b0, sc);
+              tmem_ld16x64_x8(tSc + R + cb + 2 * b0, sr);
             } else {
-              tmem_ld16x64_x16(tSc + 2 * b0, sc);
-              tmem_ld16x64_x16(tSc + R + 2 * b0, sr);
+              tmem_ld16x64_x16(tSc + cb + 2 * b0, sc);
+              tmem_ld16x64_x16(tSc + R + cb + 2 * b0, sr);
             }
             tmem_wait_ld();
             reg_tie(sc);
@@ -571,43 +600,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           over |= (x[j] > m4.x + kRescaleLog2) | (x[j + 1] > m4.y + kRescaleLog2) |
                   (x[j + 2] > m4.z + kRescaleLog2) | (x[j + 3] > m4.w + kRescaleLog2);
         }
-        if (group_any(over || !got)) {
-          if (group_any(!got)) { ok = false; break; }
+        if (group_any(over || !got, gbar)) {
+          if (group_any(!got, gbar)) { ok = false; break; }
           float v[NJ];
 #pragma unroll
           for (int j = 0; j < NJ; ++j) v[j] = x[j];
           reduce_store(v, true);
-          named_bar_sync(1, kSoftThreads);
+          named_bar_sync(gbar, kGroupThreads);
           bool mine = false;
-          if (t < R) {
-            // thread t < R updates column slot t (parity-major order)
-            const float mt = fmaxf(fmaxf(ms.red[0][t], ms.red[1][t]), fmaxf(ms.red[2][t], ms.red[3][t]));
-            const float mo = ms.mu[t];
+          if (t < NH) {
+            // thread t < NH updates the group's column slot cb + t
+            const int sl = cb + t;
+            const float mt = fmaxf(fmaxf(ms.red[0][sl], ms.red[1][sl]), fmaxf(ms.red[2][sl], ms.red[3][sl]));
+            const float mo = ms.mu[sl];
             float cr = 1.f;
             if (mt > mo + kRescaleLog2) {
               cr = (mo == -INFINITY) ? 0.f : ex2(mo - mt);
-              ms.mu[t] = mt;
+              ms.mu[sl] = mt;
               mine = true;
             }
-            ms.corr[t] = cr;
+            ms.corr[sl] = cr;
           }
-          if (group_any(mine) && p > it.p0) {
+          if (group_any(mine, gbar) && p > it.p0) {
             // O^T holds this item's earlier tiles: rescale it once the previous tile's output
             // MMAs are complete
             bool done = true;
             if (t == 0) done = pv_wait(tile_n - 1);
-            if (!group_all(done)) { ok = false; break; }
+            if (!group_all(done, gbar)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
 #pragma unroll
-              for (int c0 = 0; c0 < R; c0 += 16) {
-                uint32_t ov[16];
-                tmem_ld16(tl + m * R + c0, ov);
-                tmem_wait_ld(ov);
+              for (int c0 = 0; c0 < NH; c0 += kOcols) {
+                uint32_t ov[kOcols];
+                tmem_ld_o(tl + m * R + cb + c0, ov);
+                tmem_wait_ld();
+                reg_tie(ov);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[pm(c0 + e)]);
-                tmem_st16(tl + m * R + c0, ov);
+                for (int e = 0; e < kOcols; ++e)
+                  ov[e] = __float_as_uint(__uint_as_float(ov[e]) * ms.corr[cb + pm(c0 + e)]);
+                tmem_st_o(tl + m * R + cb + c0, ov);
                 tmem_wait_st();
               }
             }
@@ -617,8 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         }
         // probabilities, running column sums, and P^T into the RoPE-key slot, token-major: row `tok`
         // holds the token's R probabilities (2R bytes), 16-byte units swizzled by row.  The two threads
-        // of a token swap a quarter of their values (shuffle with lane ^ 2), so that each holds complete
-        // column pairs: parity 0 columns 0 .. R/2 - 1, parity 1 columns R/2 .. R - 1.
+        // of a token in a group swap half of their values (shuffle with lane ^ 2), so that each holds
+        // complete column pairs: parity 0 the group's local columns 0 .. NH/2 - 1, parity 1 the rest.
         {
           float pr[NJ];
 #pragma unroll
@@ -637,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           for (int j = 0; j < NP; ++j) {
             const float send = par == 0 ? pr[j + NP] : pr[j];
             const float got2 = __shfl_xor_sync(0xffffffffu, send, 2);
-            // parity 0: columns (2j, 2j + 1) = (mine, partner's); parity 1: columns
+            // parity 0: local columns (2j, 2j + 1) = (mine, partner's); parity 1: local columns
             // (2(j + NP), 2(j + NP) + 1) = (partner's, mine)
             const __nv_bfloat162 b2 = par == 0 ? __floats2bfloat162_rn(pr[j], got2)
                                                : __floats2bfloat162_rn(got2, pr[j + NP]);
@@ -645,21 +677,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           }
           uint8_t* prow = smem + C::KR_OFF + ks * kKrBytes + tok * (2 * R);
           const int swz = (R == 16) ? ((tok >> 2) & 1) : (R == 32) ? ((tok >> 1) & 3) : (tok & 7);
+          // this thread's NP words start at byte 2 (cb + par NH / 2) of the row
+          const int byte0 = 2 * (cb + par * (NH / 2));
+          if constexpr (NP == 2) {                       // R = 16: half of a 16-byte unit
+            const int unit = byte0 >> 4;
+            *reinterpret_cast<uint2*>(prow + ((unit ^ swz) << 4) + (byte0 & 15)) = make_uint2(words[0], words[1]);
+          } else {
 #pragma unroll
-          for (int u = 0; u < NP / 4; ++u) {
-            const int unit = par * (NP / 4) + u;         // 16-byte unit of the row
-            *reinterpret_cast<uint4*>(prow + ((unit ^ swz) << 4)) =
-                make_uint4(words[4 * u], words[4 * u + 1], words[4 * u + 2], words[4 * u + 3]);
+            for (int u = 0; u < NP / 4; ++u) {
+              const int unit = (byte0 >> 4) + u;         // 16-byte unit of the row
+              *reinterpret_cast<uint4*>(prow + ((unit ^ swz) << 4)) =
+                  make_uint4(words[4 * u], words[4 * u + 1], words[4 * u + 2], words[4 * u + 3]);
+            }
           }
         }
         // the S buffer is free for the tile after next
         tc_fence_before();
         mbar_arrive(smem_u32(&ms.s_empty[sbuf]));
-        // rows of the page past the context: zero them so that 0 * garbage cannot reach O (the two
-        // threads of a token take four of its eight chunks each)
+        // rows of the page past the context: zero them so that 0 * garbage cannot reach O (the four
+        // threads of a token take two of its eight chunks each)
         if (!row_ok) {
 #pragma unroll
-          for (int k = par * 4; k < par * 4 + 4; ++k) {
+          for (int k = (2 * hg + par) * 2; k < (2 * hg + par) * 2 + 2; ++k) {
             const int sl = c_first + k / 2 < NS ? c_first + k / 2 : c_first + k / 2 - NS;
             uint4* rowp = reinterpret_cast<uint4*>(smem + C::C_OFF + sl * kSlotBytes + (k & 1) * kChunkBytes + tok * 128);
 #pragma unroll
@@ -680,34 +719,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         if (tile_n > 1) got = pv_wait(tile_n - 2);
         got = got && pv_wait(tile_n - 1);
       }
-      if (!group_all(got)) { ok = false; break; }
+      if (!group_all(got, gbar)) { ok = false; break; }
       tc_fence_after();
       reduce_store(lpart, false);
-      named_bar_sync(1, kSoftThreads);
-      if (t < R) {
-        const int c = pm(t);
-        const float l = ms.red[0][c] + ms.red[1][c] + ms.red[2][c] + ms.red[3][c];
-        ms.linv[t] = l > 0.f ? 1.f / l : 0.f;
-        a.part_lse[(int64_t)it.slot * R + t] = l > 0.f ? (ms.mu[c] + log2f(l)) * kLn2 : -INFINITY;
+      named_bar_sync(gbar, kGroupThreads);
+      if (t < NH) {
+        const int c = cb + t;                            // the column (query row of the tile)
+        const int sl = cb + pm(t);
+        const float l = ms.red[0][sl] + ms.red[1][sl] + ms.red[2][sl] + ms.red[3][sl];
+        ms.linv[c] = l > 0.f ? 1.f / l : 0.f;
+        a.part_lse[(int64_t)it.slot * R + c] = l > 0.f ? (ms.mu[sl] + log2f(l)) * kLn2 : -INFINITY;
       }
-      named_bar_sync(1, kSoftThreads);
+      named_bar_sync(gbar, kGroupThreads);
       float* po = a.part_o + (int64_t)it.slot * R * kRkv;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
 #pragma unroll
-        for (int c0 = 0; c0 < R; c0 += 16) {
-          uint32_t ov[16];
-          tmem_ld16(tl + m * R + c0, ov);
-          tmem_wait_ld(ov);
+        for (int c0 = cb; c0 < cb + NH; c0 += kOcols) {
+          uint32_t ov[kOcols];
+          tmem_ld_o(tl + m * R + c0, ov);
+          tmem_wait_ld();
+          reg_tie(ov);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
+          for (int e = 0; e < kOcols; ++e)
             po[(int64_t)(c0 + e) * kRkv + m * 128 + t] = __uint_as_float(ov[e]) * ms.linv[c0 + e];
         }
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&ms.o_empty));
       // the CTA holding a segment's first split tells the merge kernel where its splits are
-      if (t == 0 && it.p0 == 0) {
+      if (threadIdx.x == 0 && it.p0 == 0) {
         const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota);
         a.seg_desc[it.b * a.ht_count + it.ht] = make_int2(it.b * a.ht_count + it.ht + sg.c0, sg.nitems);
       }
@@ -719,19 +760,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     }
     // A sequence whose length was rejected (outside [s_q, max_blocks * 64]) has no units: its rows
     // are written as zero with lse = -inf, and the status records QKN_ERR_BOUNDS.
+    const int ts = threadIdx.x;                        // 0 .. kSoftThreads - 1 over both groups
     for (int b = blockIdx.x; rejected && b < a.batch; b += gridDim.x) {
       if (pages_of(a.seq_lens[b], sp) != 0) continue;
-      if (t == 0) record_status(a.status, QKN_ERR_BOUNDS);
-      for (int ht = t; ht < a.ht_count; ht += kSoftThreads) a.seg_desc[b * a.ht_count + ht] = make_int2(0, 0);
+      if (ts == 0) record_status(a.status, QKN_ERR_BOUNDS);
+      for (int ht = ts; ht < a.ht_count; ht += kSoftThreads) a.seg_desc[b * a.ht_count + ht] = make_int2(0, 0);
       uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * qrows * kRkv);
-      for (int64_t e = t; e < (int64_t)qrows * kRkv / 8; e += kSoftThreads) ob[e] = make_uint4(0, 0, 0, 0);
-      for (int e = t; e < qrows; e += kSoftThreads) a.lse[(int64_t)b * qrows + e] = -INFINITY;
+      for (int64_t e = ts; e < (int64_t)qrows * kRkv / 8; e += kSoftThreads) ob[e] = make_uint4(0, 0, 0, 0);
+      for (int e = ts; e < qrows; e += kSoftThreads) a.lse[(int64_t)b * qrows + e] = -INFINITY;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kScoreWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
