@@ -134,6 +134,18 @@ typedef struct {
                               new tokens.  0 (default): it waits before reading anything. */
 } qkn_decode_opts;
 
+/* qkn_key_gram — G_g = W^K_g (W^K_g)^T for every group g, the r_kv x r_kv
+ * matrix with which qkn_append computes the key statistic without forming
+ * the key: sum over the n_g * d_h columns of (c W^K_g)^2 equals c G_g c^T.
+ * The pages define the statistic on the up-projected key (technical summary,
+ * Metodología items 2-4); the Gram form is the same sum, reached through
+ * r_kv x r_kv products instead of r_kv x n_g d_h, and is this library's.
+ * Accumulated in fp64, stored in fp32.  Compute it once per weight set.
+ *   w_k      [num_groups, r_kv, n_g * d_h] fp32
+ *   key_gram [num_groups, r_kv, r_kv] fp32 (out), symmetric
+ * Returns QKN_ERR_INVALID_ARG for bad dims or NULL pointers. */
+QKN_EXPORT qkn_status qkn_key_gram(const qkn_dims* dims, const float* w_k, float* key_gram, void* stream);
+
 /* qkn_append — write n_tok new tokens into the cache.
  * For token i with slot s = slot[i] and position p = pos[i]:
  *   latent[s]  = c_new[i]                                    (copied as is)
@@ -147,12 +159,18 @@ typedef struct {
  *   k_rope_raw [n_tok, d_rope] dtype
  *   slot, pos  [n_tok] int32; every slot in [0, num_blocks * block_size)
  *   w_k        [num_groups, r_kv, n_g * d_h] fp32
+ *   key_gram   [num_groups, r_kv, r_kv] fp32 from qkn_key_gram(w_k), or NULL.
+ *              Given, the statistic is summed as c G_g c^T and w_k is not read
+ *              (it may be NULL); NULL, as sum((c W^K_g)^2) from w_k.  The two
+ *              agree up to fp32 rounding.
  *   gamma_kr   [d_rope] fp32 (shared by all heads)
- * n_tok == 0 is a no-op.  Slots must be distinct within one call. */
+ * n_tok == 0 is a no-op.  Slots must be distinct within one call.  Returns
+ * QKN_ERR_INVALID_ARG when both w_k and key_gram are NULL. */
 QKN_EXPORT qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache,
                       const void* c_new, const void* k_rope_raw,
                       const int32_t* slot, const int32_t* pos, int32_t n_tok,
-                      const float* w_k, const float* gamma_kr, void* stream);
+                      const float* w_k, const float* key_gram, const float* gamma_kr,
+                      void* stream);
 
 /* qkn_absorb_query — fold the static norm weights into the query
  * (technical summary, Metodología item 1 and the decode-logit equation).
@@ -179,7 +197,8 @@ QKN_EXPORT qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, cons
  * Metodología items 1-4): the append writes the cache's new tokens and their
  * key statistic, the absorption folds the norm weights into the step's
  * queries; neither reads what the other writes.  Arguments are those of the
- * two calls (qpos are the query rows' RoPE positions; w_k is shared), with
+ * two calls (qpos are the query rows' RoPE positions; w_k is shared; key_gram
+ * is the append's and may be NULL), with
  * the same layouts, validation and results.  One launch is used when the
  * cache carries ak_scratch, 0 < n_tok <= 256 and n_q > 0; otherwise the two
  * steps run as their own launches, in this order, on `stream`.  It exists so
@@ -189,8 +208,8 @@ QKN_EXPORT qkn_status qkn_append_absorb(const qkn_dims* dims, const qkn_cache* c
                       const void* c_new, const void* k_rope_raw,
                       const int32_t* slot, const int32_t* pos, int32_t n_tok,
                       const void* q, const void* q_rope, const int32_t* qpos, int32_t n_q,
-                      const float* w_k, const float* gamma_q, const float* gamma_k,
-                      const float* gamma_qr, const float* gamma_kr,
+                      const float* w_k, const float* key_gram, const float* gamma_q,
+                      const float* gamma_k, const float* gamma_qr, const float* gamma_kr,
                       void* q_tilde, float* a_q, void* q_rope_hat, void* stream);
 
 /* Bytes of decode workspace needed for `batch` sequences of `s_q` query

@@ -26,7 +26,7 @@ KERNEL_AUTO, KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1, 2
 
 EXPORTED = ["qkn_append", "qkn_absorb_query", "qkn_decode_workspace_size", "qkn_workspace_init",
             "qkn_decode", "qkn_read_device_status", "qkn_decode_kernel_for", "qkn_status_string",
-            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb"]
+            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb", "qkn_key_gram"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -61,7 +61,8 @@ def _load() -> ctypes.CDLL:
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     PD, PC, PO = ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), ctypes.POINTER(_Opts)
     sig = {
-        "qkn_append": (I32, [PD, PC, P, P, P, P, I32, P, P, P]),
+        "qkn_append": (I32, [PD, PC, P, P, P, P, I32, P, P, P, P]),
+        "qkn_key_gram": (I32, [PD, P, P, P]),
         "qkn_absorb_query": (I32, [PD, P, P, P, I32, P, P, P, P, P, P, P, P]),
         "qkn_decode_workspace_size": (I32, [PD, I32, I32, I32, ctypes.POINTER(SZ)]),
         "qkn_workspace_init": (I32, [P, SZ, P]),
@@ -71,7 +72,7 @@ def _load() -> ctypes.CDLL:
         "qkn_status_string": (ctypes.c_char_p, [I32]),
         "qkn_version": (I32, []),
         "qkn_decode_noalloc": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, P, P, PO, P]),
-        "qkn_append_absorb": (I32, [PD, PC, P, P, P, P, I32, P, P, P, I32, P, P, P, P, P, P, P, P, P]),
+        "qkn_append_absorb": (I32, [PD, PC, P, P, P, P, I32, P, P, P, I32, P, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -152,11 +153,17 @@ def _opts(kernel=KERNEL_AUTO, max_ctas=0, head_tile=0, wait_limit=0, split_event
 
 
 # ----------------------------------------------------------------- calls
-def append(dims: Dims, cache: Cache, c_new, k_rope_raw, slot, pos, w_k, gamma_kr, stream=None) -> None:
-    """Write tokens into the cache and compute their a_k (see qkn_append)."""
+def key_gram(dims: Dims, w_k, out, stream=None) -> None:
+    """out[g] = W^K_g (W^K_g)^T, fp32 [num_groups, r_kv, r_kv] (see qkn_key_gram)."""
+    _check(_lib.qkn_key_gram(ctypes.byref(dims.c()), _ptr(w_k), _ptr(out), _stream(stream)), "qkn_key_gram")
+
+
+def append(dims: Dims, cache: Cache, c_new, k_rope_raw, slot, pos, w_k, key_gram, gamma_kr, stream=None) -> None:
+    """Write tokens into the cache and compute their a_k (see qkn_append); key_gram may be None."""
     n_tok = int(c_new.shape[0]) if c_new is not None else 0
     _check(_lib.qkn_append(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(c_new), _ptr(k_rope_raw),
-                           _ptr(slot), _ptr(pos), n_tok, _ptr(w_k), _ptr(gamma_kr), _stream(stream)),
+                           _ptr(slot), _ptr(pos), n_tok, _ptr(w_k), _ptr(key_gram), _ptr(gamma_kr),
+                           _stream(stream)),
            "qkn_append")
 
 
@@ -169,12 +176,13 @@ def absorb_query(dims: Dims, q, q_rope, pos, w_k, gamma_q, gamma_k, gamma_qr, q_
                                  _ptr(q_rope_hat), _stream(stream)), "qkn_absorb_query")
 
 
-def append_absorb(dims: Dims, cache: Cache, c_new, k_rope_raw, slot, pos, q, q_rope, qpos, w_k, gamma_q, gamma_k,
-                  gamma_qr, gamma_kr, q_tilde, a_q, q_rope_hat, stream=None) -> None:
+def append_absorb(dims: Dims, cache: Cache, c_new, k_rope_raw, slot, pos, q, q_rope, qpos, w_k, key_gram, gamma_q,
+                  gamma_k, gamma_qr, gamma_kr, q_tilde, a_q, q_rope_hat, stream=None) -> None:
     """qkn_append followed by qkn_absorb_query, in one launch where possible (see qkn_append_absorb)."""
     _check(_lib.qkn_append_absorb(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(c_new), _ptr(k_rope_raw),
                                   _ptr(slot), _ptr(pos), int(c_new.shape[0]), _ptr(q), _ptr(q_rope), _ptr(qpos),
-                                  int(q.shape[0]), _ptr(w_k), _ptr(gamma_q), _ptr(gamma_k), _ptr(gamma_qr),
+                                  int(q.shape[0]), _ptr(w_k), _ptr(key_gram), _ptr(gamma_q), _ptr(gamma_k),
+                                  _ptr(gamma_qr),
                                   _ptr(gamma_kr), _ptr(q_tilde), _ptr(a_q), _ptr(q_rope_hat), _stream(stream)),
            "qkn_append_absorb")
 

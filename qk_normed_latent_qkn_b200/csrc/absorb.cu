@@ -10,7 +10,7 @@
 
 namespace qkn {
 
-// grid (H, ceil(r / kAbsK) + 1); block 256 (see absorb_block).
+// grid (H, ceil(r / 64) + 1); block 256 (see absorb_block).
 template <typename T>
 __global__ void __launch_bounds__(256) absorb_qtilde_kernel(const __grid_constant__ AbsorbArgs a) {
   extern __shared__ float4 smem4[];
@@ -21,14 +21,14 @@ __global__ void __launch_bounds__(256) absorb_qtilde_kernel(const __grid_constan
 
 template <typename T>
 static cudaError_t launch_absorb_t(const AbsorbArgs& a, cudaStream_t st) {
-  const size_t smem = ((size_t)kAbsK * (a.d_h + 4) + (size_t)kAbsQ * a.d_h + (size_t)a.d_h) * sizeof(float);
+  const size_t smem = absorb_smem_bytes(absorb_rows<8>(), a.d_h);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = set_smem_attrs(absorb_qtilde_kernel<T>, 200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(a.heads, (a.r + kAbsK - 1) / kAbsK + 1);
+  dim3 grid(a.heads, (a.r + absorb_rows<8>() - 1) / absorb_rows<8>() + 1);
   return launch_chained(absorb_qtilde_kernel<T>, grid, dim3(256), smem, st, a);
 }
 

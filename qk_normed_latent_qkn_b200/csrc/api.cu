@@ -135,14 +135,15 @@ namespace {
 // Validated launch arguments of an append (n_tok > 0) or QKN_OK with *empty for n_tok == 0.
 qkn_status append_args(const qkn_dims* dims, const qkn_cache* cache, const void* c_new, const void* k_rope_raw,
                        const int32_t* slot, const int32_t* pos, int32_t n_tok, const float* w_k,
-                       const float* gamma_kr, AppendArgs* a, bool* empty) {
+                       const float* key_gram, const float* gamma_kr, AppendArgs* a, bool* empty) {
   qkn_status st = check_dims(dims);
   if (st != QKN_OK) return st;
   if (n_tok < 0) return QKN_ERR_INVALID_ARG;
   *empty = n_tok == 0;
   if (*empty) return QKN_OK;
   if ((st = check_cache(dims, cache)) != QKN_OK) return st;
-  if (!c_new || !k_rope_raw || !slot || !pos || !w_k || !gamma_kr) return QKN_ERR_INVALID_ARG;
+  if (!c_new || !k_rope_raw || !slot || !pos || !(w_k || key_gram) || !gamma_kr) return QKN_ERR_INVALID_ARG;
+  if (!aligned(key_gram, 4)) return QKN_ERR_INVALID_ARG;
   if (!aligned(c_new, 16) || !aligned(k_rope_raw, 16)) return QKN_ERR_INVALID_ARG;
   a->latent = cache->latent;
   a->k_rope = cache->k_rope;
@@ -153,12 +154,14 @@ qkn_status append_args(const qkn_dims* dims, const qkn_cache* cache, const void*
   a->slot = slot;
   a->pos = pos;
   a->w_k = w_k;
+  a->key_gram = key_gram;
   a->gamma_kr = gamma_kr;
   a->n_tok = n_tok;
   a->r = dims->r_kv;
   a->d_rope = dims->d_rope;
   a->groups = dims->num_groups;
   a->width = (dims->num_heads / dims->num_groups) * dims->d_h;
+  a->ncols = key_gram ? dims->r_kv : a->width;
   a->eps = dims->eps;
   a->rope_theta = dims->rope_theta;
   a->freq = rope_freqs(dims);
@@ -205,12 +208,23 @@ qkn_status absorb_args(const qkn_dims* dims, const void* q, const void* q_rope, 
 
 extern "C" {
 
+qkn_status qkn_key_gram(const qkn_dims* dims, const float* w_k, float* key_gram, void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (!w_k || !key_gram) return QKN_ERR_INVALID_ARG;
+  const int width = (dims->num_heads / dims->num_groups) * dims->d_h;
+  cudaError_t e = launch_key_gram(w_k, key_gram, dims->num_groups, dims->r_kv, width,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
 qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache, const void* c_new,
                       const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
-                      const float* w_k, const float* gamma_kr, void* stream) {
+                      const float* w_k, const float* key_gram, const float* gamma_kr, void* stream) {
   AppendArgs a;
   bool empty = false;
-  qkn_status st = append_args(dims, cache, c_new, k_rope_raw, slot, pos, n_tok, w_k, gamma_kr, &a, &empty);
+  qkn_status st = append_args(dims, cache, c_new, k_rope_raw, slot, pos, n_tok, w_k, key_gram, gamma_kr, &a,
+                              &empty);
   if (st != QKN_OK || empty) return st;
   cudaError_t e = launch_append(a, dims->dtype == QKN_BF16, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
@@ -232,12 +246,14 @@ qkn_status qkn_absorb_query(const qkn_dims* dims, const void* q, const void* q_r
 qkn_status qkn_append_absorb(const qkn_dims* dims, const qkn_cache* cache, const void* c_new,
                              const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
                              const void* q, const void* q_rope, const int32_t* qpos, int32_t n_q,
-                             const float* w_k, const float* gamma_q, const float* gamma_k, const float* gamma_qr,
-                             const float* gamma_kr, void* q_tilde, float* a_q, void* q_rope_hat, void* stream) {
+                             const float* w_k, const float* key_gram, const float* gamma_q, const float* gamma_k,
+                             const float* gamma_qr, const float* gamma_kr, void* q_tilde, float* a_q,
+                             void* q_rope_hat, void* stream) {
   AppendArgs ap;
   AbsorbArgs ab;
   bool no_append = false, no_absorb = false;
-  qkn_status st = append_args(dims, cache, c_new, k_rope_raw, slot, pos, n_tok, w_k, gamma_kr, &ap, &no_append);
+  qkn_status st = append_args(dims, cache, c_new, k_rope_raw, slot, pos, n_tok, w_k, key_gram, gamma_kr, &ap,
+                              &no_append);
   if (st != QKN_OK) return st;
   st = absorb_args(dims, q, q_rope, qpos, n_q, w_k, gamma_q, gamma_k, gamma_qr, q_tilde, a_q, q_rope_hat, &ab,
                    &no_absorb);

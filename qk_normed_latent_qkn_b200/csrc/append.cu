@@ -9,9 +9,10 @@
 // three launches on the caller's stream:
 //   1. append_copy:     one warp per token — latent copy, RoPE key
 //                       (RMS-normalise, weight, rotate), a_k slots zeroed;
-//   2. append_keyrms:   z = c W^K_g tiled over (16-column block, token
-//                       tile, group); each CTA adds sum(z^2) of its columns
-//                       into the token's a_k slot;
+//   2. append_keyrms:   z = c W^K_g (or c G_g with the Gram matrix) tiled
+//                       over (16-column block, token tile, group); each CTA
+//                       adds its columns' terms of sum(z^2) into the token's
+//                       a_k slot;
 //   3. append_finalize: a_k = 1 / sqrt(sum / (n_g d_h) + eps).
 // The key z is only ever held in registers; it is never written anywhere.
 #include "prep_blocks.cuh"
@@ -61,7 +62,7 @@ static cudaError_t launch_keyrms(const AppendArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int nblk = (a.width + kRmsCols - 1) / kRmsCols;
+  const int nblk = (a.ncols + kRmsCols - 1) / kRmsCols;
   dim3 grid(nblk + (FUSED ? 1 : 0), (a.n_tok + TT - 1) / TT, a.groups);
   return launch_chained(append_keyrms_kernel<T, TT, FUSED>, grid, dim3(kRmsCols * kRmsSlices), smem, st, a);
 }

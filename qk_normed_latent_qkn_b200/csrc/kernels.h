@@ -25,8 +25,10 @@ struct AppendArgs {
   const int32_t* slot;
   const int32_t* pos;
   const float* w_k;        // [groups, r, width]
+  const float* key_gram;   // [groups, r, r] = W W^T per group, or null (then w_k)
   const float* gamma_kr;   // [d_rope]
   int32_t n_tok, r, d_rope, groups, width;   // width = n_g * d_h
+  int32_t ncols;           // columns of the key-statistic matrix: r with key_gram, else width
   float eps, rope_theta;
   RopeFreqs freq;
 };
@@ -88,6 +90,7 @@ struct CombineArgs {
 };
 
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_key_gram(const float* w_k, float* gram, int groups, int r, int width, cudaStream_t st);
 // One launch for both (prep.cu) when the append can run as one launch and is a decode step's size.
 bool prep_fusable(const AppendArgs& ap, const AbsorbArgs& ab);
 cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, cudaStream_t st);

@@ -51,13 +51,14 @@ cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, c
   PrepArgs p;
   p.ap = ap;
   p.ab = ab;
-  p.append_x = (ap.width + kRmsCols - 1) / kRmsCols + 1;
+  p.append_x = (ap.ncols + kRmsCols - 1) / kRmsCols + 1;
   p.append_y = (ap.n_tok + kPrepTT - 1) / kPrepTT;
   p.append_ctas = p.append_x * p.append_y * ap.groups;
-  p.absorb_y = (ab.r + kAbsK - 1) / kAbsK + 1;
+  constexpr int kAbsRows = absorb_rows<kPrepThreads / 32>();
+  p.absorb_y = (ab.r + kAbsRows - 1) / kAbsRows + 1;
   const int64_t ctas = (int64_t)p.append_ctas + (int64_t)ab.heads * p.absorb_y;
   const size_t smem_append = ((size_t)kPrepTT * ap.r + (size_t)kRmsSlices * kPrepTT * kRmsCols) * sizeof(float);
-  const size_t smem_absorb = ((size_t)kAbsK * (ab.d_h + 4) + (size_t)kAbsQ * ab.d_h + (size_t)ab.d_h) * sizeof(float);
+  const size_t smem_absorb = absorb_smem_bytes(kAbsRows, ab.d_h);
   const size_t smem = smem_append > smem_absorb ? smem_append : smem_absorb;
   auto kernel = bf16 ? prep_kernel<__nv_bfloat16> : prep_kernel<float>;
   static bool attr_set[2] = {false, false};

@@ -72,14 +72,19 @@ __device__ __forceinline__ void append_token(const AppendArgs& a, int i, int lan
   __syncwarp();
 }
 
-// Key statistic sum(z^2), z = c W^K_g.  CTA = (16 key columns, TT tokens,
-// group); its 512 threads are 16 columns x 32 slices of the latent
-// dimension, so a decode step's handful of tokens still spreads over about a
-// hundred CTAs per group.  Every thread loads its slice of one W column in
-// one batch of independent loads and applies it to the TT tokens held in
-// shared memory; slices are summed in shared memory, squared, reduced over
-// the CTA's 16 columns and added into the token's a_k slot (zeroed by
-// append_copy_kernel).
+// Key statistic sum(z^2) over the n_g d_h columns of z = c W^K_g.  Two forms
+// of the same sum:
+//   direct: sum_n z_n^2 with z = c W^K_g             (matrix W, width columns)
+//   Gram:   sum_n (c G)_n c_n with G = W^K_g W^K_g^T  (matrix G, r columns)
+// The Gram form (the identity |cW|^2 = c (W W^T) c^T) reads an r x r matrix
+// instead of r x n_g d_h, a 32-fold cut at r = 512 and n_g d_h = 16384.
+// CTA = (16 matrix columns, TT tokens, group); its 512 threads are 16 columns
+// x 32 slices of the latent dimension, so a decode step's handful of tokens
+// still spreads over several CTAs per group.  Every thread loads its slice of
+// one matrix column in one batch of independent loads and applies it to the
+// TT tokens held in shared memory; slices are summed in shared memory, turned
+// into the column's term (z^2, or (cG)_n c_n), reduced over the CTA's 16
+// columns and added into the token's a_k slot (zeroed by append_copy_kernel).
 constexpr int kRmsCols = 16;
 constexpr int kRmsSlices = 32;
 
@@ -96,10 +101,11 @@ __device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by
   const int g = bz;
   const int t0 = by * TT;
   const int ntok = min(TT, a.n_tok - t0);
-  const int width = a.width;
+  const int ncols = a.ncols;
+  const bool gram = a.key_gram != nullptr;
   const int col = threadIdx.x % kRmsCols, slice = threadIdx.x / kRmsCols;
   const int n = bx * kRmsCols + col;
-  const int nblk = (width + kRmsCols - 1) / kRmsCols;
+  const int nblk = (ncols + kRmsCols - 1) / kRmsCols;
   if constexpr (FUSED) {
     if (bx == nblk) {
       __shared__ float rows[kRmsCols * kRmsSlices / 32][128];
@@ -113,11 +119,11 @@ __device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by
   // latent rows [k0, k1) of this slice; W loads are issued before the token tile is staged
   const int k0 = (int)((int64_t)slice * a.r / kRmsSlices);
   const int k1 = (int)((int64_t)(slice + 1) * a.r / kRmsSlices);
-  const float* w = a.w_k + (int64_t)g * a.r * width + min(n, width - 1);
+  const float* w = (gram ? a.key_gram : a.w_k) + (int64_t)g * a.r * ncols + min(n, ncols - 1);
   constexpr int kBatch = 16;
   float wv[kBatch];
 #pragma unroll
-  for (int u = 0; u < kBatch; ++u) wv[u] = (k0 + u < k1) ? w[(int64_t)(k0 + u) * width] : 0.f;
+  for (int u = 0; u < kBatch; ++u) wv[u] = (k0 + u < k1) ? w[(int64_t)(k0 + u) * ncols] : 0.f;
 
   {   // stage the token tile as fp32, 16 bytes of input per load
     constexpr int kPer = 16 / (int)sizeof(T);          // elements per 16-byte load
@@ -174,18 +180,18 @@ __device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by
     kb += kBatch;
     if (kb >= k1) break;
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) wv[u] = (kb + u < k1) ? w[(int64_t)(kb + u) * width] : 0.f;
+    for (int u = 0; u < kBatch; ++u) wv[u] = (kb + u < k1) ? w[(int64_t)(kb + u) * ncols] : 0.f;
   }
 #pragma unroll
   for (int t = 0; t < TT; ++t) zp[(slice * TT + t) * kRmsCols + col] = acc[t];
   __syncthreads();
-  // thread (slice, col) finishes tokens slice, slice + 16, ...: z summed over slices, squared,
-  // then summed over the 16 columns of its half-warp
+  // thread (slice, col) finishes tokens slice, slice + 32, ...: z summed over slices, turned into
+  // the column's term, then summed over the 16 columns of its half-warp
   for (int t = slice; t < TT; t += kRmsSlices) {
     float z = 0.f;
 #pragma unroll
     for (int sl = 0; sl < kRmsSlices; ++sl) z += zp[(sl * TT + t) * kRmsCols + col];
-    float v = (n < width) ? z * z : 0.f;
+    float v = (n < ncols) ? z * (gram ? cs[t * a.r + n] : z) : 0.f;
 #pragma unroll
     for (int o = kRmsCols / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (col == 0 && t < ntok) {
@@ -198,7 +204,7 @@ __device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by
         if (atomicAdd(cnt, 1u) == (unsigned int)(nblk - 1)) {
           __threadfence();
           const float total = atomicExch(acc, 0.f);
-          a.a_k[i] = 1.0f / sqrtf(total / (float)width + a.eps);
+          a.a_k[i] = 1.0f / sqrtf(total / (float)a.width + a.eps);
           atomicExch(cnt, 0u);
         }
       } else {
@@ -247,35 +253,46 @@ __device__ __forceinline__ void absorb_row(const AbsorbArgs& a, int i, int h, fl
   __syncwarp();
 }
 
-constexpr int kAbsK = 64;        // latent rows of W^K_{g,h} per CTA (two per lane)
 constexpr int kAbsQ = 32;        // query rows per pass
 
-// CTA (h, y < last) of the absorption grid (H, ceil(r / kAbsK) + 1), NW warps:
-// stages its kAbsK x d_h slice of W^K_{g,h} once, with gamma_q * gamma_k folded
-// into its columns, and computes q~[i, h, k] for its latent rows k and every
-// query row i: lane l holds rows l and l + 32, warp w the query rows w, w + NW,
-// ... of a pass, so a warp's W reads hit 32 banks and its query reads are
-// broadcasts.  The slice, the gamma product and the first pass's queries are
-// loaded in one round.  The CTA with y == last produces a_q and the RoPE query
-// of head h.
+// Latent rows of W^K_{g,h} per absorption CTA of NW warps, and its shared memory.
+template <int NW>
+__host__ __device__ constexpr int absorb_rows() { return NW * 8; }
+inline size_t absorb_smem_bytes(int rows, int d_h) {
+  return ((size_t)rows * (d_h + 4) + (size_t)kAbsQ * (d_h + 4) + (size_t)d_h) * sizeof(float);
+}
+
+// CTA (h, y < last) of the absorption grid (H, ceil(r / KB) + 1), NW warps,
+// KB = 8 NW latent rows: stages its KB x d_h slice of W^K_{g,h} once, with
+// gamma_q * gamma_k folded into its columns, and computes q~[i, h, k] for its
+// latent rows k and every query row i, kAbsQ query rows per pass.  Warp w
+// takes 16 rows (w mod NW/2) and 16 query rows (w div NW/2) of a pass; lane
+// (rg, qg) = (lane % 8, lane / 8) takes rows rg, rg + 8 and query rows qg,
+// qg + 4, qg + 8, qg + 12 of those: per 4 columns of d_h it reads 2 W and 4
+// query vectors (16 bytes each) for 32 FMAs, and with row pitch d_h + 4 the
+// 8 distinct rows (and 4 distinct query rows) of one read fall in distinct
+// banks, so every read is one shared-memory wavefront.  The slice, the gamma
+// product and the first pass's queries are loaded in one round.  The CTA with
+// y == last produces a_q and the RoPE query of head h.
 template <typename T, int NW>
 __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by, float* smem) {
   constexpr int kThreadsAbs = NW * 32;
-  constexpr int kJ = kAbsQ / NW;                           // query rows per warp per pass
-  // row pitch d_h + 4: 16-byte aligned rows, and the eight lanes of a quarter-warp read distinct banks
+  constexpr int KB = absorb_rows<NW>();
+  constexpr int kRowWarps = NW / 2;
+  static_assert(kRowWarps * 16 == KB && kAbsQ == 32, "warp tiling of the absorption CTA");
   const int pitch = a.d_h + 4;
-  float* wc = smem;                                        // [kAbsK][d_h + 4]
-  float* sv = wc + kAbsK * pitch;                          // [kAbsQ][d_h]
-  float* g2 = sv + kAbsQ * a.d_h;                          // [d_h] gamma_q * gamma_k of head h
+  float* wc = smem;                                        // [KB][d_h + 4]
+  float* sv = wc + KB * pitch;                             // [kAbsQ][d_h + 4]
+  float* g2 = sv + kAbsQ * pitch;                          // [d_h] gamma_q * gamma_k of head h
   const int h = bx;
-  const int nkb = (a.r + kAbsK - 1) / kAbsK;
+  const int nkb = (a.r + KB - 1) / KB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (by == nkb) {
     __shared__ float rowbuf[NW][128];
     for (int i = warp; i < a.n_q; i += NW) absorb_row<T>(a, i, h, rowbuf[warp], lane);
     return;
   }
-  const int kbase = by * kAbsK;
+  const int kbase = by * KB;
   const int ng = a.heads / a.groups;
   const int g = h / ng, m = h - g * ng;
   const int width = ng * a.d_h;
@@ -283,9 +300,9 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
   const int dq = a.d_h / 4;
   const T* q = static_cast<const T*>(a.q);
   T* out = static_cast<T*>(a.q_tilde);
-  constexpr int kB = 4;                                    // 16-byte loads per thread per batch
-  // stage query rows [i0, i0 + nq) of head h as fp32, batch by batch (loads, then stores)
+  // stage query rows [i0, i0 + nq) of head h as fp32 (zeros past nq)
   auto stage_q = [&](int i0, int nq) {
+    constexpr int kB = 2;
     for (int e0 = threadIdx.x; e0 < kAbsQ * dq; e0 += kB * kThreadsAbs) {
       float4 v[kB];
 #pragma unroll
@@ -301,37 +318,26 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
         const int e = e0 + u * kThreadsAbs;
-        if (e < kAbsQ * dq) reinterpret_cast<float4*>(sv)[e] = v[u];
+        if (e < kAbsQ * dq) {
+          const int qi = e / dq, d4 = e - qi * dq;
+          *reinterpret_cast<float4*>(sv + qi * pitch + d4 * 4) = v[u];
+        }
       }
     }
   };
-  // the slice times the gamma product, batch by batch; the first batch's loads go out with the
-  // gamma and first-pass query loads
-  auto load_w = [&](int e0, float4 (&v)[kB]) {
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int e = e0 + u * kThreadsAbs;
-      const int rr = e / dq, d4 = e - rr * dq;
-      v[u] = (e < kAbsK * dq && kbase + rr < a.r)
-                 ? *reinterpret_cast<const float4*>(w + (int64_t)(kbase + rr) * width + d4 * 4)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto store_w = [&](int e0, const float4 (&v)[kB]) {
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int e = e0 + u * kThreadsAbs;
-      if (e < kAbsK * dq) {
-        const int rr = e / dq, d4 = e - rr * dq;
-        const float4 gg = reinterpret_cast<const float4*>(g2)[d4];
-        *reinterpret_cast<float4*>(wc + rr * pitch + d4 * 4) =
-            make_float4(v[u].x * gg.x, v[u].y * gg.y, v[u].z * gg.z, v[u].w * gg.w);
-      }
-    }
-  };
+  // the slice times the gamma product: all of a thread's loads go out before its first store
   {
+    constexpr int kB = 8;
     float4 wv[kB];
-    load_w(threadIdx.x, wv);
+    const int total = KB * dq;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int e = threadIdx.x + u * kThreadsAbs;
+      const int rr = e / dq, d4 = e - rr * dq;
+      wv[u] = (e < total && kbase + rr < a.r)
+                  ? *reinterpret_cast<const float4*>(w + (int64_t)(kbase + rr) * width + d4 * 4)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float4 gq = make_float4(0.f, 0.f, 0.f, 0.f), gk = gq;
     if ((int)threadIdx.x < dq) {
       gq = *reinterpret_cast<const float4*>(a.gamma_q + h * a.d_h + threadIdx.x * 4);
@@ -341,14 +347,29 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
     if ((int)threadIdx.x < dq)
       reinterpret_cast<float4*>(g2)[threadIdx.x] = make_float4(gq.x * gk.x, gq.y * gk.y, gq.z * gk.z, gq.w * gk.w);
     __syncthreads();
-    store_w(threadIdx.x, wv);
-    for (int e0 = threadIdx.x + kB * kThreadsAbs; e0 < kAbsK * dq; e0 += kB * kThreadsAbs) {
-      load_w(e0, wv);
-      store_w(e0, wv);
+    auto store_w = [&](int e, const float4& v) {
+      const int rr = e / dq, d4 = e - rr * dq;
+      const float4 gg = reinterpret_cast<const float4*>(g2)[d4];
+      *reinterpret_cast<float4*>(wc + rr * pitch + d4 * 4) = make_float4(v.x * gg.x, v.y * gg.y, v.z * gg.z, v.w * gg.w);
+    };
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int e = threadIdx.x + u * kThreadsAbs;
+      if (e < total) store_w(e, wv[u]);
+    }
+    // d_h > 4 * kB * kThreadsAbs / KB: the rest of the slice, one vector at a time
+    for (int e = threadIdx.x + kB * kThreadsAbs; e < total; e += kThreadsAbs) {
+      const int rr = e / dq, d4 = e - rr * dq;
+      const float4 v = kbase + rr < a.r ? *reinterpret_cast<const float4*>(w + (int64_t)(kbase + rr) * width + d4 * 4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      store_w(e, v);
     }
   }
-  const float* wrow0 = wc + lane * pitch;
-  const float* wrow1 = wc + (lane + 32) * pitch;
+  const int rw = warp % kRowWarps, qw = warp / kRowWarps;
+  const int rg = lane & 7, qg = lane >> 3;
+  const int k0 = rw * 16 + rg;                             // rows k0 and k0 + 8 of the slice
+  const float* wrow0 = wc + k0 * pitch;
+  const float* wrow1 = wrow0 + 8 * pitch;
   for (int i0 = 0; i0 < a.n_q; i0 += kAbsQ) {
     const int nq = min(kAbsQ, a.n_q - i0);
     if (i0 > 0) {
@@ -356,30 +377,27 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
       stage_q(i0, nq);
     }
     __syncthreads();
-    float acc0[kJ], acc1[kJ];
-#pragma unroll
-    for (int j = 0; j < kJ; ++j) acc0[j] = acc1[j] = 0.f;
-    // query rows warp, warp + NW, ... of the pass that exist (warp-uniform)
-    const int nj = (nq - warp + NW - 1) / NW;
+    if (qw * 16 >= nq) continue;                           // no query rows for this warp (warp-uniform)
+    const float* qrow = sv + (qw * 16 + qg) * pitch;
+    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int d = 0; d < a.d_h; d += 4) {
       const float4 w0 = *reinterpret_cast<const float4*>(wrow0 + d);
       const float4 w1 = *reinterpret_cast<const float4*>(wrow1 + d);
 #pragma unroll
-      for (int j = 0; j < kJ; ++j) {
-        if (j < nj) {
-          const float4 sq = *reinterpret_cast<const float4*>(sv + (warp + NW * j) * a.d_h + d);
-          acc0[j] = fmaf(w0.x, sq.x, fmaf(w0.y, sq.y, fmaf(w0.z, sq.z, fmaf(w0.w, sq.w, acc0[j]))));
-          acc1[j] = fmaf(w1.x, sq.x, fmaf(w1.y, sq.y, fmaf(w1.z, sq.z, fmaf(w1.w, sq.w, acc1[j]))));
-        }
+      for (int v = 0; v < 4; ++v) {
+        const float4 sq = *reinterpret_cast<const float4*>(qrow + 4 * v * pitch + d);
+        acc0[v] = fmaf(w0.x, sq.x, fmaf(w0.y, sq.y, fmaf(w0.z, sq.z, fmaf(w0.w, sq.w, acc0[v]))));
+        acc1[v] = fmaf(w1.x, sq.x, fmaf(w1.y, sq.y, fmaf(w1.z, sq.z, fmaf(w1.w, sq.w, acc1[v]))));
       }
     }
 #pragma unroll
-    for (int j = 0; j < kJ; ++j) {
-      const int qi = warp + NW * j;
+    for (int v = 0; v < 4; ++v) {
+      const int qi = qw * 16 + qg + 4 * v;
       if (qi < nq) {
         T* o = out + ((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase;
-        if (kbase + lane < a.r) o[lane] = from_f32<T>(acc0[j]);
-        if (kbase + lane + 32 < a.r) o[lane + 32] = from_f32<T>(acc1[j]);
+        if (kbase + k0 < a.r) o[k0] = from_f32<T>(acc0[v]);
+        if (kbase + k0 + 8 < a.r) o[k0 + 8] = from_f32<T>(acc1[v]);
       }
     }
   }

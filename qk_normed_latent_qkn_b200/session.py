@@ -12,7 +12,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, append_absorb, decode,
+from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, append_absorb, decode, key_gram,
                decode_workspace_size, read_device_status, workspace_init)
 
 
@@ -27,7 +27,7 @@ class DecodeSession:
         self.dims = dims
         self.device = torch.device(device)
         self.cache = Cache(dims, num_blocks, device=self.device)
-        self.w_k = self.gamma_q = self.gamma_k = self.gamma_qr = self.gamma_kr = None
+        self.w_k = self.key_gram = self.gamma_q = self.gamma_k = self.gamma_qr = self.gamma_kr = None
         self.q_tilde = self.a_q = self.q_rope_hat = None
         self.workspace: Optional[torch.Tensor] = None
 
@@ -35,6 +35,9 @@ class DecodeSession:
     def load_weights(self, w_k, gamma_q, gamma_k, gamma_qr, gamma_kr) -> None:
         f32, dev = torch.float32, self.device
         self.w_k = to_device(w_k, f32, dev)
+        d = self.dims
+        self.key_gram = torch.empty((d.num_groups, d.r_kv, d.r_kv), dtype=f32, device=dev)
+        key_gram(d, self.w_k, self.key_gram)
         self.gamma_q = to_device(gamma_q, f32, dev)
         self.gamma_k = to_device(gamma_k, f32, dev)
         self.gamma_qr = to_device(gamma_qr, f32, dev)
@@ -49,7 +52,7 @@ class DecodeSession:
             sl = slice(t0, min(n, t0 + chunk))
             append(self.dims, self.cache, to_device(c[sl], dt, dev), to_device(k_rope_raw[sl], dt, dev),
                    to_device(slot[sl], torch.int32, dev), to_device(pos[sl], torch.int32, dev),
-                   self.w_k, self.gamma_kr)
+                   self.w_k, self.key_gram, self.gamma_kr)
 
     # ------------------------------------------------------------ queries
     def absorb(self, q, q_rope, pos) -> None:
@@ -69,7 +72,8 @@ class DecodeSession:
         self.ensure_query_buffers(q.shape[0])
         append_absorb(d, self.cache, to_device(c, dt, dev), to_device(k_rope_raw, dt, dev),
                       to_device(slot, torch.int32, dev), to_device(pos, torch.int32, dev), q,
-                      to_device(q_rope, dt, dev), to_device(qpos, torch.int32, dev), self.w_k, self.gamma_q,
+                      to_device(q_rope, dt, dev), to_device(qpos, torch.int32, dev), self.w_k, self.key_gram,
+                      self.gamma_q,
                       self.gamma_k, self.gamma_qr, self.gamma_kr, self.q_tilde, self.a_q, self.q_rope_hat)
 
     def ensure_query_buffers(self, n_q: int) -> None:

@@ -82,7 +82,8 @@ class DecodeStep:
         s, d, di = self.session, self.session.dims, self.dev_in
         self._dev_in_buf.copy_(self._host_in_buf, non_blocking=True)
         append_absorb(d, s.cache, di["c"], di["k_rope"], di["slot"], di["pos"], di["q"], di["q_rope"], di["qpos"],
-                      s.w_k, s.gamma_q, s.gamma_k, s.gamma_qr, s.gamma_kr, s.q_tilde, s.a_q, s.q_rope_hat)
+                      s.w_k, s.key_gram, s.gamma_q, s.gamma_k, s.gamma_qr, s.gamma_kr, s.q_tilde, s.a_q,
+                      s.q_rope_hat)
         decode(d, s.cache, s.q_tilde, s.a_q, s.q_rope_hat, di["block_table"], di["seq_lens"], self.s_q,
                self.workspace, self.out, self.lse, ak_mode=self.ak_mode, kernel=self.kernel, step_writes_only=True)
         self._host_out_buf.copy_(self._dev_out_buf, non_blocking=True)

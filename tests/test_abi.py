@@ -95,12 +95,20 @@ def test_append_and_absorb_reject_bad_arguments():
     lib = qkn.raw_library()
     dims = DIMS.c()
     cache = qkn._Cache(0x1000, 0x2000, 0x3000, 4)
-    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 0, None, None,
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 0, None, None, None,
                           None) == qkn.OK          # n_tok == 0 is a no-op
-    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 3, None, None,
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 3, None, None, None,
                           None) == qkn.ERR_INVALID_ARG
     assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), 0x100, 0x100, 0x100, 0x100, -1, 0x100,
-                          0x100, None) == qkn.ERR_INVALID_ARG
+                          None, 0x100, None) == qkn.ERR_INVALID_ARG
+    # neither w_k nor key_gram
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), 0x100, 0x100, 0x100, 0x100, 3, None,
+                          None, 0x100, None) == qkn.ERR_INVALID_ARG
+    # a misaligned Gram matrix
+    assert lib.qkn_append(ctypes.byref(dims), ctypes.byref(cache), 0x100, 0x100, 0x100, 0x100, 3, 0x100,
+                          0x102, 0x100, None) == qkn.ERR_INVALID_ARG
+    assert lib.qkn_key_gram(ctypes.byref(dims), None, 0x100, None) == qkn.ERR_INVALID_ARG
+    assert lib.qkn_key_gram(ctypes.byref(dims), 0x100, None, None) == qkn.ERR_INVALID_ARG
     assert lib.qkn_absorb_query(ctypes.byref(dims), None, None, None, 0, None, None, None, None, None, None,
                                 None, None) == qkn.OK
     assert lib.qkn_absorb_query(ctypes.byref(dims), None, None, None, 2, None, None, None, None, None, None,

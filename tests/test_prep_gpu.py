@@ -63,3 +63,42 @@ def test_one_launch_append_matches_three_launch_append(name):
     lb, rb, akb = _slots(b, slot)
     assert np.array_equal(la, lb) and np.array_equal(ra, rb)
     np.testing.assert_allclose(akb, aka, rtol=1e-5, atol=0)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "small_mla_bf16", "grouped_mtp_bf16"])
+def test_key_gram_matches_fp64(name):
+    import qk_normed_latent_qkn_b200 as qkn
+    inp = make_inputs(WORKLOADS[name])
+    s = session_from_inputs(inp)
+    torch.cuda.synchronize()
+    w = inp.w_k.astype(np.float64)                          # [G, r, n_g d_h]
+    ref = np.einsum("gik,gjk->gij", w, w)
+    got = s.key_gram.cpu().numpy()
+    # fp64 accumulation rounded once to fp32
+    assert np.abs(got - ref).max() <= 2 ** -23 * np.abs(ref).max()
+    assert np.array_equal(got, np.swapaxes(got, 1, 2))      # symmetric
+    assert s.key_gram.shape == (inp.wl.groups, inp.wl.r_kv, inp.wl.r_kv)
+    del qkn
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "grouped_mtp_bf16"])
+@pytest.mark.parametrize("scratch", [True, False])
+def test_gram_and_direct_key_statistic_match_oracle(name, scratch):
+    """qkn_append with key_gram (c G c^T) and without (sum of (c W)^2), in the one-launch and the
+    three-launch append, against the oracle's key statistic from explicitly formed keys."""
+    import oracle
+    import qk_normed_latent_qkn_b200 as qkn
+    inp = make_inputs(WORKLOADS[name])
+    c, kr, slot, pos, *_ = _step(inp)
+    s = session_from_inputs(inp)
+    if not scratch:
+        s.cache.ak_scratch = None
+    ref = oracle.key_inv_rms(c, inp.w_k, inp.wl.eps)
+    dev = lambda x, dt: torch.as_tensor(np.ascontiguousarray(x)).to(device=s.device, dtype=dt)
+    args = (dev(c, s.dims.torch_dtype), dev(kr, s.dims.torch_dtype), dev(slot, torch.int32), dev(pos, torch.int32))
+    for gram in (s.key_gram, None):
+        s.cache.a_k.zero_()
+        qkn.append(s.dims, s.cache, *args, s.w_k, gram, s.gamma_kr)
+        torch.cuda.synchronize()
+        ak = _slots(s, slot)[2]
+        np.testing.assert_allclose(ak, ref, rtol=2e-5, atol=0)
