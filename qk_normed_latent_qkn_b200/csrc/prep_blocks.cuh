@@ -5,6 +5,8 @@
 // CTAs of both kinds.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -255,6 +257,21 @@ __device__ __forceinline__ void absorb_row(const AbsorbArgs& a, int i, int h, fl
 
 constexpr int kAbsQ = 32;        // query rows per pass
 
+// fp32 -> TF32 (round to nearest, ties away), kept in an fp32 register
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+// D += A B, m16n8k8, TF32 inputs, fp32 accumulators (warp-wide)
+__device__ __forceinline__ void mma_tf32_m16n8k8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // Latent rows of W^K_{g,h} per absorption CTA of NW warps, and its shared memory.
 template <int NW>
 __host__ __device__ constexpr int absorb_rows() { return NW * 8; }
@@ -280,6 +297,9 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
   constexpr int KB = absorb_rows<NW>();
   constexpr int kRowWarps = NW / 2;
   static_assert(kRowWarps * 16 == KB && kAbsQ == 32, "warp tiling of the absorption CTA");
+  // bf16 storage: q~ is rounded to bf16 anyway, so the products run on the tensor cores in TF32
+  // (10-bit mantissa, fp32 accumulation); fp32 storage keeps fp32 FMAs
+  constexpr bool kTensor = std::is_same<T, __nv_bfloat16>::value;
   const int pitch = a.d_h + 4;
   float* wc = smem;                                        // [KB][d_h + 4]
   float* sv = wc + KB * pitch;                             // [kAbsQ][d_h + 4]
@@ -344,13 +364,18 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
       gk = *reinterpret_cast<const float4*>(a.gamma_k + h * a.d_h + threadIdx.x * 4);
     }
     stage_q(0, min(kAbsQ, a.n_q));
+    // the 4 pad columns of every W and query row stay zero: the TF32 loop reads them when d_h % 8 == 4
+    for (int rr = threadIdx.x; rr < KB + kAbsQ; rr += kThreadsAbs)
+      *reinterpret_cast<float4*>(wc + rr * pitch + a.d_h) = make_float4(0.f, 0.f, 0.f, 0.f);
     if ((int)threadIdx.x < dq)
       reinterpret_cast<float4*>(g2)[threadIdx.x] = make_float4(gq.x * gk.x, gq.y * gk.y, gq.z * gk.z, gq.w * gk.w);
     __syncthreads();
     auto store_w = [&](int e, const float4& v) {
       const int rr = e / dq, d4 = e - rr * dq;
       const float4 gg = reinterpret_cast<const float4*>(g2)[d4];
-      *reinterpret_cast<float4*>(wc + rr * pitch + d4 * 4) = make_float4(v.x * gg.x, v.y * gg.y, v.z * gg.z, v.w * gg.w);
+      float4 x = make_float4(v.x * gg.x, v.y * gg.y, v.z * gg.z, v.w * gg.w);
+      if constexpr (kTensor) x = make_float4(round_tf32(x.x), round_tf32(x.y), round_tf32(x.z), round_tf32(x.w));
+      *reinterpret_cast<float4*>(wc + rr * pitch + d4 * 4) = x;
     };
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
@@ -366,10 +391,6 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
     }
   }
   const int rw = warp % kRowWarps, qw = warp / kRowWarps;
-  const int rg = lane & 7, qg = lane >> 3;
-  const int k0 = rw * 16 + rg;                             // rows k0 and k0 + 8 of the slice
-  const float* wrow0 = wc + k0 * pitch;
-  const float* wrow1 = wrow0 + 8 * pitch;
   for (int i0 = 0; i0 < a.n_q; i0 += kAbsQ) {
     const int nq = min(kAbsQ, a.n_q - i0);
     if (i0 > 0) {
@@ -378,26 +399,64 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
     }
     __syncthreads();
     if (qw * 16 >= nq) continue;                           // no query rows for this warp (warp-uniform)
-    const float* qrow = sv + (qw * 16 + qg) * pitch;
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (kTensor) {
+      // m16n8k8 TF32 products: A = 16 rows of the slice, B = 8 query rows, per 8 columns of d_h.
+      // Fragments (lane = 4 gid + tig): A holds (row gid | gid + 8, column tig | tig + 4), B
+      // (query row gid, column tig | tig + 4), D (row gid | gid + 8, query row 2 tig | 2 tig + 1).
+      // With row pitch d_h + 4 the 32 lanes of every fragment read hit 32 distinct banks.
+      const int gid = lane >> 2, tig = lane & 3;
+      const float* wa = wc + (rw * 16 + gid) * pitch + tig;
+      const float* qb = sv + (qw * 16 + gid) * pitch + tig;
+      float dacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 4
-    for (int d = 0; d < a.d_h; d += 4) {
-      const float4 w0 = *reinterpret_cast<const float4*>(wrow0 + d);
-      const float4 w1 = *reinterpret_cast<const float4*>(wrow1 + d);
+      for (int d = 0; d < a.d_h; d += 8) {
+        const uint32_t af[4] = {__float_as_uint(wa[d]), __float_as_uint(wa[8 * pitch + d]),
+                                __float_as_uint(wa[d + 4]), __float_as_uint(wa[8 * pitch + d + 4])};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t bf[2] = {__float_as_uint(qb[j * 8 * pitch + d]), __float_as_uint(qb[j * 8 * pitch + d + 4])};
+          mma_tf32_m16n8k8(dacc[j], af, bf);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = rw * 16 + gid + (e >> 1) * 8;
+          const int qi = qw * 16 + j * 8 + 2 * tig + (e & 1);
+          if (qi < nq && kbase + row < a.r)
+            out[((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase + row] = from_f32<T>(dacc[j][e]);
+        }
+      }
+    } else {
+      // fp32 storage keeps fp32 FMAs: lane (rg, qg) = (lane % 8, lane / 8) takes rows rg, rg + 8
+      // of the warp's 16 and query rows qg, qg + 4, qg + 8, qg + 12: per 4 columns of d_h 2 W and
+      // 4 query vectors (16 bytes each, one wavefront per read) for 32 FMAs
+      const int rg = lane & 7, qg = lane >> 3;
+      const int k0 = rw * 16 + rg;
+      const float* wrow0 = wc + k0 * pitch;
+      const float* wrow1 = wrow0 + 8 * pitch;
+      const float* qrow = sv + (qw * 16 + qg) * pitch;
+      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int d = 0; d < a.d_h; d += 4) {
+        const float4 w0 = *reinterpret_cast<const float4*>(wrow0 + d);
+        const float4 w1 = *reinterpret_cast<const float4*>(wrow1 + d);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 sq = *reinterpret_cast<const float4*>(qrow + 4 * v * pitch + d);
+          acc0[v] = fmaf(w0.x, sq.x, fmaf(w0.y, sq.y, fmaf(w0.z, sq.z, fmaf(w0.w, sq.w, acc0[v]))));
+          acc1[v] = fmaf(w1.x, sq.x, fmaf(w1.y, sq.y, fmaf(w1.z, sq.z, fmaf(w1.w, sq.w, acc1[v]))));
+        }
+      }
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const float4 sq = *reinterpret_cast<const float4*>(qrow + 4 * v * pitch + d);
-        acc0[v] = fmaf(w0.x, sq.x, fmaf(w0.y, sq.y, fmaf(w0.z, sq.z, fmaf(w0.w, sq.w, acc0[v]))));
-        acc1[v] = fmaf(w1.x, sq.x, fmaf(w1.y, sq.y, fmaf(w1.z, sq.z, fmaf(w1.w, sq.w, acc1[v]))));
-      }
-    }
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int qi = qw * 16 + qg + 4 * v;
-      if (qi < nq) {
-        T* o = out + ((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase;
-        if (kbase + k0 < a.r) o[k0] = from_f32<T>(acc0[v]);
-        if (kbase + k0 + 8 < a.r) o[k0 + 8] = from_f32<T>(acc1[v]);
+        const int qi = qw * 16 + qg + 4 * v;
+        if (qi < nq) {
+          T* o = out + ((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase;
+          if (kbase + k0 < a.r) o[k0] = from_f32<T>(acc0[v]);
+          if (kbase + k0 + 8 < a.r) o[k0 + 8] = from_f32<T>(acc1[v]);
+        }
       }
     }
   }
