@@ -443,7 +443,7 @@ def run_ours(args, world, rank, local):
     t_qkn = statistics.median(per_mode[qkn.AK_CACHE])
     t_mla = statistics.median(per_mode[qkn.AK_ONE])
 
-    # end to end through the public API: DecodeStep replays copy-in, append || absorb, decode and
+    # end to end through the public API: DecodeStep replays copy-in, append + absorb (one launch), decode and
     # copy-out as one graph per step, from and to pinned host buffers, with a synchronize per step
     from qk_normed_latent_qkn_b200.step import DecodeStep
     names = {"c": "c", "kr": "k_rope", "slot": "slot", "pos": "pos", "q": "q", "qr": "q_rope", "qpos": "qpos",
@@ -504,7 +504,7 @@ def run_ours(args, world, rank, local):
             "breakdown_us": {"append_absorb": statistics.median(prep_ms) * 1e3,
                              "decode_split": statistics.median(split_ms) * 1e3,
                              "combine": statistics.median(combine_ms) * 1e3, "decode_op_timed": op_avg * 1e3,
-                             "what": "append and absorb (side stream) / split-KV kernel / merge kernel, from "
+                             "what": "append + absorb (one launch) / split-KV kernel / merge kernel, from "
                                      "separate graphs with an event between every stage; decode_op_timed is the "
                                      "split-KV + merge pair inside the timed steps"},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -513,9 +513,9 @@ def run_ours(args, world, rank, local):
                                           "committed ncu capture (profiles/); null when the kernel source "
                                           "or the workload differs from the capture's"),
                          "algorithmic_bytes": cost.bytes, "peak_source": f"{peak_src} HBM copy bandwidth",
-                         "kernel": ("decode op: split-KV kernel (tcgen05) + merge kernel, averaged over the timed "
-                                    "steps" if kernel_used == qkn.KERNEL_TCGEN05 else
-                                    "decode op: split-KV kernel (simt) + merge kernel, averaged over the timed steps"),
+                         "kernel": ("decode op: split-KV kernel (%s) + merge kernel, averaged over the timed steps, "
+                                    "from the end of the preparation kernel (all decode inputs written) to the end "
+                                    "of the merge" % ("tcgen05" if kernel_used == qkn.KERNEL_TCGEN05 else "simt")),
                          "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                     "frac": tflops / peaks["bf16_tflops"], "flops": cost.flops}},
             "overhead_vs_mla": {"qkn_us": t_qkn * 1e3, "mla_us": t_mla * 1e3, "frac": t_qkn / t_mla - 1.0,
@@ -523,7 +523,7 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "what": "DecodeStep.run(): one graph per step with copy-in from pinned host buffers, "
-                            "append || absorb, decode, copy-out to pinned host buffers; synchronize per step"},
+                            "append + absorb (one launch), decode, copy-out to pinned host buffers; synchronize per step"},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": sampler.summary(window),
             "cpu_baseline": cpu,

@@ -1,4 +1,4 @@
-"""DecodeStep (one graph per step: copy-in, append || absorb, decode, copy-out)
+"""DecodeStep (one graph per step: copy-in, append + absorb, decode, copy-out)
 against the eager session calls and the fp64 oracle (GPU)."""
 import copy
 
