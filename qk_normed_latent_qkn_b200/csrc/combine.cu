@@ -3,9 +3,10 @@
 // log-sum-exp lse_s; the row's result is
 //   lse = log sum_s exp(lse_s),   o = sum_s exp(lse_s - lse) * o_s,
 // which is exactly the softmax over the union of the splits' tokens.
-// One CTA per query row: warp 0 turns the row's split lse values into weights
-// (shared memory), then every thread owns 16 bytes of the row and streams the
-// splits' partials for them with independent loads.
+// One CTA per query row.  Every thread owns 16 bytes of the row and loads
+// them from the first eight splits while warp 0 turns the splits' lse values
+// into weights (shared memory); then the threads combine, streaming any
+// further splits eight at a time.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,19 +44,18 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   const int rho = ht * a.rows + row;
   if (b >= a.batch || rho >= qrows) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the row's splits: from the segment descriptor the tcgen05 decode wrote (every thread reads it,
+  // so that the partials' loads go out at once), else from the schedule, recomputed by warp 0
+  int64_t first;
+  int nitems;
   if (a.seg_desc) {
-    // a sequence with a rejected length has no splits: the tcgen05 kernel wrote its rows itself
     const int2 d = a.seg_desc[seg];
+    // a sequence with a rejected length has no splits: the tcgen05 kernel wrote its rows itself
     if (d.y <= 0) return;
-  }
-  if (warp == 0) {
-    int64_t first;
-    int nitems;
-    if (a.seg_desc) {
-      const int2 d = a.seg_desc[seg];
-      first = (int64_t)d.x * a.rows + row;
-      nitems = d.y;
-    } else {
+    first = (int64_t)d.x * a.rows + row;
+    nitems = d.y;
+  } else {
+    if (warp == 0) {
       SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
       const int64_t total = sched_total_units(sp);
       const int64_t before = sched_pages_before(sp, b);
@@ -64,9 +64,26 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
       const int64_t q = total > 0 ? (total + a.ncta - 1) / a.ncta : 1;
       const int64_t u0 = before * a.ht_count + (int64_t)ht * n;
       const int64_t c0 = u0 / q;
-      nitems = n > 0 ? (int)((u0 + n - 1) / q - c0 + 1) : 0;
-      first = (int64_t)(seg + c0) * a.rows + row;   // partial row of the first split
+      if (lane == 0) {
+        nitems_s = n > 0 ? (int)((u0 + n - 1) / q - c0 + 1) : 0;
+        first_s = (int64_t)(seg + c0) * a.rows + row;   // partial row of the first split
+      }
     }
+    __syncthreads();
+    first = first_s;
+    nitems = nitems_s;
+  }
+  // this thread's 16 bytes of the row from the first kHead splits, loaded beside the lse values
+  constexpr int kHead = 8;
+  const int nvec = a.r / 4;
+  const int64_t stride = (int64_t)a.rows * a.r / 4;        // float4s between consecutive splits of this row
+  const float4* src0 = reinterpret_cast<const float4*>(a.part_o + first * a.r);
+  float4 head[kHead];
+  const int v0 = threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < kHead; ++u)
+    head[u] = (u < nitems && v0 < nvec) ? src0[(int64_t)u * stride + v0] : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == 0) {
     float mx = -INFINITY;
     for (int c = lane; c < nitems; c += 32) mx = fmaxf(mx, a.part_lse[first + (int64_t)c * a.rows]);
 #pragma unroll
@@ -83,22 +100,26 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     const float inv = den > 0.f ? 1.f / den : 0.f;
     __syncwarp();
     for (int c = lane; c < nitems; c += 32) wsm[c] *= inv;
-    if (lane == 0) {
-      first_s = first;
-      nitems_s = nitems;
-      lse_s = (mx == -INFINITY) ? -INFINITY : mx + logf(den);
-    }
+    if (lane == 0) lse_s = (mx == -INFINITY) ? -INFINITY : mx + logf(den);
   }
   __syncthreads();
-  const int nitems = nitems_s;
   const int64_t orow = (int64_t)b * qrows + rho;
   T* out = static_cast<T*>(a.out) + orow * a.r;
-  const int nvec = a.r / 4;
-  const int64_t stride = (int64_t)a.rows * a.r / 4;        // float4s between consecutive splits of this row
-  for (int v = threadIdx.x; v < nvec; v += kCombThreads) {
-    const float4* src = reinterpret_cast<const float4*>(a.part_o + first_s * a.r) + v;
+  for (int v = v0; v < nvec; v += kCombThreads) {
+    const float4* src = src0 + v;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     int c = 0;
+    if (v == v0) {
+#pragma unroll
+      for (int u = 0; u < kHead; ++u) {
+        const float w = u < nitems ? wsm[u] : 0.f;
+        acc.x = fmaf(w, head[u].x, acc.x);
+        acc.y = fmaf(w, head[u].y, acc.y);
+        acc.z = fmaf(w, head[u].z, acc.z);
+        acc.w = fmaf(w, head[u].w, acc.w);
+      }
+      c = kHead;
+    }
     for (; c + 8 <= nitems; c += 8) {
       float4 x[8];
 #pragma unroll
