@@ -341,6 +341,9 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   a.rows = kernel == QKN_KERNEL_TCGEN05 ? tc_rows(dims, s_q, opts) : kSimtRows;
   a.ht_count = ceil_div(s_q * dims->num_heads, a.rows);
   a.ncta = ncta;
+  // starting an item costs about one page of time per 16 query rows of the tile (query tile,
+  // pipeline refill, the previous item's epilogue), measured on the tcgen05 kernel
+  a.item_cost = kernel == QKN_KERNEL_TCGEN05 ? (a.rows == 64 ? 3 : a.rows / 16) : 1;
   a.part_lse = reinterpret_cast<float*>(ws + w.lse_off);
   a.part_o = reinterpret_cast<float*>(ws + w.o_off);
   a.status = reinterpret_cast<int32_t*>(ws);
@@ -368,6 +371,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   c.rows = a.rows;
   c.ht_count = a.ht_count;
   c.ncta = ncta;
+  c.item_cost = a.item_cost;
   c.max_blocks = max_blocks;
   c.max_items = ncta + 1;
   c.part_o = a.part_o;

@@ -56,17 +56,16 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     nitems = d.y;
   } else {
     if (warp == 0) {
-      SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
+      SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost};
       const int64_t total = sched_total_units(sp);
-      const int64_t before = sched_pages_before(sp, b);
       const int32_t n = pages_of(a.seq_lens[b], sp);
       if (n == 0 && ht == 0 && row == 0 && lane == 0) record_status(a.status, QKN_ERR_BOUNDS);
       const int64_t q = total > 0 ? (total + a.ncta - 1) / a.ncta : 1;
-      const int64_t u0 = before * a.ht_count + (int64_t)ht * n;
-      const int64_t c0 = u0 / q;
+      const int64_t u0 = sched_units_before(sp, b) + (int64_t)ht * seg_units(n, sp);
+      const SegSplit sg = seg_split(u0, n, q, sp.item_cost);
       if (lane == 0) {
-        nitems_s = n > 0 ? (int)((u0 + n - 1) / q - c0 + 1) : 0;
-        first_s = (int64_t)(seg + c0) * a.rows + row;   // partial row of the first split
+        nitems_s = n > 0 ? sg.nitems : 0;
+        first_s = (int64_t)(seg + sg.c0) * a.rows + row;   // partial row of the first split
       }
     }
     __syncthreads();

@@ -90,6 +90,12 @@ __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
 // Q = ceil(total / ncta).  The piece of segment s that CTA c works on is an
 // "item"; its partial result goes to workspace slot s + c, which is unique
 // because segments and CTAs advance together.
+// Every segment starts with `item_cost` units that carry no page: starting an
+// item (loading its query tile, refilling the pipeline, writing the previous
+// item's result) costs about that many pages of time, so a CTA whose range
+// holds a segment start gets that many pages fewer, and CTAs that cross
+// segment boundaries no longer finish last.  A segment of sequence b is then
+// X + n(b) units, X = item_cost, its pages being the last n(b) of them.
 struct SchedParams {
   const int32_t* seq_lens;
   int32_t batch;
@@ -97,6 +103,7 @@ struct SchedParams {
   int32_t max_blocks;
   int32_t ht_count;     // query-row tiles per sequence
   int32_t ncta;
+  int32_t item_cost;    // units without pages at the start of every segment
 };
 
 __device__ __forceinline__ int32_t pages_of(int32_t L, const SchedParams& p) {
@@ -104,13 +111,18 @@ __device__ __forceinline__ int32_t pages_of(int32_t L, const SchedParams& p) {
   return (L + kBlockSize - 1) / kBlockSize;
 }
 
-// Total units, computed by one full warp (all lanes get the result).
-__device__ __forceinline__ int64_t sched_total_units(const SchedParams& p) {
+// Units of one segment of a sequence with n pages (none for a rejected length).
+__device__ __forceinline__ int64_t seg_units(int32_t n, const SchedParams& p) {
+  return n > 0 ? (int64_t)n + p.item_cost : 0;
+}
+
+// Units of the segments of sequences [0, b_end), computed by one full warp (all lanes get the result).
+__device__ __forceinline__ int64_t sched_units_before(const SchedParams& p, int32_t b_end) {
   const int lane = threadIdx.x & 31;
   int64_t acc = 0;
-  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+  for (int b0 = 0; b0 < b_end; b0 += 32) {
     int b = b0 + lane;
-    int64_t n = (b < p.batch) ? pages_of(p.seq_lens[b], p) : 0;
+    int64_t n = (b < b_end) ? seg_units(pages_of(p.seq_lens[b], p), p) : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
     acc += n;
@@ -118,18 +130,9 @@ __device__ __forceinline__ int64_t sched_total_units(const SchedParams& p) {
   return acc * p.ht_count;
 }
 
-// Pages before sequence b (P(b)), computed by one full warp.
-__device__ __forceinline__ int64_t sched_pages_before(const SchedParams& p, int32_t b_end) {
-  const int lane = threadIdx.x & 31;
-  int64_t acc = 0;
-  for (int b0 = 0; b0 < b_end; b0 += 32) {
-    int b = b0 + lane;
-    int64_t n = (b < b_end) ? pages_of(p.seq_lens[b], p) : 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-    acc += n;
-  }
-  return acc;
+// Total units, computed by one full warp.
+__device__ __forceinline__ int64_t sched_total_units(const SchedParams& p) {
+  return sched_units_before(p, p.batch);
 }
 
 // Cursor over the items of one CTA.  Start it with sched_begin (one full
@@ -143,7 +146,7 @@ struct Cursor {
 };
 
 // Item handed to the roles: pages [p0, p1) of sequence b, row tile ht; the
-// segment's units are [seg_u0, seg_u0 + (pages of b)).
+// segment's units are [seg_u0, seg_u0 + item_cost + (pages of b)).
 struct Item {
   int32_t b, ht, p0, p1, L, slot;
   int64_t seg_u0;
@@ -166,7 +169,7 @@ __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta)
   int64_t base = 0;
   for (int b0 = 0; b0 < p.batch; b0 += 32) {
     int b = b0 + lane;
-    int64_t n = (b < p.batch) ? pages_of(p.seq_lens[b], p) * (int64_t)p.ht_count : 0;
+    int64_t n = (b < p.batch) ? seg_units(pages_of(p.seq_lens[b], p), p) * p.ht_count : 0;
     int64_t incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -180,10 +183,11 @@ __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta)
       const int64_t seq_lo = __shfl_sync(0xffffffffu, lo, src);
       const int32_t bb = b0 + src;
       const int32_t nn = pages_of(p.seq_lens[bb], p);
+      const int64_t su = seg_units(nn, p);
       cur.b = bb;
       cur.n = nn;
-      cur.ht = (int32_t)((cur.begin - seq_lo) / nn);
-      cur.seg_u0 = seq_lo + (int64_t)cur.ht * nn;
+      cur.ht = (int32_t)((cur.begin - seq_lo) / su);
+      cur.seg_u0 = seq_lo + (int64_t)cur.ht * su;
       return cur;
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
@@ -194,13 +198,16 @@ __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta)
 // Returns false when the CTA has no further item.  Any single thread.
 __device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, int32_t cta, Item& it) {
   while (cur.b < p.batch && cur.seg_u0 < cur.end) {
-    const int64_t s0 = cur.seg_u0, s1 = cur.seg_u0 + cur.n;
-    const bool overlaps = cur.n > 0 && s1 > cur.begin;
+    // the segment's pages are units [s0 + item_cost, s1)
+    const int64_t s0 = cur.seg_u0, s1 = cur.seg_u0 + seg_units(cur.n, p);
+    const int64_t pg0 = s0 + p.item_cost;
+    const int64_t lo = cur.begin > pg0 ? cur.begin : pg0, hi = cur.end < s1 ? cur.end : s1;
+    const bool overlaps = cur.n > 0 && lo < hi;
     if (overlaps) {
       it.b = cur.b;
       it.ht = cur.ht;
-      it.p0 = (int32_t)((cur.begin > s0 ? cur.begin : s0) - s0);
-      it.p1 = (int32_t)((cur.end < s1 ? cur.end : s1) - s0);
+      it.p0 = (int32_t)(lo - pg0);
+      it.p1 = (int32_t)(hi - pg0);
       it.L = p.seq_lens[cur.b];
       it.slot = cur.b * p.ht_count + cur.ht + cta;
       it.seg_u0 = s0;
@@ -218,16 +225,18 @@ __device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, in
   return false;
 }
 
-// The CTAs that share a segment: units [u0, u0 + n) are split over CTAs
-// c0 .. c0 + nitems - 1 (quota q units each), whose partial results sit in
-// workspace slots seg + c0 .. seg + c0 + nitems - 1.
+// The CTAs that share a segment: its pages, units [u0 + item_cost, u0 +
+// item_cost + n), are split over CTAs c0 .. c0 + nitems - 1 (quota q units
+// each), whose partial results sit in workspace slots seg + c0 .. seg + c0 +
+// nitems - 1.
 struct SegSplit {
   int32_t c0, nitems;
 };
-__device__ __forceinline__ SegSplit seg_split(int64_t u0, int32_t n, int64_t q) {
+__device__ __forceinline__ SegSplit seg_split(int64_t u0, int32_t n, int64_t q, int32_t item_cost) {
   SegSplit s;
-  s.c0 = (int32_t)(u0 / q);
-  s.nitems = (int32_t)((u0 + n - 1) / q) - s.c0 + 1;
+  const int64_t pg0 = u0 + item_cost;
+  s.c0 = (int32_t)(pg0 / q);
+  s.nitems = (int32_t)((pg0 + n - 1) / q) - s.c0 + 1;
   return s;
 }
 

@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
   MiscT& ms = *reinterpret_cast<MiscT*>(smem + C::MISC_OFF);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta};
+  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost};
   const int qrows = a.s_q * a.heads;
   const int G = a.groups;
 
@@ -749,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       mbar_arrive(smem_u32(&ms.o_empty));
       // the CTA holding a segment's first split tells the merge kernel where its splits are
       if (threadIdx.x == 0 && it.p0 == 0) {
-        const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota);
+        const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota, sp.item_cost);
         a.seg_desc[it.b * a.ht_count + it.ht] = make_int2(it.b * a.ht_count + it.ht + sg.c0, sg.nitems);
       }
       ++n_item;

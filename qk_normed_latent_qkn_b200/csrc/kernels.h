@@ -65,6 +65,7 @@ struct DecodeArgs {
   int32_t rows;              // query rows per tile (R)
   int32_t ht_count;          // tiles per sequence = ceil(s_q*H / R)
   int32_t ncta;
+  int32_t item_cost;         // schedule units without pages at the start of every segment
   float* part_o;             // [slots, R, r] fp32
   float* part_lse;           // [slots, R] fp32
   int32_t* status;           // workspace status word
@@ -80,6 +81,7 @@ struct DecodeArgs {
 struct CombineArgs {
   const int32_t* seq_lens;
   int32_t batch, s_q, heads, r, rows, ht_count, ncta, max_blocks;
+  int32_t item_cost;         // as in DecodeArgs
   int32_t max_items;         // upper bound on splits per row (ncta + 1)
   const float* part_o;
   const float* part_lse;
