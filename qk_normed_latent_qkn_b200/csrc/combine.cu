@@ -31,8 +31,10 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4
   *reinterpret_cast<uint2*>(dst) = u;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kCombThreads, 12) combine_kernel(CombineArgs a) {
+// kDesc: the splits come from the segment descriptors the tcgen05 decode wrote; else from the
+// schedule, recomputed (one instantiation each keeps the descriptor path small)
+template <typename T, bool kDesc>
+__global__ void __launch_bounds__(kCombThreads, kDesc ? 12 : 8) combine_kernel(CombineArgs a) {
   __shared__ int64_t first_s;
   __shared__ int nitems_s;
   pdl_trigger();
@@ -47,7 +49,7 @@ __global__ void __launch_bounds__(kCombThreads, 12) combine_kernel(CombineArgs a
   // schedule, recomputed by warp 0
   int64_t first;
   int nitems;
-  if (a.seg_desc) {
+  if constexpr (kDesc) {
     const int2 d = a.seg_desc[seg];
     // a sequence with a rejected length has no splits: the tcgen05 kernel wrote its rows itself
     if (d.y <= 0) return;
@@ -60,12 +62,12 @@ __global__ void __launch_bounds__(kCombThreads, 12) combine_kernel(CombineArgs a
       const int64_t total = sched_total_units(sp);
       const int32_t n = pages_of(a.seq_lens[b], sp);
       if (n == 0 && ht == 0 && row == 0 && lane == 0) record_status(a.status, QKN_ERR_BOUNDS);
-      const int64_t q = total > 0 ? (total + a.ncta - 1) / a.ncta : 1;
-      const int64_t u0 = sched_units_before(sp, b) + (int64_t)ht * seg_units(n, sp);
-      const SegSplit sg = seg_split(u0, n, q, sp.item_cost);
+      const int32_t ng = sched_groups(sp);
+      const int64_t q = total > 0 ? (total + ng - 1) / ng : 1;
+      const SegSplit sg = seg_split(sched_units_before(sp, b), n, q, sp.item_cost);
       if (lane == 0) {
         nitems_s = n > 0 ? sg.nitems : 0;
-        first_s = (int64_t)(seg + sg.c0) * a.rows + row;   // partial row of the first split
+        first_s = ((int64_t)(b + sg.c0) * a.ht_count + ht) * a.rows + row;   // partial row of the first split
       }
     }
     __syncthreads();
@@ -77,7 +79,9 @@ __global__ void __launch_bounds__(kCombThreads, 12) combine_kernel(CombineArgs a
   // The lse values and the partials of kDepth splits are loaded together.
   constexpr int kDepth = 4;
   const int nvec = a.r / 4;
-  const int64_t stride = (int64_t)a.rows * a.r / 4;        // float4s between consecutive splits of this row
+  // consecutive splits of a segment sit ht_count slots apart
+  const int64_t lstride = (int64_t)a.rows * a.ht_count;
+  const int64_t stride = lstride * a.r / 4;                 // float4s between consecutive splits of this row
   const float4* src0 = reinterpret_cast<const float4*>(a.part_o + first * a.r);
   const float* lsrc = a.part_lse + first;
   const int64_t orow = (int64_t)b * qrows + rho;
@@ -91,7 +95,7 @@ __global__ void __launch_bounds__(kCombThreads, 12) combine_kernel(CombineArgs a
 #pragma unroll
       for (int u = 0; u < kDepth; ++u) {
         const bool in = c + u < nitems;
-        ls[u] = in ? lsrc[(int64_t)(c + u) * a.rows] : -INFINITY;
+        ls[u] = in ? lsrc[(int64_t)(c + u) * lstride] : -INFINITY;
         x[u] = in ? src0[(int64_t)(c + u) * stride + v] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       float mc = m;
@@ -121,8 +125,12 @@ __global__ void __launch_bounds__(kCombThreads, 12) combine_kernel(CombineArgs a
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st) {
   const int64_t rows = (int64_t)a.batch * a.ht_count * a.rows;
   const size_t smem = 0;
-  if (bf16) return launch_chained(combine_kernel<__nv_bfloat16>, dim3((unsigned)rows), dim3(kCombThreads), smem, st, a);
-  return launch_chained(combine_kernel<float>, dim3((unsigned)rows), dim3(kCombThreads), smem, st, a);
+  const dim3 grid((unsigned)rows), block(kCombThreads);
+  if (a.seg_desc)
+    return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, true>, grid, block, smem, st, a)
+                : launch_chained(combine_kernel<float, true>, grid, block, smem, st, a);
+  return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, false>, grid, block, smem, st, a)
+              : launch_chained(combine_kernel<float, false>, grid, block, smem, st, a);
 }
 
 }  // namespace qkn

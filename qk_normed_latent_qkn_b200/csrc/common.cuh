@@ -81,29 +81,31 @@ __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
 }
 
 // ---------------------------------------------------------------- schedule
-// The decode work of one step is a list of "units": one cache page (64
-// tokens) of one segment, a segment being (sequence b, query-row tile ht).
-// Segments are ordered (b, ht) and units inside a segment by page, so the
-// units of segment (b, ht) are [HT*P(b) + ht*n(b), ... + n(b)) where n(b) is
-// the page count of sequence b and P(b) the pages of sequences before it.
-// CTA c of `ncta` takes the contiguous unit range [c*Q, (c+1)*Q) with
-// Q = ceil(total / ncta).  The piece of segment s that CTA c works on is an
-// "item"; its partial result goes to workspace slot s + c, which is unique
-// because segments and CTAs advance together.
-// Every segment starts with `item_cost` units that carry no page: starting an
-// item (loading its query tile, refilling the pipeline, writing the previous
-// item's result) costs about that many pages of time, so a CTA whose range
-// holds a segment start gets that many pages fewer, and CTAs that cross
-// segment boundaries no longer finish last.  A segment of sequence b is then
-// X + n(b) units, X = item_cost, its pages being the last n(b) of them.
+// The decode work of one step: every sequence b has n(b) cache pages of 64
+// tokens and HT query-row tiles; a segment is (sequence b, row tile ht).
+// The CTAs form groups of HC = min(HT, ncta) CTAs, G = floor(ncta / HC) of
+// them; CTA c is member c mod HC of group c / HC and takes the row tiles ht
+// with ht mod HC = c mod HC.  The pages are laid out in "units", sequence by
+// sequence; group g takes the contiguous unit range [g*Q, (g+1)*Q),
+// Q = ceil(total / G), and every member works on the same pages for its own
+// row tiles.  So the CTAs that read a page for different row tiles read it at
+// about the same time, and the second read comes from L2 rather than HBM.
+// Every sequence starts with `item_cost` units that carry no page: starting
+// an item (loading its query tile, refilling the pipeline, writing the
+// previous item's result) costs about that many pages of time, so a group
+// whose range holds a sequence start gets that many pages fewer.  Sequence b
+// is X + n(b) units (X = item_cost), its pages the last n(b) of them.
+// The piece of segment (b, ht) that a CTA of group g works on is an "item";
+// its partial result goes to workspace slot (b + g) * HT + ht, unique because
+// sequences and groups advance together.
 struct SchedParams {
   const int32_t* seq_lens;
   int32_t batch;
   int32_t s_q;
   int32_t max_blocks;
-  int32_t ht_count;     // query-row tiles per sequence
+  int32_t ht_count;     // query-row tiles per sequence (HT)
   int32_t ncta;
-  int32_t item_cost;    // units without pages at the start of every segment
+  int32_t item_cost;    // units without pages at the start of every sequence
 };
 
 __device__ __forceinline__ int32_t pages_of(int32_t L, const SchedParams& p) {
@@ -111,23 +113,32 @@ __device__ __forceinline__ int32_t pages_of(int32_t L, const SchedParams& p) {
   return (L + kBlockSize - 1) / kBlockSize;
 }
 
-// Units of one segment of a sequence with n pages (none for a rejected length).
-__device__ __forceinline__ int64_t seg_units(int32_t n, const SchedParams& p) {
+// Units of a sequence with n pages (none for a rejected length).
+__device__ __forceinline__ int64_t seq_units(int32_t n, const SchedParams& p) {
   return n > 0 ? (int64_t)n + p.item_cost : 0;
 }
 
-// Units of the segments of sequences [0, b_end), computed by one full warp (all lanes get the result).
+// CTAs per group (HC) and groups (G).
+__device__ __forceinline__ int32_t sched_group_size(const SchedParams& p) {
+  return p.ht_count < p.ncta ? p.ht_count : (p.ncta > 0 ? p.ncta : 1);
+}
+__device__ __forceinline__ int32_t sched_groups(const SchedParams& p) {
+  const int32_t g = p.ncta / sched_group_size(p);
+  return g > 0 ? g : 1;
+}
+
+// Units of sequences [0, b_end), computed by one full warp (all lanes get the result).
 __device__ __forceinline__ int64_t sched_units_before(const SchedParams& p, int32_t b_end) {
   const int lane = threadIdx.x & 31;
   int64_t acc = 0;
   for (int b0 = 0; b0 < b_end; b0 += 32) {
     int b = b0 + lane;
-    int64_t n = (b < b_end) ? seg_units(pages_of(p.seq_lens[b], p), p) : 0;
+    int64_t n = (b < b_end) ? seq_units(pages_of(p.seq_lens[b], p), p) : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
     acc += n;
   }
-  return acc * p.ht_count;
+  return acc;
 }
 
 // Total units, computed by one full warp.
@@ -138,15 +149,17 @@ __device__ __forceinline__ int64_t sched_total_units(const SchedParams& p) {
 // Cursor over the items of one CTA.  Start it with sched_begin (one full
 // warp), copy it to every role, then step with sched_next (any thread).
 struct Cursor {
-  int64_t begin, end;    // this CTA's unit range
-  int64_t seg_u0;        // first unit of the current segment
-  int32_t b, ht;         // current segment
+  int64_t begin, end;    // the group's unit range
+  int64_t seq_u0;        // first unit of the current sequence
+  int32_t b, ht;         // current sequence and row tile
   int32_t n;             // pages of sequence b
+  int32_t group;         // g
+  int32_t ht0, hstep;    // this CTA's first row tile and the step between its row tiles (HC)
   int64_t quota;         // Q
 };
 
 // Item handed to the roles: pages [p0, p1) of sequence b, row tile ht; the
-// segment's units are [seg_u0, seg_u0 + item_cost + (pages of b)).
+// sequence's units are [seg_u0, seg_u0 + item_cost + (pages of b)).
 struct Item {
   int32_t b, ht, p0, p1, L, slot;
   int64_t seg_u0;
@@ -156,20 +169,27 @@ __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta)
   Cursor cur;
   const int lane = threadIdx.x & 31;
   const int64_t total = sched_total_units(p);
-  const int64_t q = (total + p.ncta - 1) / (p.ncta > 0 ? p.ncta : 1);
-  cur.quota = q;
-  cur.begin = (int64_t)cta * q;
-  cur.end = cur.begin + q < total ? cur.begin + q : total;
+  const int32_t hc = sched_group_size(p), ng = sched_groups(p);
+  const int64_t q = (total + ng - 1) / ng;
+  cur.quota = q > 0 ? q : 1;
+  cur.group = cta / hc;
+  cur.ht0 = cta - cur.group * hc;
+  cur.hstep = hc;
+  cur.ht = cur.ht0;
+  cur.begin = (int64_t)cur.group * cur.quota;
+  cur.end = cur.begin + cur.quota < total ? cur.begin + cur.quota : total;
   cur.b = p.batch;
-  cur.ht = 0;
   cur.n = 0;
-  cur.seg_u0 = total;
-  if (cur.begin >= cur.end) return cur;
+  cur.seq_u0 = total;
+  if (cur.group >= ng || cur.ht0 >= p.ht_count || cur.begin >= cur.end) {
+    cur.begin = cur.end = total;                     // no work
+    return cur;
+  }
   // Find the sequence holding unit `begin`: scan with a warp prefix sum.
   int64_t base = 0;
   for (int b0 = 0; b0 < p.batch; b0 += 32) {
     int b = b0 + lane;
-    int64_t n = (b < p.batch) ? seg_units(pages_of(p.seq_lens[b], p), p) * p.ht_count : 0;
+    int64_t n = (b < p.batch) ? seq_units(pages_of(p.seq_lens[b], p), p) : 0;
     int64_t incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -180,14 +200,9 @@ __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta)
     const unsigned hit = __ballot_sync(0xffffffffu, b < p.batch && n > 0 && cur.begin >= lo && cur.begin < hi);
     if (hit) {
       const int src = __ffs(hit) - 1;
-      const int64_t seq_lo = __shfl_sync(0xffffffffu, lo, src);
-      const int32_t bb = b0 + src;
-      const int32_t nn = pages_of(p.seq_lens[bb], p);
-      const int64_t su = seg_units(nn, p);
-      cur.b = bb;
-      cur.n = nn;
-      cur.ht = (int32_t)((cur.begin - seq_lo) / su);
-      cur.seg_u0 = seq_lo + (int64_t)cur.ht * su;
+      cur.seq_u0 = __shfl_sync(0xffffffffu, lo, src);
+      cur.b = b0 + src;
+      cur.n = pages_of(p.seq_lens[cur.b], p);
       return cur;
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
@@ -197,40 +212,41 @@ __device__ __forceinline__ Cursor sched_begin(const SchedParams& p, int32_t cta)
 
 // Returns false when the CTA has no further item.  Any single thread.
 __device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, int32_t cta, Item& it) {
-  while (cur.b < p.batch && cur.seg_u0 < cur.end) {
-    // the segment's pages are units [s0 + item_cost, s1)
-    const int64_t s0 = cur.seg_u0, s1 = cur.seg_u0 + seg_units(cur.n, p);
+  (void)cta;
+  while (cur.b < p.batch && cur.seq_u0 < cur.end) {
+    // the sequence's pages are units [s0 + item_cost, s1)
+    const int64_t s0 = cur.seq_u0, s1 = s0 + seq_units(cur.n, p);
     const int64_t pg0 = s0 + p.item_cost;
     const int64_t lo = cur.begin > pg0 ? cur.begin : pg0, hi = cur.end < s1 ? cur.end : s1;
-    const bool overlaps = cur.n > 0 && lo < hi;
+    const bool overlaps = cur.n > 0 && lo < hi && cur.ht < p.ht_count;
     if (overlaps) {
       it.b = cur.b;
       it.ht = cur.ht;
       it.p0 = (int32_t)(lo - pg0);
       it.p1 = (int32_t)(hi - pg0);
       it.L = p.seq_lens[cur.b];
-      it.slot = cur.b * p.ht_count + cur.ht + cta;
+      it.slot = (cur.b + cur.group) * p.ht_count + cur.ht;
       it.seg_u0 = s0;
+      cur.ht += cur.hstep;                       // this CTA's next row tile of the same pages
+      if (cur.ht < p.ht_count) return true;
     }
-    // advance to the next segment
-    cur.seg_u0 = s1;
-    if (++cur.ht >= p.ht_count || cur.n == 0) {
-      cur.ht = 0;
-      ++cur.b;
-      cur.n = cur.b < p.batch ? pages_of(p.seq_lens[cur.b], p) : 0;
-      if (cur.n == 0) cur.ht = 0;
-    }
+    // advance to the next sequence
+    cur.ht = cur.ht0;
+    cur.seq_u0 = s1;
+    ++cur.b;
+    cur.n = cur.b < p.batch ? pages_of(p.seq_lens[cur.b], p) : 0;
     if (overlaps) return true;
   }
   return false;
 }
 
-// The CTAs that share a segment: its pages, units [u0 + item_cost, u0 +
-// item_cost + n), are split over CTAs c0 .. c0 + nitems - 1 (quota q units
-// each), whose partial results sit in workspace slots seg + c0 .. seg + c0 +
-// nitems - 1.
+// The groups that share a sequence: its pages, units [u0 + item_cost, u0 +
+// item_cost + n), are split over groups g0 .. g0 + nitems - 1 (quota q units
+// each); the partial results of segment (b, ht) sit in workspace slots
+// (b + g) * HT + ht for those groups: first slot (b + g0) * HT + ht, then
+// every HT-th slot.
 struct SegSplit {
-  int32_t c0, nitems;
+  int32_t c0, nitems;   // first group, number of splits
 };
 __device__ __forceinline__ SegSplit seg_split(int64_t u0, int32_t n, int64_t q, int32_t item_cost) {
   SegSplit s;

@@ -750,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       // the CTA holding a segment's first split tells the merge kernel where its splits are
       if (threadIdx.x == 0 && it.p0 == 0) {
         const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota, sp.item_cost);
-        a.seg_desc[it.b * a.ht_count + it.ht] = make_int2(it.b * a.ht_count + it.ht + sg.c0, sg.nitems);
+        a.seg_desc[it.b * a.ht_count + it.ht] = make_int2((it.b + sg.c0) * a.ht_count + it.ht, sg.nitems);
       }
       ++n_item;
     }
