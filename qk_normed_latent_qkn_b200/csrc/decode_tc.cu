@@ -102,6 +102,7 @@ struct Cfg {
 template <int R, int NS, int NKR>
 struct Misc {
   uint64_t full[NS], empty[NS], krfull[NKR], krempty[NKR];
+  uint64_t akfull[NKR];           // the page's a_k rows landed (read by the softmax only)
   uint64_t s_full[2], s_empty[2];
   // Per-tile handshakes alternate between two barriers by tile parity (tile n: barrier n & 1,
   // phase n >> 1): the softmax may run two tiles ahead of the output issuer, and a parity wait
@@ -223,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     }
     for (int s = 0; s < NKR; ++s) {
       mbar_init(smem_u32(&ms.krfull[s]), 1);
+      mbar_init(smem_u32(&ms.akfull[s]), 1);
       mbar_init(smem_u32(&ms.krempty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -326,11 +328,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           }
           if (!ok) break;
           if (!mbar_wait_warp(smem_u32(&ms.krempty[kw.slot]), kw.phase ^ 1u, a.wait_limit)) { ok = false; break; }
+          // the RoPE keys feed the score MMAs; the a_k rows only the softmax, so they get their own
+          // barrier and their latency stays off the score path
           const uint32_t kb = smem_u32(&ms.krfull[kw.slot]);
-          mbar_arrive_expect_tx_elect(kb, kKrBytes + (AK_ONE ? 0u : akpage));
+          mbar_arrive_expect_tx_elect(kb, kKrBytes);
           tma_load_2d_elect(sb + C::KR_OFF + kw.slot * kKrBytes, &maps.krope, 0, blk * kPage, kb);
-          if (!AK_ONE)
-            bulk_load_elect(sb + C::AK_OFF + kw.slot * kAkSlotBytes, a.a_k + (int64_t)blk * kPage * G, akpage, kb);
+          if (!AK_ONE) {
+            const uint32_t akb = smem_u32(&ms.akfull[kw.slot]);
+            mbar_arrive_expect_tx_elect(akb, akpage);
+            bulk_load_elect(sb + C::AK_OFF + kw.slot * kAkSlotBytes, a.a_k + (int64_t)blk * kPage * G, akpage, akb);
+          }
           kw.next();
           ++k_issued;
         }
@@ -347,8 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       for (int64_t i = first; i < c_issued; ++i)
         mbar_wait(smem_u32(&ms.full[i % NS]), (i / NS) & 1, kDrainLimit);
       const int64_t kfirst = k_issued > NKR ? k_issued - NKR : 0;
-      for (int64_t i = kfirst; i < k_issued; ++i)
+      for (int64_t i = kfirst; i < k_issued; ++i) {
         mbar_wait(smem_u32(&ms.krfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
+        if (!AK_ONE) mbar_wait(smem_u32(&ms.akfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
+      }
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------------------ score MMA issuer (whole warp)
@@ -549,11 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const int tpos = tok0 + tok;
         const float* akrow = reinterpret_cast<const float*>(smem + C::AK_OFF + ks * kAkSlotBytes) + tok * G;
         float ak0 = 1.f;
-        if (!AK_ONE) {
-          // the RoPE-key barrier also covers the a_k rows; it completed before S did
-          got = mbar_wait(smem_u32(&ms.krfull[ks]), kr.phase, a.wait_limit) && got;
-          ak0 = akrow[0];
-        }
         // this token's scaled logits, log2 units, of this thread's columns (-inf where not visible)
         float x[NJ];
         {
@@ -570,6 +574,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
             } else {
               tmem_ld16x64_x16(tSc + cb + 2 * b0, sc);
               tmem_ld16x64_x16(tSc + R + cb + 2 * b0, sr);
+            }
+            if (!AK_ONE && b0 == 0) {
+              // the a_k rows: their barrier and load overlap the TMEM loads' latency
+              got = mbar_wait(smem_u32(&ms.akfull[ks]), kr.phase, a.wait_limit) && got;
+              ak0 = akrow[0];
             }
             tmem_wait_ld();
             reg_tie(sc);
