@@ -152,3 +152,15 @@ def test_bad_sequence_length_is_reported_not_faulted():
     assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
     s.clear_status()
     assert s.device_status() == qkn.OK
+
+
+@pytest.mark.parametrize("kernel,max_ctas", [("tcgen05", 1), ("tcgen05", 3), ("tcgen05", 7), ("simt", 5), ("simt", 1)])
+def test_cta_group_edges(kernel, max_ctas):
+    # 128 heads: two 64-row tiles per sequence on the tensor cores (groups of two CTAs; an odd CTA
+    # count leaves one idle, one CTA takes both tiles of every sequence), sixteen 8-row tiles on the
+    # CUDA cores (five CTAs form one group, each taking every fifth tile of the same pages)
+    inp = make_inputs(SMALL["large_mla_bf16"])
+    s, o, lse = run_decode(inp, kernel=KERNELS[kernel], max_ctas=max_ctas)
+    assert_close_to_oracle(inp, o, lse, what=f"{kernel}, {max_ctas} CTAs")
+    _, o_all, _ = run_decode(inp, kernel=KERNELS[kernel], session=s)
+    assert np.abs(o - o_all).max() <= 1e-2 * np.abs(o_all).max()
