@@ -70,8 +70,9 @@ struct DecodeArgs {
   float* part_lse;           // [slots, R] fp32
   int32_t* status;           // workspace status word
   int64_t wait_limit;        // bounded-wait cycles (tcgen05 kernel)
-  // tcgen05 kernel only: a segment finished by one CTA is written to out / lse directly, and
-  // seg_desc[segment] = (first split slot, number of splits) tells the merge kernel the rest
+  // tcgen05 kernel only: the rows of a sequence with a rejected length are written to out / lse
+  // directly (zeros, -inf), and seg_desc[segment] = (first split slot, number of splits; the
+  // splits sit ht_count slots apart) tells the merge kernel where the partials are
   void* out;                 // [batch, s_q, H, r] bf16
   float* lse;                // [batch, s_q, H]
   int2* seg_desc;            // [batch * ht_count]
