@@ -119,3 +119,22 @@ def test_kernel_choice_is_host_logic():
     f32 = qkn.Dims(num_heads=4, num_groups=1, r_kv=64, d_h=32, d_rope=16, dtype=qkn.F32)
     assert qkn.decode_kernel_for(f32, 1) == qkn.KERNEL_SIMT
     assert qkn.decode_kernel_for(f32, 1, kernel=qkn.KERNEL_TCGEN05) == -1
+
+
+def test_append_absorb_validates_both_halves_before_any_launch():
+    lib = qkn.raw_library()
+    dims = DIMS.c()
+    cache = qkn._Cache(0x1000, 0x2000, 0x3000, 4)
+    P = 0x100
+    # nothing to do: no tokens, no query rows
+    assert lib.qkn_append_absorb(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 0, None, None,
+                                 None, 0, None, None, None, None, None, None, None, None, None, None) == qkn.OK
+    # tokens without their arrays
+    assert lib.qkn_append_absorb(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 2, None, None,
+                                 None, 0, P, None, P, P, P, P, None, None, None, None) == qkn.ERR_INVALID_ARG
+    # query rows without their outputs
+    assert lib.qkn_append_absorb(ctypes.byref(dims), ctypes.byref(cache), None, None, None, None, 0, P, P, P, 2,
+                                 P, None, P, P, P, P, None, None, None, None) == qkn.ERR_INVALID_ARG
+    # negative counts
+    assert lib.qkn_append_absorb(ctypes.byref(dims), ctypes.byref(cache), P, P, P, P, -1, P, P, P, 1,
+                                 P, None, P, P, P, P, P, P, P, None) == qkn.ERR_INVALID_ARG
