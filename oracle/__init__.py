@@ -16,7 +16,7 @@ The GPU path never forms these keys; the pages state that the absorbed form is
 exactly equal to this one in exact arithmetic (technical summary,
 "Contribuciones Clave" item 1; arXiv abstract).
 
-Readings of points the pages leave open (each is listed in the design doc):
+Readings of points the pages leave open:
   * key RMS over the whole n_g*d_h output of W^K_g, one statistic per token
     and KV group (summary, Metodología item 2: one inverse-RMS scalar per
     token and KV group);

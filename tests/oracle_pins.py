@@ -100,6 +100,37 @@ def _absorbed_logits(inp, b):
     return out
 
 
+def check_absorbed_query_row_scale():
+    """The absorbed route's content logit a_q * a_k * (q~ . c_t), with q~ and a_q taken from
+    oracle.absorbed_query, equals sigma * RMSNorm(q) gamma_q . RMSNorm(c_t W^K_g)_h gamma_k with
+    the key materialised here (technical summary, Metodología, decode-logit equation: the row
+    scalar carries the query's inverse RMS over d_h and the softmax scale).  a_k comes from the
+    Gram identity, so no oracle helper enters the expected value."""
+    for wl in (TINY, TINY_MTP):
+        inp = make_inputs(wl)
+        ng, d_h = wl.heads // wl.groups, wl.d_h
+        sigma = 1.0 / math.sqrt(wl.d_h + wl.d_rope)
+        w = inp.w_k.astype(np.float64)
+        for b in range(wl.batch):
+            c = inp.c[inp.sequence(b)].astype(np.float64)
+            qt, a_q = oracle.absorbed_query(inp.q[b], inp.w_k, inp.gamma_q, inp.gamma_k, wl.eps, sigma)
+            assert a_q.shape == (wl.s_q, wl.heads)
+            for g in range(wl.groups):
+                gram = w[g] @ w[g].T
+                a_k = 1.0 / np.sqrt(np.einsum("ti,ij,tj->t", c, gram, c) / (ng * d_h) + wl.eps)
+                z = c @ w[g]                                           # materialised keys [L, n_g*d_h]
+                zn = z / np.sqrt((z * z).mean(-1, keepdims=True) + wl.eps)
+                for m in range(ng):
+                    h = g * ng + m
+                    key = zn[:, m * d_h:(m + 1) * d_h] * inp.gamma_k[h].astype(np.float64)
+                    for j in range(wl.s_q):
+                        qv = inp.q[b, j, h].astype(np.float64)
+                        qn = qv / math.sqrt(float(np.mean(qv * qv)) + wl.eps) * inp.gamma_q[h].astype(np.float64)
+                        expl = sigma * (key @ qn)
+                        absb = a_q[j, h] * a_k * (c @ qt[j, h])
+                        np.testing.assert_allclose(absb, expl, rtol=1e-10, atol=1e-12)
+
+
 def check_absorbed_logits_match():
     for wl in (TINY, TINY_MTP):
         inp = make_inputs(wl)
@@ -322,6 +353,7 @@ def check_permutation_invariance():
 
 ALL_CHECKS = [
     check_absorbed_query_exact,
+    check_absorbed_query_row_scale,
     check_absorbed_logits_match,
     check_key_inv_rms_gram,
     check_latent_scale_invariance,

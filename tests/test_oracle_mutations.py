@@ -27,6 +27,9 @@ MUTATIONS = {
     "key_rope_unnormalised": ("return rope(rms_norm(k_rope, gamma_kr, eps), pos, theta)",
                               "return rope(np.asarray(k_rope, np.float64) * gamma_kr, pos, theta)"),
     "values_normalised": ("return p @ c, lse", "return p @ (c / np.abs(c).max()), lse"),
+    "row_scale_without_sigma": ("a_q = softmax_scale * inv_rms(q, eps)", "a_q = inv_rms(q, eps)"),
+    "row_scale_half_width": ("a_q = softmax_scale * inv_rms(q, eps)",
+                             "a_q = softmax_scale * inv_rms(q[..., ::2], eps)"),
 }
 
 
