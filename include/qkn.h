@@ -85,7 +85,7 @@ typedef struct {
   int32_t d_rope;        /* RoPE dimension d_R (even) */
   int32_t block_size;    /* cache page size in tokens; must be 64 */
   float eps;             /* RMSNorm: S(z) = sqrt(mean(z^2) + eps), all four norms */
-  float softmax_scale;   /* sigma, applied to the whole logit (content + RoPE) */
+  float softmax_scale;   /* sigma, applied to the whole logit (content + RoPE); 0 = 1/sqrt(d_h + d_rope) */
   float rope_theta;      /* RoPE base; pairs (i, i + d_R/2), angle pos * theta^(-2i/d_R) */
   qkn_dtype dtype;
 } qkn_dims;
@@ -132,6 +132,12 @@ typedef struct {
                               table and streams the other cache pages while that kernel is still
                               running, and waits for it only before the queries and the pages that hold
                               new tokens.  0 (default): it waits before reading anything. */
+  int32_t test_withhold_ak;/* tests only: 1 makes the tcgen05 decode's producer skip the a_k copy of
+                              every CTA's first cache page, so that the softmax's bounded wait for it
+                              runs out: the decode records QKN_ERR_TIMEOUT, winds down (copies and
+                              MMAs in flight are waited for, tensor memory is freed) and the merge
+                              writes no partial it cannot vouch for.  It exercises the timeout path
+                              without faulting or hanging the GPU.  Ignored with QKN_AK_ONE.  0 in use. */
 } qkn_decode_opts;
 
 /* qkn_key_gram — G_g = W^K_g (W^K_g)^T for every group g, the r_kv x r_kv
@@ -264,8 +270,10 @@ QKN_EXPORT qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, q
  *   Arguments are those of qkn_decode without the workspace.  The split-KV
  *   partial results go to a fixed QKN_NOALLOC_SCRATCH_BYTES array inside the
  *   library instead; nothing is allocated and no allocating routine is called.
- *   device_status: optional DEVICE pointer to one int32; the decode's status
- *   word (a qkn_status) is copied there on `stream` after the decode.
+ *   device_status: optional DEVICE pointer to one int32; whenever the call
+ *   returns QKN_OK, the decode's status word (a qkn_status) is written there on
+ *   `stream` after the decode (QKN_OK for batch == 0).  When the call returns
+ *   an error it is not written: the return value is then the status.
  *   Returns QKN_ERR_UNSUPPORTED, before enqueuing anything, when the problem
  *   needs more scratch than QKN_NOALLOC_SCRATCH_BYTES (that is, when
  *   qkn_decode_workspace_size for these dims, batch and s_q exceeds it).

@@ -51,7 +51,7 @@ class _Cache(ctypes.Structure):
 class _Opts(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("max_ctas", ctypes.c_int32), ("head_tile", ctypes.c_int32),
                 ("wait_limit", ctypes.c_int64), ("split_event", ctypes.c_void_p),
-                ("step_writes_only", ctypes.c_int32)]
+                ("step_writes_only", ctypes.c_int32), ("test_withhold_ak", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -105,13 +105,13 @@ class Dims:
     d_h: int
     d_rope: int
     eps: float = 1e-6
-    softmax_scale: Optional[float] = None     # default 1/sqrt(d_h + d_rope)
+    softmax_scale: Optional[float] = None     # None: the library's default, 1/sqrt(d_h + d_rope)
     rope_theta: float = 10000.0
     dtype: int = BF16
     block_size: int = 64
 
     def c(self) -> _Dims:
-        scale = self.softmax_scale if self.softmax_scale is not None else (self.d_h + self.d_rope) ** -0.5
+        scale = self.softmax_scale if self.softmax_scale is not None else 0.0
         return _Dims(self.num_heads, self.num_groups, self.r_kv, self.d_h, self.d_rope, self.block_size,
                      self.eps, scale, self.rope_theta, self.dtype)
 
@@ -148,8 +148,9 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _opts(kernel=KERNEL_AUTO, max_ctas=0, head_tile=0, wait_limit=0, split_event=None, step_writes_only=0) -> _Opts:
-    return _Opts(kernel, max_ctas, head_tile, wait_limit, split_event, step_writes_only)
+def _opts(kernel=KERNEL_AUTO, max_ctas=0, head_tile=0, wait_limit=0, split_event=None, step_writes_only=0,
+          test_withhold_ak=0) -> _Opts:
+    return _Opts(kernel, max_ctas, head_tile, wait_limit, split_event, step_writes_only, test_withhold_ak)
 
 
 # ----------------------------------------------------------------- calls
@@ -207,12 +208,13 @@ def decode_kernel_for(dims: Dims, s_q: int, kernel=KERNEL_AUTO, head_tile=0) -> 
 def decode(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_lens, s_q: int,
            workspace: torch.Tensor, out, lse, ak_mode: int = AK_CACHE, kernel: int = KERNEL_AUTO,
            max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0, split_event=None, step_writes_only=False,
-           stream=None) -> None:
+           test_withhold_ak=False, stream=None) -> None:
     """One decode step over the cache (see qkn_decode).  ``split_event`` is a raw cudaEvent_t handle;
-    ``step_writes_only`` is the qkn_decode_opts promise of that name."""
+    ``step_writes_only`` and ``test_withhold_ak`` are the qkn_decode_opts fields of those names."""
     batch = int(block_table.shape[0])
     max_blocks = int(block_table.shape[1])
-    opts = _opts(kernel, max_ctas, head_tile, wait_limit, split_event, int(bool(step_writes_only)))
+    opts = _opts(kernel, max_ctas, head_tile, wait_limit, split_event, int(bool(step_writes_only)),
+                 int(bool(test_withhold_ak)))
     _check(_lib.qkn_decode(ctypes.byref(dims.c()), ctypes.byref(cache.c()), ak_mode, _ptr(q_tilde), _ptr(a_q),
                            _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens), batch, s_q,
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),

@@ -22,12 +22,9 @@ __global__ void __launch_bounds__(256) absorb_qtilde_kernel(const __grid_constan
 template <typename T>
 static cudaError_t launch_absorb_t(const AbsorbArgs& a, cudaStream_t st) {
   const size_t smem = absorb_smem_bytes(absorb_rows<8>(), a.d_h);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = set_smem_attrs(absorb_qtilde_kernel<T>, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [] { return set_smem_attrs(absorb_qtilde_kernel<T>, 200 * 1024); });
+  if (e != cudaSuccess) return e;
   dim3 grid(a.heads, (a.r + absorb_rows<8>() - 1) / absorb_rows<8>() + 1);
   return launch_chained(absorb_qtilde_kernel<T>, grid, dim3(256), smem, st, a);
 }

@@ -27,7 +27,7 @@ qkn_status check_dims(const qkn_dims* d) {
   if (d->d_rope <= 0 || d->d_rope > 128 || (d->d_rope % 2) ||
       (d->d_rope * elem_size(d->dtype)) % 16)
     return QKN_ERR_INVALID_ARG;
-  if (!(d->eps >= 0.f) || !(d->softmax_scale > 0.f) || !(d->rope_theta > 0.f)) return QKN_ERR_INVALID_ARG;
+  if (!(d->eps >= 0.f) || !(d->softmax_scale >= 0.f) || !(d->rope_theta > 0.f)) return QKN_ERR_INVALID_ARG;
   const int64_t width = (int64_t)(d->num_heads / d->num_groups) * d->d_h;
   if (width > (1 << 24)) return QKN_ERR_INVALID_ARG;
   return QKN_OK;
@@ -58,6 +58,12 @@ int sm_count(int* out) {
 }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// sigma: the caller's, or 1 / sqrt(d_h + d_R) when the caller passes 0 (the usual scale for a
+// logit whose dot products span the content and the RoPE block).
+float softmax_scale_of(const qkn_dims* d) {
+  return d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / sqrt((double)(d->d_h + d->d_rope)));
+}
 
 // RoPE pair frequencies theta^(-2i/d_R) in fp64 (constants of the dims).
 RopeFreqs rope_freqs(const qkn_dims* d) {
@@ -198,7 +204,7 @@ qkn_status absorb_args(const qkn_dims* dims, const void* q, const void* q_rope, 
   a->d_h = dims->d_h;
   a->d_rope = dims->d_rope;
   a->eps = dims->eps;
-  a->softmax_scale = dims->softmax_scale;
+  a->softmax_scale = softmax_scale_of(dims);
   a->rope_theta = dims->rope_theta;
   a->freq = rope_freqs(dims);
   return QKN_OK;
@@ -352,6 +358,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   a.lse = lse;
   a.seg_desc = reinterpret_cast<int2*>(ws + w.desc_off);
   a.step_writes_only = (opts && opts->step_writes_only) ? 1 : 0;
+  a.withhold_ak = (opts && opts->test_withhold_ak) ? 1 : 0;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const bool bf16 = dims->dtype == QKN_BF16;
@@ -374,6 +381,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   c.item_cost = a.item_cost;
   c.max_blocks = max_blocks;
   c.max_items = ncta + 1;
+  c.nslots = sched_slots(batch, a.ht_count, ncta);
   c.part_o = a.part_o;
   c.part_lse = a.part_lse;
   c.out = out;

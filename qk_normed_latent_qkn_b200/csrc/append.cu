@@ -56,12 +56,10 @@ __global__ void append_finalize_kernel(AppendArgs a) {
 template <typename T, int TT, bool FUSED>
 static cudaError_t launch_keyrms(const AppendArgs& a, cudaStream_t st) {
   const size_t smem = ((size_t)TT * a.r + (size_t)kRmsSlices * TT * kRmsCols) * sizeof(float);
-  static bool attr_set = false;   // one attribute per instantiation
-  if (!attr_set) {
-    cudaError_t e = set_smem_attrs(append_keyrms_kernel<T, TT, FUSED>, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attrs;   // one per instantiation
+  cudaError_t e =
+      once_per_device(attrs, [] { return set_smem_attrs(append_keyrms_kernel<T, TT, FUSED>, 200 * 1024); });
+  if (e != cudaSuccess) return e;
   const int nblk = (a.ncols + kRmsCols - 1) / kRmsCols;
   dim3 grid(nblk + (FUSED ? 1 : 0), (a.n_tok + TT - 1) / TT, a.groups);
   return launch_chained(append_keyrms_kernel<T, TT, FUSED>, grid, dim3(kRmsCols * kRmsSlices), smem, st, a);

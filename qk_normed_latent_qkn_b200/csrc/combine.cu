@@ -53,6 +53,17 @@ __global__ void __launch_bounds__(kCombThreads, kDesc ? 12 : 8) combine_kernel(C
     const int2 d = a.seg_desc[seg];
     // a sequence with a rejected length has no splits: the tcgen05 kernel wrote its rows itself
     if (d.y <= 0) return;
+    // A decode that stopped early (a bounded wait ran out) leaves some descriptors unwritten, i.e.
+    // holding a previous call's values or nothing meaningful.  Every descriptor is checked against
+    // this launch's slots before a partial is read; a bad one gives zero rows, lse = -inf.
+    if (d.x < 0 || d.y > a.max_items || (int64_t)d.x + (int64_t)(d.y - 1) * a.ht_count >= a.nslots) {
+      if (threadIdx.x == 0) record_status(a.status, QKN_ERR_BOUNDS);
+      const int64_t orow = (int64_t)b * qrows + rho;
+      T* out = static_cast<T*>(a.out) + orow * a.r;
+      for (int v = threadIdx.x; v < a.r / 4; v += kCombThreads) store4<T>(out + v * 4, make_float4(0.f, 0.f, 0.f, 0.f));
+      if (threadIdx.x == 0) a.lse[orow] = -INFINITY;
+      return;
+    }
     first = (int64_t)d.x * a.rows + row;
     nitems = d.y;
   } else {

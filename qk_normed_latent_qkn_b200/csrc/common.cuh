@@ -8,6 +8,7 @@
 
 #include <utility>
 
+#include "per_device.h"
 #include "qkn.h"
 
 namespace qkn {
@@ -59,6 +60,16 @@ inline cudaError_t set_smem_attrs(void (*kernel)(KArgs...), int max_dynamic_byte
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                               (int)cudaSharedmemCarveoutMaxShared);
+}
+
+// Run a kernel's one-time attribute set-up on the current device: attributes
+// are per device, so each device of the process gets its own (per_device.h).
+template <typename F>
+inline cudaError_t once_per_device(PerDeviceOnce& once, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  return once.run(dev, cudaSuccess, std::forward<F>(setup));
 }
 
 // ---------------------------------------------------------------- RoPE

@@ -52,11 +52,15 @@ extern "C" qkn_status qkn_decode_noalloc(const qkn_dims* dims, const qkn_cache* 
   qkn_status st = qkn_decode_workspace_size(dims, batch, s_q, 0, &need);
   if (st != QKN_OK) return st;
   if (need > (size_t)QKN_NOALLOC_SCRATCH_BYTES) return QKN_ERR_UNSUPPORTED;
-  if (batch == 0) return QKN_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (batch == 0) {
+    // nothing to decode: the status the caller reads is QKN_OK (zero), written on the stream
+    if (device_status && cudaMemsetAsync(device_status, 0, sizeof(int32_t), cs) != cudaSuccess) return QKN_ERR_CUDA;
+    return QKN_OK;
+  }
 
   void* scratch = scratch_for_current_device();
   if (!scratch) return QKN_ERR_CUDA;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // The array keeps whatever the previous call left in it; only the status
   // word has to start from zero (everything else is written before it is read).
   if (cudaMemsetAsync(scratch, 0, qkn::kStatusBytes, cs) != cudaSuccess) return QKN_ERR_CUDA;

@@ -155,12 +155,9 @@ template <typename T, int NK>
 static cudaError_t launch_simt_nk(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)kBlockSize * (a.r + a.d_rope) * sizeof(T) +
                       (size_t)kBlockSize * a.groups * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = set_smem_attrs(decode_simt_kernel<T, NK>, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [] { return set_smem_attrs(decode_simt_kernel<T, NK>, 200 * 1024); });
+  if (e != cudaSuccess) return e;
   return launch_chained(decode_simt_kernel<T, NK>, dim3(a.ncta), dim3(kSimtRows * 32), smem, st, a);
 }
 

@@ -45,6 +45,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -277,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     const uint32_t akpage = (uint32_t)kPage * (uint32_t)G * 4u;
     bool waited = !a.step_writes_only;
     int early_pages = 0;                  // pages issued before the first query tile
+    int q_last = -1;                      // item whose query tile was issued last
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
       const int32_t* row = a.block_table + (int64_t)it.b * a.max_blocks;
       // the first 32 block-table entries of the item are read before the query tile is issued, so
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         for (int k = 0; k < kChunks; ++k) tma_load_2d_elect(sb + C::Q_OFF + k * R * 128, &maps.qt, k * 64, qrow0, qf);
         tma_load_2d_elect(sb + C::QR_OFF, &maps.qr, 0, qrow0, qf);
         q_pending = false;
+        q_last = n_item;
         return true;
       };
       if (waited && !issue_q()) { ok = false; break; }
@@ -333,7 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           const uint32_t kb = smem_u32(&ms.krfull[kw.slot]);
           mbar_arrive_expect_tx_elect(kb, kKrBytes);
           tma_load_2d_elect(sb + C::KR_OFF + kw.slot * kKrBytes, &maps.krope, 0, blk * kPage, kb);
-          if (!AK_ONE) {
+          // (a test of the timeout path withholds the first page's a_k copy: nothing else completes
+          // that barrier phase, so the softmax's bounded wait for it runs out)
+          if (!AK_ONE && !(a.withhold_ak && k_issued == 0)) {
             const uint32_t akb = smem_u32(&ms.akfull[kw.slot]);
             mbar_arrive_expect_tx_elect(akb, akpage);
             bulk_load_elect(sb + C::AK_OFF + kw.slot * kAkSlotBytes, a.a_k + (int64_t)blk * kPage * G, akpage, akb);
@@ -356,8 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       const int64_t kfirst = k_issued > NKR ? k_issued - NKR : 0;
       for (int64_t i = kfirst; i < k_issued; ++i) {
         mbar_wait(smem_u32(&ms.krfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
-        if (!AK_ONE) mbar_wait(smem_u32(&ms.akfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
+        if (!AK_ONE && !(a.withhold_ak && i == 0))
+          mbar_wait(smem_u32(&ms.akfull[i % NKR]), (i / NKR) & 1, kDrainLimit);
       }
+      // and the last query tile (the one before it was complete when its q_empty wait returned)
+      if (q_last >= 0) mbar_wait(smem_u32(&ms.q_full), (uint32_t)(q_last & 1), kDrainLimit);
     }
   } else if (warp == kScoreWarp) {
     // ------------------------------------------------------------ score MMA issuer (whole warp)
@@ -832,15 +841,61 @@ bool make_latent_map(CUtensorMap* m, const void* base, uint64_t rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Encoded tensor maps, cached by what they encode (base address, extents and box), so that an
+// eager decode does not pay four host-side encodings per call.  A map holds only an address and a
+// geometry, so an entry stays valid for any buffer later placed at the same address with the same
+// extents.  A small table with least-recently-used replacement, under a mutex.
+class TmapCache {
+ public:
+  template <typename Encode>
+  bool get(const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows, int kind, CUtensorMap* out,
+           Encode&& encode) {
+    std::lock_guard<std::mutex> lock(mu_);
+    ++tick_;
+    int victim = 0;
+    for (int i = 0; i < kEntries; ++i) {
+      Entry& e = e_[i];
+      if (e.used && e.base == base && e.inner == inner && e.rows == rows && e.box_rows == box_rows &&
+          e.kind == kind) {
+        e.used = tick_;
+        *out = e.map;
+        return true;
+      }
+      if (e.used < e_[victim].used) victim = i;
+    }
+    if (!encode(out)) return false;
+    e_[victim] = Entry{base, inner, rows, box_rows, kind, tick_, *out};
+    return true;
+  }
+
+ private:
+  static constexpr int kEntries = 32;
+  struct Entry {
+    const void* base;
+    uint64_t inner, rows;
+    uint32_t box_rows;
+    int kind;
+    uint64_t used;   // 0: empty
+    CUtensorMap map;
+  };
+  std::mutex mu_;
+  uint64_t tick_ = 0;
+  Entry e_[kEntries] = {};
+};
+
+TmapCache& tmap_cache() {
+  static TmapCache c;
+  return c;
+}
+
 template <int R, bool AK_ONE>
 cudaError_t launch_tc(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<R, AK_ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<R>::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [] {
+    return cudaFuncSetAttribute(decode_tc_kernel<R, AK_ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<R>::SMEM);
+  });
+  if (e != cudaSuccess) return e;
   return launch_chained(decode_tc_kernel<R, AK_ONE>, dim3(a.ncta), dim3(kThreads), Cfg<R>::SMEM, st, a, maps);
 }
 
@@ -856,10 +911,15 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   TcMaps maps;
   const uint64_t cache_rows = (uint64_t)a.num_blocks * 64;
   const uint64_t q_rows = (uint64_t)a.batch * a.s_q * a.heads;
-  if (!make_latent_map(&maps.latent, a.latent, cache_rows) ||
-      !make_map(&maps.krope, a.k_rope, kDrope, cache_rows, 64, 64) ||
-      !make_map(&maps.qt, a.q_tilde, kRkv, q_rows, 64, a.rows) ||
-      !make_map(&maps.qr, a.q_rope_hat, kDrope, q_rows, 64, a.rows))
+  TmapCache& tc = tmap_cache();
+  if (!tc.get(a.latent, kRkv, cache_rows, 64, 0, &maps.latent,
+              [&](CUtensorMap* m) { return make_latent_map(m, a.latent, cache_rows); }) ||
+      !tc.get(a.k_rope, kDrope, cache_rows, 64, 1, &maps.krope,
+              [&](CUtensorMap* m) { return make_map(m, a.k_rope, kDrope, cache_rows, 64, 64); }) ||
+      !tc.get(a.q_tilde, kRkv, q_rows, a.rows, 1, &maps.qt,
+              [&](CUtensorMap* m) { return make_map(m, a.q_tilde, kRkv, q_rows, 64, a.rows); }) ||
+      !tc.get(a.q_rope_hat, kDrope, q_rows, a.rows, 1, &maps.qr,
+              [&](CUtensorMap* m) { return make_map(m, a.q_rope_hat, kDrope, q_rows, 64, a.rows); }))
     return cudaErrorInvalidValue;
   switch (a.rows * 2 + (a.ak_one ? 1 : 0)) {
     case 32: return launch_tc<16, false>(a, maps, st);

@@ -77,6 +77,7 @@ struct DecodeArgs {
   float* lse;                // [batch, s_q, H]
   int2* seg_desc;            // [batch * ht_count]
   int32_t step_writes_only;  // qkn_decode_opts.step_writes_only: read inputs and old pages before the wait
+  int32_t withhold_ak;       // qkn_decode_opts.test_withhold_ak (tests of the timeout path)
 };
 
 struct CombineArgs {
@@ -84,6 +85,7 @@ struct CombineArgs {
   int32_t batch, s_q, heads, r, rows, ht_count, ncta, max_blocks;
   int32_t item_cost;         // as in DecodeArgs
   int32_t max_items;         // upper bound on splits per row (ncta + 1)
+  int64_t nslots;            // workspace slots of this launch (batch * ht_count + ncta), each `rows` rows
   const float* part_o;
   const float* part_lse;
   void* out;                 // [batch, s_q, H, r]

@@ -61,12 +61,9 @@ cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, c
   const size_t smem_absorb = absorb_smem_bytes(kAbsRows, ab.d_h);
   const size_t smem = smem_append > smem_absorb ? smem_append : smem_absorb;
   auto kernel = bf16 ? prep_kernel<__nv_bfloat16> : prep_kernel<float>;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[bf16 ? 1 : 0]) {
-    cudaError_t e = set_smem_attrs(kernel, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set[bf16 ? 1 : 0] = true;
-  }
+  static PerDeviceOnce attrs[2];
+  cudaError_t e = once_per_device(attrs[bf16 ? 1 : 0], [&] { return set_smem_attrs(kernel, 200 * 1024); });
+  if (e != cudaSuccess) return e;
   return launch_chained(kernel, dim3((unsigned)ctas), dim3(kPrepThreads), smem, st, p);
 }
 

@@ -49,7 +49,7 @@ def test_workspace_size_host_only():
 
 @pytest.mark.parametrize("bad", [
     dict(num_heads=0), dict(num_groups=3), dict(r_kv=12), dict(d_rope=7), dict(d_rope=256),
-    dict(block_size=32), dict(eps=-1.0), dict(softmax_scale=0.0), dict(dtype=7),
+    dict(block_size=32), dict(eps=-1.0), dict(softmax_scale=-1.0), dict(dtype=7),
 ])
 def test_bad_dims_rejected(bad):
     import dataclasses
@@ -57,6 +57,14 @@ def test_bad_dims_rejected(bad):
     with pytest.raises(qkn.QknError) as e:
         _ws(d)
     assert e.value.status == qkn.ERR_INVALID_ARG
+
+
+def test_default_softmax_scale_is_accepted():
+    """softmax_scale = 0 asks the library for its default, 1/sqrt(d_h + d_rope); the binding passes 0
+    when Dims.softmax_scale is None."""
+    import dataclasses
+    assert DIMS.softmax_scale is None and DIMS.c().softmax_scale == 0.0
+    assert _ws(dataclasses.replace(DIMS, softmax_scale=0.0)) == _ws(DIMS)
 
 
 def test_decode_rejects_null_pointers_before_any_launch():

@@ -76,3 +76,17 @@ def test_noalloc_rejects_a_problem_larger_than_its_scratch():
                                 s.q_tilde.data_ptr(), s.a_q.data_ptr(), s.q_rope_hat.data_ptr(), 0x100, 1, 0x100,
                                 big_batch, 1, 0x100, 0x100, None, None, torch.cuda.current_stream().cuda_stream)
     assert rc == qkn.ERR_UNSUPPORTED
+
+
+def test_noalloc_with_nothing_to_decode_reports_ok():
+    """batch == 0 decodes nothing, returns QKN_OK and writes QKN_OK to the caller's status word."""
+    inp = make_inputs(CASES["small_mla_bf16"])
+    s = session_from_inputs(inp)
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    lib = qkn.raw_library()
+    rc = lib.qkn_decode_noalloc(ctypes.byref(s.dims.c()), ctypes.byref(s.cache.c()), qkn.AK_CACHE,
+                                s.q_tilde.data_ptr(), s.a_q.data_ptr(), s.q_rope_hat.data_ptr(), 0x100, 1, 0x100,
+                                0, 1, 0x100, 0x100, status.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == qkn.OK
+    assert int(status.item()) == qkn.OK
