@@ -117,8 +117,11 @@ typedef struct {
 /* Optional decode knobs (pass NULL for defaults). */
 typedef struct {
   qkn_kernel kernel;       /* default QKN_KERNEL_AUTO */
-  int32_t max_ctas;        /* cap on decode CTAs (split-KV width); 0 = one per SM */
-  int32_t head_tile;       /* tcgen05: query rows per CTA (16, 32 or 64); 0 = automatic */
+  int32_t max_ctas;        /* cap on decode CTAs (split-KV width; CTA pairs take max_ctas / 2);
+                              0 = one per SM */
+  int32_t head_tile;       /* tcgen05: query rows per tile (16, 32 or 64 on one CTA; 128 on a pair of
+                              CTAs that split the latent width); 0 = automatic (128 when a sequence
+                              has more than 64 query rows) */
   int64_t wait_limit;      /* bounded-wait limit in clock cycles for the mbarrier waits; 0 = default (~2 s) */
   void* split_event;       /* optional cudaEvent_t recorded between the split-KV kernel and the combine
                               kernel (external record, so it also works inside stream capture) */

@@ -72,20 +72,28 @@ RopeFreqs rope_freqs(const qkn_dims* d) {
   return r;
 }
 
-// Rows per tile for the tcgen05 kernel: the smallest supported tile that
-// covers the per-sequence query rows, capped at 64 (the accumulator of a
-// 64-row tile already fills the tensor memory of one SM).
+// Rows per tile for the tcgen05 kernels: the smallest supported tile that
+// covers the per-sequence query rows.  Up to 64 rows one CTA takes a tile
+// (the fp32 accumulator of a 64-row tile already fills an SM's tensor
+// memory); above that, tiles of 128 rows go to CTA pairs that split the
+// latent width, so that every MMA has 128 rows.
 int tc_rows(const qkn_dims* d, int s_q, const qkn_decode_opts* o) {
   if (o && o->head_tile) return o->head_tile;
   const int qrows = s_q * d->num_heads;
   if (qrows <= 16) return 16;
   if (qrows <= 32) return 32;
-  return 64;
+  if (qrows <= 64 || !decode_pair_supported(d->r_kv, d->d_rope, d->num_groups)) return 64;
+  return kPairRows;
+}
+
+bool tc_supported(const qkn_dims* d, int rows) {
+  if (rows == kPairRows) return decode_pair_supported(d->r_kv, d->d_rope, d->num_groups);
+  return decode_tc_supported(d->r_kv, d->d_rope, rows, d->num_groups);
 }
 
 int pick_kernel(const qkn_dims* d, int s_q, const qkn_decode_opts* o) {
   const qkn_kernel want = o ? o->kernel : QKN_KERNEL_AUTO;
-  const bool tc_ok = d->dtype == QKN_BF16 && decode_tc_supported(d->r_kv, d->d_rope, tc_rows(d, s_q, o), d->num_groups);
+  const bool tc_ok = d->dtype == QKN_BF16 && tc_supported(d, tc_rows(d, s_q, o));
   if (want == QKN_KERNEL_SIMT) return QKN_KERNEL_SIMT;
   if (want == QKN_KERNEL_TCGEN05) return tc_ok ? QKN_KERNEL_TCGEN05 : -1;
   if (want != QKN_KERNEL_AUTO) return -1;
@@ -101,9 +109,10 @@ WsLayout ws_layout(const qkn_dims* d, int batch, int s_q, int ncta) {
   // serves every kernel choice.
   int64_t slot_rows = 0, segments = 0;
   const int qrows = s_q * d->num_heads;
-  for (int rows : {kSimtRows, 16, 32, 64}) {
+  for (int rows : {kSimtRows, 16, 32, 64, kPairRows}) {
     const int64_t ht = ceil_div(qrows, rows);
-    const int64_t sr = sched_slots(batch, ht, ncta) * rows;
+    // the CTA-pair kernel's schedule counts pairs: at most half the CTAs
+    const int64_t sr = sched_slots(batch, ht, rows == kPairRows ? ncta / 2 : ncta) * rows;
     if (sr > slot_rows) slot_rows = sr;
     if (batch * ht > segments) segments = batch * ht;
   }
@@ -313,7 +322,8 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   if (!aligned(q_tilde, 16) || !aligned(q_rope_hat, 16) || !aligned(workspace, 256) || !aligned(out, 16))
     return QKN_ERR_INVALID_ARG;
   if (opts && (opts->max_ctas < 0 || opts->wait_limit < 0 ||
-               (opts->head_tile && opts->head_tile != 16 && opts->head_tile != 32 && opts->head_tile != 64)))
+               (opts->head_tile && opts->head_tile != 16 && opts->head_tile != 32 && opts->head_tile != 64 &&
+                opts->head_tile != kPairRows)))
     return QKN_ERR_INVALID_ARG;
   const int kernel = pick_kernel(dims, s_q, opts);
   if (kernel < 0) return QKN_ERR_UNSUPPORTED;
@@ -324,6 +334,13 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   if (ws_bytes < w.total) return QKN_ERR_INVALID_ARG;
   int ncta = nsm;
   if (opts && opts->max_ctas > 0 && opts->max_ctas < ncta) ncta = opts->max_ctas;
+  const bool pair = kernel == QKN_KERNEL_TCGEN05 && tc_rows(dims, s_q, opts) == kPairRows;
+  if (pair) {
+    // the schedule's unit is a CTA pair: as many as fit at once, within the CTA cap
+    const int most = decode_pair_max_pairs(nsm);
+    ncta = ncta / 2 < most ? ncta / 2 : most;
+    if (ncta < 1) ncta = 1;
+  }
 
   char* ws = static_cast<char*>(workspace);
   DecodeArgs a;
@@ -349,7 +366,7 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   a.ncta = ncta;
   // starting an item costs about one page of time per 16 query rows of the tile (query tile,
   // pipeline refill, the previous item's epilogue), measured on the tcgen05 kernel
-  a.item_cost = kernel == QKN_KERNEL_TCGEN05 ? (a.rows == 64 ? 3 : a.rows / 16) : 1;
+  a.item_cost = kernel == QKN_KERNEL_TCGEN05 ? (a.rows >= 64 ? 3 : a.rows / 16) : 1;
   a.part_lse = reinterpret_cast<float*>(ws + w.lse_off);
   a.part_o = reinterpret_cast<float*>(ws + w.o_off);
   a.status = reinterpret_cast<int32_t*>(ws);
@@ -362,7 +379,8 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const bool bf16 = dims->dtype == QKN_BF16;
-  cudaError_t e = kernel == QKN_KERNEL_TCGEN05 ? launch_decode_tc(a, cs) : launch_decode_simt(a, bf16, cs);
+  cudaError_t e = pair ? launch_decode_pair(a, cs)
+                  : kernel == QKN_KERNEL_TCGEN05 ? launch_decode_tc(a, cs) : launch_decode_simt(a, bf16, cs);
   if (e != cudaSuccess) return QKN_ERR_CUDA;
   if (opts && opts->split_event &&
       cudaEventRecordWithFlags(static_cast<cudaEvent_t>(opts->split_event), cs, cudaEventRecordExternal) !=

@@ -3,12 +3,12 @@
 // log-sum-exp lse_s; the row's result is
 //   lse = log sum_s exp(lse_s),   o = sum_s exp(lse_s - lse) * o_s,
 // which is exactly the softmax over the union of the splits' tokens.
-// One CTA per query row.  Every thread owns 16 bytes of the row and merges
-// the splits for them on its own: it loads the splits' lse values together
-// with its 16 bytes of their partials, four splits at a time, and keeps a
-// running maximum.  After the segment descriptor, one round of memory latency
-// per four splits; no shared memory and no barrier (few registers, so that
-// many rows are in flight at once).
+// One CTA per four query rows of a segment.  Every thread owns the same 16
+// bytes of each row and merges the splits for them on its own: it loads the
+// splits' lse values together with its 16 bytes of their partials, two
+// splits of all four rows at a time, and keeps a running maximum per row.
+// After the segment descriptor, one round of memory latency per two splits;
+// no shared memory and no barrier.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,21 +32,27 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4
 }
 
 // kDesc: the splits come from the segment descriptors the tcgen05 decode wrote; else from the
-// schedule, recomputed (one instantiation each keeps the descriptor path small)
-template <typename T, bool kDesc>
-__global__ void __launch_bounds__(kCombThreads, kDesc ? 12 : 8) combine_kernel(CombineArgs a) {
+// schedule, recomputed (one instantiation each keeps the descriptor path small).  RPC: query rows
+// per CTA; every thread owns the same 16 bytes of each of them, and the rows' loads are issued
+// together, so that a CTA keeps RPC times as many loads in flight and the grid fits in fewer waves.
+// The RPC rows of a CTA lie in one segment (RPC divides the tile's row count).
+template <typename T, bool kDesc, int RPC>
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   __shared__ int64_t first_s;
   __shared__ int nitems_s;
   pdl_trigger();
   pdl_wait();
-  const int grow = blockIdx.x;                            // (segment, row)
-  const int seg = grow / a.rows, row = grow - seg * a.rows;
+  const int grow0 = blockIdx.x * RPC;                     // first (segment, row) of this CTA
+  const int seg = grow0 / a.rows, row0 = grow0 - seg * a.rows;
   const int b = seg / a.ht_count, ht = seg - b * a.ht_count;
   const int qrows = a.s_q * a.heads;
-  const int rho = ht * a.rows + row;
-  if (b >= a.batch || rho >= qrows) return;
-  // the row's splits: from the segment descriptor the tcgen05 decode wrote, else from the
-  // schedule, recomputed by warp 0
+  const int rho0 = ht * a.rows + row0;
+  if (b >= a.batch || rho0 >= qrows) return;
+  const int nrows = min(RPC, qrows - rho0);               // rows of this CTA inside the sequence
+  const int64_t orow0 = (int64_t)b * qrows + rho0;
+  const int nvec = a.r / 4;
+  // the splits of the segment: from the descriptor the tcgen05 decode wrote, else from the
+  // schedule, recomputed by warp 0.  first: partial row of row0 in the first split.
   int64_t first;
   int nitems;
   if constexpr (kDesc) {
@@ -58,13 +64,14 @@ __global__ void __launch_bounds__(kCombThreads, kDesc ? 12 : 8) combine_kernel(C
     // this launch's slots before a partial is read; a bad one gives zero rows, lse = -inf.
     if (d.x < 0 || d.y > a.max_items || (int64_t)d.x + (int64_t)(d.y - 1) * a.ht_count >= a.nslots) {
       if (threadIdx.x == 0) record_status(a.status, QKN_ERR_BOUNDS);
-      const int64_t orow = (int64_t)b * qrows + rho;
-      T* out = static_cast<T*>(a.out) + orow * a.r;
-      for (int v = threadIdx.x; v < a.r / 4; v += kCombThreads) store4<T>(out + v * 4, make_float4(0.f, 0.f, 0.f, 0.f));
-      if (threadIdx.x == 0) a.lse[orow] = -INFINITY;
+      for (int i = 0; i < nrows; ++i) {
+        T* out = static_cast<T*>(a.out) + (orow0 + i) * a.r;
+        for (int v = threadIdx.x; v < nvec; v += kCombThreads) store4<T>(out + v * 4, make_float4(0.f, 0.f, 0.f, 0.f));
+        if (threadIdx.x == 0) a.lse[orow0 + i] = -INFINITY;
+      }
       return;
     }
-    first = (int64_t)d.x * a.rows + row;
+    first = (int64_t)d.x * a.rows + row0;
     nitems = d.y;
   } else {
     if (threadIdx.x < 32) {
@@ -72,76 +79,100 @@ __global__ void __launch_bounds__(kCombThreads, kDesc ? 12 : 8) combine_kernel(C
       SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost};
       const int64_t total = sched_total_units(sp);
       const int32_t n = pages_of(a.seq_lens[b], sp);
-      if (n == 0 && ht == 0 && row == 0 && lane == 0) record_status(a.status, QKN_ERR_BOUNDS);
+      if (n == 0 && ht == 0 && row0 == 0 && lane == 0) record_status(a.status, QKN_ERR_BOUNDS);
       const int32_t ng = sched_groups(sp);
       const int64_t q = total > 0 ? (total + ng - 1) / ng : 1;
       const SegSplit sg = seg_split(sched_units_before(sp, b), n, q, sp.item_cost);
       if (lane == 0) {
         nitems_s = n > 0 ? sg.nitems : 0;
-        first_s = ((int64_t)(b + sg.c0) * a.ht_count + ht) * a.rows + row;   // partial row of the first split
+        first_s = ((int64_t)(b + sg.c0) * a.ht_count + ht) * a.rows + row0;
       }
     }
     __syncthreads();
     first = first_s;
     nitems = nitems_s;
   }
-  // Every thread owns 16 bytes of the row and merges the splits on its own, with a running
-  // maximum of their lse values: acc = sum_s exp(lse_s - m) o_s, den = sum_s exp(lse_s - m).
-  // The lse values and the partials of kDepth splits are loaded together.
-  constexpr int kDepth = 4;
-  const int nvec = a.r / 4;
+  // Every thread owns 16 bytes of each row and merges the splits for them on its own, with a
+  // running maximum of their lse values: acc = sum_s exp(lse_s - m) o_s, den = sum_s exp(lse_s - m).
+  // The lse values and the partials of kDepth splits of all the CTA's rows are loaded together.
+  constexpr int kDepth = 2;
   // consecutive splits of a segment sit ht_count slots apart
   const int64_t lstride = (int64_t)a.rows * a.ht_count;
-  const int64_t stride = lstride * a.r / 4;                 // float4s between consecutive splits of this row
+  const int64_t stride = lstride * a.r / 4;                 // float4s between consecutive splits of a row
   const float4* src0 = reinterpret_cast<const float4*>(a.part_o + first * a.r);
   const float* lsrc = a.part_lse + first;
-  const int64_t orow = (int64_t)b * qrows + rho;
-  T* out = static_cast<T*>(a.out) + orow * a.r;
   for (int v = threadIdx.x; v < nvec; v += kCombThreads) {
-    float m = -INFINITY, den = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < nitems; c += kDepth) {
-      float ls[kDepth];
-      float4 x[kDepth];
+    float m[RPC], den[RPC];
+    float4 acc[RPC];
 #pragma unroll
-      for (int u = 0; u < kDepth; ++u) {
-        const bool in = c + u < nitems;
-        ls[u] = in ? lsrc[(int64_t)(c + u) * lstride] : -INFINITY;
-        x[u] = in ? src0[(int64_t)(c + u) * stride + v] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float mc = m;
-#pragma unroll
-      for (int u = 0; u < kDepth; ++u) mc = fmaxf(mc, ls[u]);
-      if (mc == -INFINITY) continue;                    // nothing visible so far
-      const float sc = __expf(m - mc);                  // m == -inf gives 0
-      acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
-      den *= sc;
-#pragma unroll
-      for (int u = 0; u < kDepth; ++u) {
-        const float w = __expf(ls[u] - mc);             // ls == -inf gives 0
-        den += w;
-        acc.x = fmaf(w, x[u].x, acc.x);
-        acc.y = fmaf(w, x[u].y, acc.y);
-        acc.z = fmaf(w, x[u].z, acc.z);
-        acc.w = fmaf(w, x[u].w, acc.w);
-      }
-      m = mc;
+    for (int i = 0; i < RPC; ++i) {
+      m[i] = -INFINITY;
+      den[i] = 0.f;
+      acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    store4<T>(out + v * 4, make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
-    if (v == 0) a.lse[orow] = den > 0.f ? m + logf(den) : -INFINITY;
+    for (int c = 0; c < nitems; c += kDepth) {
+      float ls[RPC][kDepth];
+      float4 x[RPC][kDepth];
+#pragma unroll
+      for (int u = 0; u < kDepth; ++u) {
+#pragma unroll
+        for (int i = 0; i < RPC; ++i) {
+          const bool in = c + u < nitems && i < nrows;
+          ls[i][u] = in ? lsrc[(int64_t)(c + u) * lstride + i] : -INFINITY;
+          x[i][u] = in ? src0[(int64_t)(c + u) * stride + (int64_t)i * nvec + v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < RPC; ++i) {
+        float mc = m[i];
+#pragma unroll
+        for (int u = 0; u < kDepth; ++u) mc = fmaxf(mc, ls[i][u]);
+        if (mc == -INFINITY) continue;                  // nothing visible so far
+        const float sc = __expf(m[i] - mc);             // m == -inf gives 0
+        acc[i].x *= sc; acc[i].y *= sc; acc[i].z *= sc; acc[i].w *= sc;
+        den[i] *= sc;
+#pragma unroll
+        for (int u = 0; u < kDepth; ++u) {
+          const float w = __expf(ls[i][u] - mc);        // ls == -inf gives 0
+          den[i] += w;
+          acc[i].x = fmaf(w, x[i][u].x, acc[i].x);
+          acc[i].y = fmaf(w, x[i][u].y, acc[i].y);
+          acc[i].z = fmaf(w, x[i][u].z, acc[i].z);
+          acc[i].w = fmaf(w, x[i][u].w, acc[i].w);
+        }
+        m[i] = mc;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < RPC; ++i) {
+      if (i >= nrows) break;
+      const float inv = den[i] > 0.f ? 1.f / den[i] : 0.f;
+      T* out = static_cast<T*>(a.out) + (orow0 + i) * a.r;
+      store4<T>(out + v * 4, make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv));
+      if (v == 0) a.lse[orow0 + i] = den[i] > 0.f ? m[i] + logf(den[i]) : -INFINITY;
+    }
   }
 }
 
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st) {
+  // rows per CTA: four when the tile's row count allows it (every tile size but odd ones)
   const int64_t rows = (int64_t)a.batch * a.ht_count * a.rows;
   const size_t smem = 0;
-  const dim3 grid((unsigned)rows), block(kCombThreads);
+  const dim3 block(kCombThreads);
+  if (a.rows % 4 == 0) {
+    const dim3 grid((unsigned)(rows / 4));
+    if (a.seg_desc)
+      return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, true, 4>, grid, block, smem, st, a)
+                  : launch_chained(combine_kernel<float, true, 4>, grid, block, smem, st, a);
+    return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, false, 4>, grid, block, smem, st, a)
+                : launch_chained(combine_kernel<float, false, 4>, grid, block, smem, st, a);
+  }
+  const dim3 grid((unsigned)rows);
   if (a.seg_desc)
-    return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, true>, grid, block, smem, st, a)
-                : launch_chained(combine_kernel<float, true>, grid, block, smem, st, a);
-  return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, false>, grid, block, smem, st, a)
-              : launch_chained(combine_kernel<float, false>, grid, block, smem, st, a);
+    return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, true, 1>, grid, block, smem, st, a)
+                : launch_chained(combine_kernel<float, true, 1>, grid, block, smem, st, a);
+  return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, false, 1>, grid, block, smem, st, a)
+              : launch_chained(combine_kernel<float, false, 1>, grid, block, smem, st, a);
 }
 
 }  // namespace qkn

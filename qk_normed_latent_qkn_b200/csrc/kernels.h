@@ -108,6 +108,13 @@ cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st);
 bool decode_tc_supported(int r, int d_rope, int rows, int groups);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
+// tcgen05 decode of 128-row tiles on CTA pairs that split the latent width (decode_pair.cu);
+// DecodeArgs.ncta counts pairs there.  Returns cudaErrorNotSupported for dims it cannot take.
+bool decode_pair_supported(int r, int d_rope, int groups);
+int decode_pair_max_pairs(int sms);    // pairs resident at once on the current device (<= sms / 2)
+cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st);
+
 constexpr int kSimtRows = 8;   // query rows per CTA of the CUDA-core decode
+constexpr int kPairRows = 128; // query rows per tile of the CTA-pair decode
 
 }  // namespace qkn
