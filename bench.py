@@ -52,6 +52,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="large_mla_bf16")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--kernel", choices=["auto", "simt", "tcgen05"], default="auto")
+    p.add_argument("--head-tile", type=int, default=0, choices=[0, 16, 32, 64, 128],
+                   help="query rows per tcgen05 tile (128: the CTA-pair kernel); 0 = automatic")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--soak-seconds", type=float, default=1.0, help="load window around the timed steps for clocks")
@@ -326,7 +328,7 @@ def run_ours(args, world, rank, local):
             evs.wait_stream(main)
             ev.record(start_event, evs.cuda_stream)
         s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event,
-                 step_writes_only=True)
+                 step_writes_only=True, head_tile=args.head_tile)
         if end_event is not None:
             ev.record(end_event, main.cuda_stream)
         if start_event is not None:
@@ -334,7 +336,8 @@ def run_ours(args, world, rank, local):
 
     def decode_only(i, split_event=None, ak_mode=qkn.AK_CACHE):
         s, d, (o, l) = sessions[i], dev_in[i], outs[i]
-        s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event)
+        s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event,
+                 head_tile=args.head_tile)
 
     ev = Events()
     stream = torch.cuda.Stream(device=device)
@@ -346,7 +349,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(device)
     status = [s.device_status() for s in sessions]
     assert all(v == qkn.OK for v in status), f"device status {status}"
-    kernel_used = qkn.decode_kernel_for(base.dims, s_q, kernel=kernel)
+    kernel_used = qkn.decode_kernel_for(base.dims, s_q, kernel=kernel, head_tile=args.head_tile)
 
     total = args.warmup + args.steps
     graphs, marks = [], []
@@ -460,7 +463,8 @@ def run_ours(args, world, rank, local):
              "bt": "block_table", "sl": "seq_lens"}
     steps = []
     for i in range(n_copies):
-        st = DecodeStep(sessions[i], B, s_q, inp.block_table.shape[1], len(last), kernel=kernel)
+        st = DecodeStep(sessions[i], B, s_q, inp.block_table.shape[1], len(last), kernel=kernel,
+                        head_tile=args.head_tile)
         for key, name in names.items():
             st.host_in[name].copy_(torch.from_numpy(np.ascontiguousarray(host[key])).to(st.host_in[name].dtype))
         st.capture()
@@ -510,6 +514,7 @@ def run_ours(args, world, rank, local):
                        "context": list(wl.context) if isinstance(wl.context, tuple) else wl.context,
                        "cached_tokens_per_gpu": int(inp.seq_lens.sum()), "paged": wl.paged,
                        "kernel": {qkn.KERNEL_TCGEN05: "tcgen05", qkn.KERNEL_SIMT: "simt"}.get(kernel_used),
+                       "head_tile": args.head_tile or "auto",
                        "l2": f"{n_copies} rotating cache copies, {n_copies * cache_bytes / 2**20:.0f} MiB "
                              f"(L2 {l2 / 2**20:.0f} MiB)", "step_launch": "CUDA graph per step",
                        "parallelism": f"replicas x{world}"},

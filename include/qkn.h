@@ -120,8 +120,9 @@ typedef struct {
   int32_t max_ctas;        /* cap on decode CTAs (split-KV width; CTA pairs take max_ctas / 2);
                               0 = one per SM */
   int32_t head_tile;       /* tcgen05: query rows per tile (16, 32 or 64 on one CTA; 128 on a pair of
-                              CTAs that split the latent width); 0 = automatic (128 when a sequence
-                              has more than 64 query rows) */
+                              CTAs that split the latent width, r_kv = 512, d_rope = 64, at most 4
+                              groups); 0 = automatic (the smallest of 16, 32, 64 that covers a
+                              sequence's query rows, 64 beyond that) */
   int64_t wait_limit;      /* bounded-wait limit in clock cycles for the mbarrier waits; 0 = default (~2 s) */
   void* split_event;       /* optional cudaEvent_t recorded between the split-KV kernel and the combine
                               kernel (external record, so it also works inside stream capture) */

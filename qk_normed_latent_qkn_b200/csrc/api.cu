@@ -72,18 +72,19 @@ RopeFreqs rope_freqs(const qkn_dims* d) {
   return r;
 }
 
-// Rows per tile for the tcgen05 kernels: the smallest supported tile that
-// covers the per-sequence query rows.  Up to 64 rows one CTA takes a tile
-// (the fp32 accumulator of a 64-row tile already fills an SM's tensor
-// memory); above that, tiles of 128 rows go to CTA pairs that split the
-// latent width, so that every MMA has 128 rows.
+// Rows per tile for the tcgen05 kernels: the smallest supported single-CTA
+// tile that covers the per-sequence query rows, at most 64 (the fp32
+// accumulator of a 64-row tile already fills an SM's tensor memory).  Tiles of
+// 128 rows on CTA pairs that split the latent width (every MMA with 128 rows)
+// are taken only when asked for (head_tile = 128): on this build they are
+// slower than two 64-row tiles, because every page costs three exchanges
+// between the two SMs in series.
 int tc_rows(const qkn_dims* d, int s_q, const qkn_decode_opts* o) {
   if (o && o->head_tile) return o->head_tile;
   const int qrows = s_q * d->num_heads;
   if (qrows <= 16) return 16;
   if (qrows <= 32) return 32;
-  if (qrows <= 64 || !decode_pair_supported(d->r_kv, d->d_rope, d->num_groups)) return 64;
-  return kPairRows;
+  return 64;
 }
 
 bool tc_supported(const qkn_dims* d, int rows) {

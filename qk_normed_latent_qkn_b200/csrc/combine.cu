@@ -3,12 +3,13 @@
 // log-sum-exp lse_s; the row's result is
 //   lse = log sum_s exp(lse_s),   o = sum_s exp(lse_s - lse) * o_s,
 // which is exactly the softmax over the union of the splits' tokens.
-// One CTA per four query rows of a segment.  Every thread owns the same 16
-// bytes of each row and merges the splits for them on its own: it loads the
-// splits' lse values together with its 16 bytes of their partials, two
-// splits of all four rows at a time, and keeps a running maximum per row.
-// After the segment descriptor, one round of memory latency per two splits;
-// no shared memory and no barrier.
+// One CTA per query row, or per four rows of a segment when there are many
+// rows.  Every thread owns the same 16 bytes of each of its rows and merges the
+// splits for them on its own: it loads the splits' lse values together with
+// its 16 bytes of their partials (four splits at a time for one row, two for
+// four rows) and keeps a running maximum per row.  After the segment
+// descriptor, one round of memory latency per group of splits; no shared
+// memory and no barrier.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   // Every thread owns 16 bytes of each row and merges the splits for them on its own, with a
   // running maximum of their lse values: acc = sum_s exp(lse_s - m) o_s, den = sum_s exp(lse_s - m).
   // The lse values and the partials of kDepth splits of all the CTA's rows are loaded together.
-  constexpr int kDepth = 2;
+  constexpr int kDepth = RPC == 1 ? 4 : 2;
   // consecutive splits of a segment sit ht_count slots apart
   const int64_t lstride = (int64_t)a.rows * a.ht_count;
   const int64_t stride = lstride * a.r / 4;                 // float4s between consecutive splits of a row
@@ -155,11 +156,12 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
 }
 
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st) {
-  // rows per CTA: four when the tile's row count allows it (every tile size but odd ones)
+  // rows per CTA: four when one row per CTA would take more than about two waves of the GPU
+  // (4,096 rows of 128 threads), one otherwise (more CTAs, four splits loaded at a time)
   const int64_t rows = (int64_t)a.batch * a.ht_count * a.rows;
   const size_t smem = 0;
   const dim3 block(kCombThreads);
-  if (a.rows % 4 == 0) {
+  if (a.rows % 4 == 0 && rows >= 4096) {
     const dim3 grid((unsigned)(rows / 4));
     if (a.seg_desc)
       return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, true, 4>, grid, block, smem, st, a)

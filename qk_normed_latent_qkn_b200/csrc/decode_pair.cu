@@ -15,13 +15,15 @@
 // page, holds O[128 x 256], and computes a partial score over its half:
 //   S_c[128 x 64] = Q~[:, half] . C[:, half]^T      (K = 256: 16 MMAs, M = 128, N = 64)
 //   S_R[128 x 64] = Q^R^[:, half] . K^R[:, half]^T  (K = 32: the RoPE block is split the same way)
-// Each CTA runs the softmax of 64 of the rows ("its" rows: lanes [64c, 64c + 64)
-// of the accumulators).  The other 64 rows' partial logits, already scaled to
-// a_q a_k S_c + S_R (log2 units), go to the peer through distributed shared
-// memory (st.async into the peer's exchange buffer).  After the softmax each
-// CTA writes the probabilities of its rows into its own P tile and copies them
-// with one bulk copy into the peer's P tile, so that both CTAs hold
-// P[128 x 64] and run
+// The softmax is split by tokens: CTA c finishes the logits of tokens
+// [32c, 32c + 32) of each page for all 128 rows.  Each CTA sends its partial
+// logits a_q a_k S_c + S_R of the other token half to the peer through
+// distributed shared memory (st.async into the peer's exchange buffer), adds
+// the peer's part to its own half, and the two exchange their row maxima, so
+// that both keep the same running reference per row (and rescale O by the
+// same factors without exchanging them).  Each CTA writes the probabilities of
+// its token half into its P tile and copies the tile into the peer with one
+// bulk copy; both then run
 //   O[128 x 256] += P[128 x 64] . C[64 x 256 of its half]   (4 MMAs, M = 128, N = 256)
 // Each cache byte is read once, by one CTA of the pair.  No load with cluster
 // multicast is used; the tensor core's commit signals both CTAs' P barrier.
@@ -30,11 +32,11 @@
 // [256 + 128 b, 256 + 128 b + 128), b = tile parity.
 //
 // Warp roles (352 threads, one CTA per SM):
-//   warps 0-7  math: warp w reads TMEM lanes 32 (w % 4) .. + 31 (quadrant w % 4) and tokens
-//              [32 (w / 4), 32 (w / 4) + 32) of a page.  In CTA c the warps of quadrants 2c and
-//              2c + 1 own their rows (softmax, P, lse); the other four send their lanes' partial
-//              logits to the peer and rescale / write out their lanes of O with the peer's
-//              factors;
+//   warps 0-7  math: warp w takes TMEM lanes 32 (w % 4) + 16 (w / 4) .. + 15 (16 query rows) in
+//              the 16x64b layout: two threads per row, one per column parity, so that a row's
+//              values meet by one shuffle.  Every math warp does the same work on all four
+//              SM sub-partitions (the lane quadrant of TMEM a warp can read is fixed by its
+//              sub-partition);
 //   warp 8     TMA producer (query tile per item; per page the latent half, the RoPE-key half and
 //              the a_k rows);
 //   warp 9     TMEM allocator and issuer of the score MMAs;
@@ -61,16 +63,14 @@ constexpr int kHalf = 256;                  // latent columns per CTA
 constexpr int kDrope = 64;                  // RoPE width this kernel takes
 constexpr int kRopeHalf = 32;               // RoPE columns per CTA
 constexpr int kRows = 128;                  // query rows per tile (MMA M)
-constexpr int kOwnRows = 64;                // rows whose softmax each CTA runs
-constexpr int kMaxGroups = 8;
+constexpr int kMaxGroups = 4;
 constexpr int kMathWarps = 8;
 constexpr int kProducerWarp = kMathWarps;
 constexpr int kScoreWarp = kMathWarps + 1;
 constexpr int kOutWarp = kMathWarps + 2;
 constexpr int kThreads = (kMathWarps + 3) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleLog2 = 8.0f;        // rescale O only when a row maximum grows by > 2^8
+constexpr float kRescale = 5.545177444479562f;   // rescale O only when a row maximum grows by > ln 256
 constexpr int64_t kDrainLimit = 4000000000LL;
 constexpr int64_t kSettleCycles = 400000;   // after an abort: time for exchanges in flight to land
 constexpr int kEarlyPages = 2;              // pages the producer may issue before the query tile
@@ -79,14 +79,16 @@ constexpr int kEarlyPages = 2;              // pages the producer may issue befo
 constexpr int kQChunk = kRows * 128;                     // 64 latent columns of 128 rows: 16 KB
 constexpr int Q_OFF = 0;                                 // Q~ half: 4 chunks, 128-byte swizzle
 constexpr int QR_OFF = Q_OFF + 4 * kQChunk;              // Q^R^ half: [128 rows][64 B], 64-byte swizzle
-constexpr int P_OFF = QR_OFF + kRows * 64;               // P: [128 rows][64 tokens] bf16, 128-byte swizzle
-constexpr int X_OFF = P_OFF + kRows * 128;               // peer's partial logits: [64 rows][64 tokens] fp32
-constexpr int MISC_OFF = X_OFF + kOwnRows * kPage * 4;
-constexpr int MISC_BYTES = 4096;
+constexpr int kPHalf = kRows * 64;                       // P of one token half: [128 rows][32 tokens] bf16
+constexpr int P_OFF = QR_OFF + kRows * 64;               // P tiles of token halves 0 and 1, 64-byte swizzle
+constexpr int kXBytes = kRows * 32 * 4;                  // the peer's partial logits of this CTA's token half
+constexpr int X_OFF = P_OFF + 2 * kPHalf;
+constexpr int MISC_OFF = X_OFF + kXBytes;
+constexpr int MISC_BYTES = 3072;
 constexpr int RING_OFF = MISC_OFF + MISC_BYTES;
 constexpr int kLatBytes = kPage * kHalf * 2;             // the page's latent half: 32 KB (4 chunks of 8 KB)
 constexpr int kKrBytes = kPage * kRopeHalf * 2;          // the page's RoPE-key half: 4 KB
-constexpr int kAkBytes = kPage * kMaxGroups * 4;         // the page's a_k rows: up to 2 KB
+constexpr int kAkBytes = kPage * kMaxGroups * 4;         // the page's a_k rows: up to 1 KB
 constexpr int SLOT_BYTES = kLatBytes + kKrBytes + kAkBytes;
 constexpr int KR_IN_SLOT = kLatBytes;
 constexpr int AK_IN_SLOT = kLatBytes + kKrBytes;
@@ -97,31 +99,30 @@ static_assert(SMEM <= 232448, "shared memory budget");
 
 struct PairMisc {
   uint64_t full[NS], empty[NS];   // ring: page landed / page's last reader (output MMAs) done
-  uint64_t s_full[2], s_empty[2]; // score accumulators of a tile parity: written / read out
-  uint64_t x_full;                // the peer's partial logits for this CTA's rows landed (1 arm + 16 KB)
-  uint64_t x_free;                // the peer's owner warps have read this CTA's partial logits (4 remote)
-  uint64_t pr_full;               // the peer's P rows and rescale factors landed (1 arm + 8.25 KB)
+  uint64_t s_full[2], s_empty[2]; // score accumulators of a tile parity: written / read out (8 warps)
+  uint64_t x_full;                // the peer's partial logits of this CTA's token half landed (1 arm + 16 KB)
+  uint64_t x_free;                // the peer's math warps have read this CTA's partial logits (8 remote)
+  uint64_t m_full[2], m_free[2];  // row maxima of a tile parity: the peer's landed (1 arm + 512 B) / read (8)
+  uint64_t pr_full;               // the peer's P half landed (1 arm + 8 KB)
   uint64_t p_ready;               // P tile complete and O rescaled: the output MMAs may run (8 warps)
   uint64_t p_free;                // output MMAs of the tile done in both CTAs (2 commits)
-  uint64_t l_full;                // the peer's 1 / l for the rows it owns landed (1 arm + 256 B)
-  uint64_t l_free;                // the peer's sender warps have read this CTA's 1 / l (4 remote)
+  uint64_t l_full, l_free;        // the peer's row sums of an item landed (1 arm + 512 B) / read (8 remote)
   uint64_t q_full, q_empty, o_empty, drain;
   uint32_t tmem_base;
   int32_t abort_flag;             // a role of this CTA stopped early
   int32_t abort_any;              // either CTA of the pair did (set by both, read after a cluster barrier)
   Cursor cursor;
-  alignas(16) float corr_send[kOwnRows];   // this CTA's rows: rescale factor of the tile
-  alignas(16) float corr_recv[kOwnRows];   // the peer's rows: its rescale factors
-  alignas(16) float linv_recv[kOwnRows];   // the peer's rows: 1 / l
-  alignas(16) float red[2][kOwnRows];      // the two token halves of each own row: maxima or sums
+  alignas(16) float mx_recv[2][kRows];   // the peer's row maxima over its token half, per tile parity
+  alignas(16) float l_recv[kRows];       // the peer's row sums over its token half
+  alignas(16) float linv[kRows];         // 1 / l per row, for the epilogue's 32x32b read-out
 };
 static_assert(sizeof(PairMisc) <= MISC_BYTES, "misc shared-memory block");
 
-// 128-byte swizzle: 16-byte unit u of row r of a [rows][128 B] tile sits at unit u ^ (r & 7).
-__device__ __forceinline__ uint32_t sw128(int row, int unit) { return (uint32_t)(row * 128 + ((unit ^ (row & 7)) << 4)); }
-// The exchange buffer holds 256-byte rows (64 fp32); its 16-byte units are swizzled by row the
-// same way within each half row, so that 8 consecutive rows hit distinct banks.
-__device__ __forceinline__ uint32_t xoff(int row, int unit) { return (uint32_t)(row * 256 + ((unit ^ (row & 7)) << 4)); }
+// 64-byte swizzle of a [rows][64 B] tile: 16-byte unit u of row r sits at unit u ^ ((r >> 1) & 3).
+__device__ __forceinline__ uint32_t sw64(int row, int unit) { return (uint32_t)(row * 64 + ((unit ^ ((row >> 1) & 3)) << 4)); }
+// The exchange buffer holds a 128-byte row per query row: 16 fp32 per column parity.  Its 16-byte
+// units are swizzled by row so that 8 consecutive rows hit distinct banks.
+__device__ __forceinline__ uint32_t xoff(int row, int unit) { return (uint32_t)(row * 128 + ((unit ^ (row & 7)) << 4)); }
 
 }  // namespace
 
@@ -157,12 +158,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ms.s_empty[b]), kMathWarps);
     }
     mbar_init(smem_u32(&ms.x_full), 1);
-    mbar_init(smem_u32(&ms.x_free), 4);
+    mbar_init(smem_u32(&ms.x_free), kMathWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ms.m_full[b]), 1);
+      mbar_init(smem_u32(&ms.m_free[b]), kMathWarps);
+    }
     mbar_init(smem_u32(&ms.pr_full), 1);
     mbar_init(smem_u32(&ms.p_ready), kMathWarps);
     mbar_init(smem_u32(&ms.p_free), 2);
     mbar_init(smem_u32(&ms.l_full), 1);
-    mbar_init(smem_u32(&ms.l_free), 4);
+    mbar_init(smem_u32(&ms.l_free), kMathWarps);
     mbar_init(smem_u32(&ms.q_full), 1);
     mbar_init(smem_u32(&ms.q_empty), 1);
     mbar_init(smem_u32(&ms.o_empty), kMathWarps);
@@ -321,7 +326,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kOutWarp) {
     // ------------------------------------------------------------ output MMA issuer (whole warp)
     constexpr uint32_t idPV = idesc_bf16(kRows, kHalf, false, true);
-    const uint64_t dP = smem_desc(sb + P_OFF, 16, 1024);                 // A: P [128 rows][64 tok], K-major
+    // A: P as two K-major [128 rows][32 tokens] tiles (token halves), 64-byte swizzle
+    const uint64_t dP = smem_desc_sw(sb + P_OFF, 16, 512, 4);
     // B: the page's latent half, MN-major: 64-column chunks LBO = 8 KB apart, 8-token groups SBO = 1 KB apart
     const uint64_t dCt = smem_desc(sb + RING_OFF, kPage * 128, 1024);
     RingPos<NS> cr;
@@ -335,9 +341,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint64_t slot = (uint64_t)((cr.slot * SLOT_BYTES) >> 4);
         const uint32_t acc0 = p > it.p0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kPage / 16; ++kk)
-          mma_bf16_elect(tmem, dP + (uint32_t)((kk * 32) >> 4), dCt + slot + (uint32_t)((kk * 2048) >> 4), idPV,
-                         kk > 0 ? 1u : acc0);
+        for (int kk = 0; kk < kPage / 16; ++kk)   // tokens 16 kk .. + 15: tile kk / 2, 32-byte step kk % 2
+          mma_bf16_elect(tmem, dP + (uint32_t)(((kk >> 1) * kPHalf + (kk & 1) * 32) >> 4),
+                         dCt + slot + (uint32_t)((kk * 2048) >> 4), idPV, kk > 0 ? 1u : acc0);
         mma_commit_elect(smem_u32(&ms.empty[cr.slot]));
         mma_commit_pair_elect(smem_u32(&ms.p_free), (uint16_t)0x3);
         cr.next();
@@ -354,23 +360,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_wait_warp(smem_u32(&ms.drain), 0, kDrainLimit);
   } else {
     // ------------------------------------------------------------ math warps
-    const int quad = warp & 3;                         // TMEM lane quadrant
-    const int half = warp >> 2;                        // token half of a page, column half of O
-    const int rho = quad * 32 + lane;                  // row of the tile (TMEM lane)
-    const bool owner = (uint32_t)(quad >> 1) == crank; // this CTA runs the softmax of this row
-    const int rl = rho & (kOwnRows - 1);               // row within its owner's 64
-    const uint32_t bar_id = owner ? 1u : 2u;           // named barrier of the owner / sender group
-    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const int quad = warp & 3;                         // TMEM lane quadrant (= the warp's sub-partition)
+    const int half = warp >> 2;
+    // 16x64b layout: thread t holds lane (t >> 2) + 8 (t & 1) of the warp's 16 and the columns of
+    // parity (t >> 1) & 1; the row's other thread is t ^ 2
+    const int rho = quad * 32 + half * 16 + (lane >> 2) + 8 * (lane & 1);
+    const int par = (lane >> 1) & 1;
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32 + half * 16) << 16);
+    const uint32_t tl32 = tmem + ((uint32_t)(quad * 32) << 16);     // 32x32b: the whole quadrant
+    const int own0 = (int)crank * 32, peer0 = (int)prank * 32;    // first token of each half of a page
+    const bool leader = threadIdx.x == 0;
     const uint32_t peer_x_full = mapa_shared(smem_u32(&ms.x_full), prank);
     const uint32_t peer_x_free = mapa_shared(smem_u32(&ms.x_free), prank);
+    const uint32_t peer_m_full = mapa_shared(smem_u32(&ms.m_full[0]), prank);     // + 8 b for parity b
+    const uint32_t peer_m_free = mapa_shared(smem_u32(&ms.m_free[0]), prank);
     const uint32_t peer_pr_full = mapa_shared(smem_u32(&ms.pr_full), prank);
     const uint32_t peer_l_full = mapa_shared(smem_u32(&ms.l_full), prank);
     const uint32_t peer_l_free = mapa_shared(smem_u32(&ms.l_free), prank);
     const uint32_t peer_x = mapa_shared(sb + X_OFF, prank);
+    const uint32_t peer_mx = mapa_shared(smem_u32(&ms.mx_recv[0][0]), prank);
+    const uint32_t peer_l = mapa_shared(smem_u32(&ms.l_recv[0]), prank);
     const uint32_t peer_p = mapa_shared(sb + P_OFF, prank);
-    const uint32_t peer_corr = mapa_shared(smem_u32(&ms.corr_recv[0]), prank);
-    const uint32_t peer_linv = mapa_shared(smem_u32(&ms.linv_recv[0]), prank);
-    const bool leader = owner && (quad & 1) == 0 && half == 0 && lane == 0;   // one owner thread
     if (a.step_writes_only) pdl_wait();                // a_q is written by the preceding kernel
     const int ng = a.heads / G;
     RingPos<NS> cr;
@@ -386,208 +396,198 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool valid = rg < qrows;
       const int j = valid ? rg / a.heads : 0;
       const int grp = (valid ? rg - j * a.heads : 0) / ng;
-      const float aq2 = valid ? a.a_q[(int64_t)it.b * qrows + rg] * kLog2e : 0.f;
+      const float aq = valid ? a.a_q[(int64_t)it.b * qrows + rg] : 0.f;
       const int qlim = valid ? it.L - a.s_q + j : -1;
-      float mu = -INFINITY, lpart = 0.f;
+      float mu = -INFINITY, lsum = 0.f;               // reference and this thread's part of the row sum
+      // A wait that runs out makes `got` false; the math warps leave together, at the next vote
+      // over all 256 of them (every named barrier of the loop is such a vote), never at a barrier
+      // that some of them would not reach.  `carry` takes the last wait of a tile to the next vote.
+      bool carry = true;
       for (int p = it.p0; p < it.p1; ++p) {
-        const int sbi = (int)(tile_n & 1);
+        const int sbi = (int)(tile_n & 1);             // score buffer of the tile and its phase parity
         const uint32_t sph = (uint32_t)((tile_n >> 1) & 1);
         const uint32_t tph = (uint32_t)(tile_n & 1);   // phase parity of the once-per-tile barriers
-        const uint32_t tS = tl + kHalf + sbi * 128 + half * 32;
-        // scores of this lane's row and this warp's 32 tokens
-        bool got = mbar_wait(smem_u32(&ms.s_full[sbi]), sph, a.wait_limit);
+        const uint32_t tS = tq + kHalf + sbi * 128;
+        // scores of this row: S_c and S_R of this thread's parity in both token halves
+        bool got = mbar_wait(smem_u32(&ms.s_full[sbi]), sph, a.wait_limit) && carry;
         tc_fence_after();
-        uint32_t sc[32], sr[32];
-        tmem_ld32(tS, sc);
-        tmem_ld32(tS + 64, sr);
+        uint32_t so[16], sp_[16], ro[16], rp[16];
+        tmem_ld16x64_x16(tS + own0, so);
+        tmem_ld16x64_x16(tS + peer0, sp_);
+        tmem_ld16x64_x16(tS + 64 + own0, ro);
+        tmem_ld16x64_x16(tS + 64 + peer0, rp);
         tmem_wait_ld();
-        reg_tie(sc);
-        reg_tie(sr);
+        reg_tie(so);
+        reg_tie(sp_);
+        reg_tie(ro);
+        reg_tie(rp);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ms.s_empty[sbi]));
         // the page's a_k rows (the ring barrier also covers them; normally complete long before)
         const float* akp = reinterpret_cast<const float*>(smem + RING_OFF + cr.slot * SLOT_BYTES + AK_IN_SLOT);
         if (!AK_ONE) got = mbar_wait(smem_u32(&ms.full[cr.slot]), cr.phase, a.wait_limit) && got;
-        // this CTA's part of the logits, log2 units: a_q a_k S_c + S_R over its latent and RoPE halves
-        float x[32];
+        // this CTA's part of the logits a_q a_k S_c + S_R (its latent and RoPE halves), token 2r + par
+        // of each half
+        float x[16], y[16];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float ak = AK_ONE ? 1.f : akp[(half * 32 + t) * G + grp];
-          x[t] = aq2 * ak * __uint_as_float(sc[t]) + kLog2e * __uint_as_float(sr[t]);
+        for (int r = 0; r < 16; ++r) {
+          const float ako = AK_ONE ? 1.f : akp[(own0 + 2 * r + par) * G + grp];
+          const float akq = AK_ONE ? 1.f : akp[(peer0 + 2 * r + par) * G + grp];
+          x[r] = fmaf(aq * ako, __uint_as_float(so[r]), __uint_as_float(ro[r]));
+          y[r] = fmaf(aq * akq, __uint_as_float(sp_[r]), __uint_as_float(rp[r]));
         }
-        if (!owner) {
-          // ---- sender: the peer owns this row; its part goes to the peer's exchange buffer
-          got = mbar_wait_cl(smem_u32(&ms.x_free), tph ^ 1u, a.wait_limit) && got;
-          if (got) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              st_async_v4(peer_x + xoff(rl, half * 8 + u), __float_as_uint(x[4 * u]), __float_as_uint(x[4 * u + 1]),
-                          __float_as_uint(x[4 * u + 2]), __float_as_uint(x[4 * u + 3]), peer_x_full);
-          }
-          // then the peer's rescale factors (with its P rows) for these rows of O
-          got = mbar_wait_cl(smem_u32(&ms.pr_full), tph, a.wait_limit) && got;
-          if (bar_any128(!got, bar_id)) { ok = false; break; }
-          const float corr = ms.corr_recv[rl];
-          if (bar_any128(corr != 1.f, bar_id) && p > it.p0) {
-            // O holds this item's earlier tiles: rescale once the previous tile's output MMAs are done
-            const bool done = mbar_wait_cl(smem_u32(&ms.p_free), tph ^ 1u, a.wait_limit);
-            if (bar_any128(!done, bar_id)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 16) {
-              uint32_t ov[16];
-              tmem_ld16(tl + half * 128 + c0, ov);
-              tmem_wait_ld();
-              reg_tie(ov);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-              tmem_st16(tl + half * 128 + c0, ov);
-            }
-            tmem_wait_st();
-          }
-        } else {
-          // ---- owner: add the peer's part, softmax, P
-          if (leader) mbar_arrive_expect_tx(smem_u32(&ms.x_full), kOwnRows * kPage * 4);
-          got = mbar_wait_cl(smem_u32(&ms.x_full), tph, a.wait_limit) && got;
-          const int tok0 = p * kPage;
-          const int nvalid = min(kPage, it.L - tok0);
-          if (got) {
-            const uint8_t* xr = smem + X_OFF;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float4 v = *reinterpret_cast<const float4*>(xr + xoff(rl, half * 8 + u));
-              x[4 * u] += v.x;
-              x[4 * u + 1] += v.y;
-              x[4 * u + 2] += v.z;
-              x[4 * u + 3] += v.w;
-            }
-          }
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const int tok = half * 32 + t;
-            if (tok >= nvalid || tok0 + tok > qlim) x[t] = -INFINITY;
-          }
-          __syncwarp();
-          if (lane == 0 && got) mbar_arrive_remote(peer_x_free);   // this warp is done with the buffer
-          // The exponentials use a running reference mu per row that only has to stay within 2^8 of
-          // the true maximum: one group vote per tile, and the row maxima only when it says yes.
-          bool over = false;
-#pragma unroll
-          for (int t = 0; t < 32; ++t) over |= x[t] > mu + kRescaleLog2;
-          float corr = 1.f;
-          if (bar_any128(over || !got, bar_id)) {
-            if (bar_any128(!got, bar_id)) { ok = false; break; }
-            float m = x[0];
-#pragma unroll
-            for (int t = 1; t < 32; ++t) m = fmaxf(m, x[t]);
-            ms.red[half][rl] = m;
-            named_bar_sync(bar_id, 128);
-            const float mt = fmaxf(ms.red[0][rl], ms.red[1][rl]);
-            named_bar_sync(bar_id, 128);
-            bool changed = false;
-            if (mt > mu + kRescaleLog2) {
-              corr = (mu == -INFINITY) ? 0.f : ex2(mu - mt);
-              mu = mt;
-              changed = true;
-            }
-            if (bar_any128(changed, bar_id) && p > it.p0) {
-              const bool done = mbar_wait_cl(smem_u32(&ms.p_free), tph ^ 1u, a.wait_limit);
-              if (bar_any128(!done, bar_id)) { ok = false; break; }
-              tc_fence_after();
-              // tcgen05.ld / st are warp-collective (.sync.aligned): the whole warp rescales when any
-              // of its rows changed, the others by 1
-              if (__any_sync(0xffffffffu, corr != 1.f)) {
-#pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 16) {
-                  uint32_t ov[16];
-                  tmem_ld16(tl + half * 128 + c0, ov);
-                  tmem_wait_ld();
-                  reg_tie(ov);
-#pragma unroll
-                  for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                  tmem_st16(tl + half * 128 + c0, ov);
-                }
-              }
-              tmem_wait_st();
-            }
-            lpart *= corr;
-          }
-          // probabilities (bf16 pairs) and this thread's part of the row sum
-          uint32_t w[16];
-#pragma unroll
-          for (int t = 0; t < 32; t += 2) {
-            const float p0 = x[t] == -INFINITY ? 0.f : ex2(x[t] - mu);
-            const float p1 = x[t + 1] == -INFINITY ? 0.f : ex2(x[t + 1] - mu);
-            lpart += p0 + p1;
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            w[t >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          // the P tile is free once the previous tile's output MMAs are done in both CTAs
-          const bool pfree = mbar_wait_cl(smem_u32(&ms.p_free), tph ^ 1u, a.wait_limit);
-          if (bar_any128(!pfree, bar_id)) { ok = false; break; }
+        // the peer's token half goes to the peer (once it has read the previous tile's)
+        got = mbar_wait_cl(smem_u32(&ms.x_free), tph ^ 1u, a.wait_limit) && got;
+        if (got) {
 #pragma unroll
           for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(smem + P_OFF + sw128(rho, half * 4 + u)) =
-                make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-          if (half == 0) ms.corr_send[rl] = corr;
-          fence_proxy_async_smem();
-          named_bar_sync(bar_id, 128);
-          if (leader) {
-            // this CTA's P rows and factors into the peer's tiles; and the arm for the peer's
-            mbar_arrive_expect_tx(smem_u32(&ms.pr_full), kOwnRows * 128 + kOwnRows * 4);
-            const uint32_t rows0 = (uint32_t)(crank * kOwnRows * 128);
-            bulk_copy_to_peer(peer_p + rows0, sb + P_OFF + rows0, kOwnRows * 128, peer_pr_full);
-            bulk_copy_to_peer(peer_corr, smem_u32(&ms.corr_send[0]), kOwnRows * 4, peer_pr_full);
+            st_async_v4(peer_x + xoff(rho, par * 4 + u), __float_as_uint(y[4 * u]), __float_as_uint(y[4 * u + 1]),
+                        __float_as_uint(y[4 * u + 2]), __float_as_uint(y[4 * u + 3]), peer_x_full);
+        }
+        // and the peer's part of this CTA's half comes back
+        if (leader) mbar_arrive_expect_tx(smem_u32(&ms.x_full), kXBytes);
+        got = mbar_wait_cl(smem_u32(&ms.x_full), tph, a.wait_limit) && got;
+        if (got) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 v = *reinterpret_cast<const float4*>(smem + X_OFF + xoff(rho, par * 4 + u));
+            x[4 * u] += v.x;
+            x[4 * u + 1] += v.y;
+            x[4 * u + 2] += v.z;
+            x[4 * u + 3] += v.w;
           }
+        }
+        __syncwarp();
+        if (lane == 0 && got) mbar_arrive_remote(peer_x_free);
+        // tokens past the context or after the row's query position get no weight (only the pages
+        // that hold such tokens need the test)
+        const int tok0 = p * kPage;
+        const int nvalid = min(kPage, it.L - tok0);
+        if (__any_sync(0xffffffffu, nvalid < kPage || tok0 + kPage - 1 > qlim)) {
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const int tok = own0 + 2 * r + par;
+            if (tok >= nvalid || tok0 + tok > qlim) x[r] = -INFINITY;
+          }
+        }
+        // row maximum over this CTA's token half, then over both: the peer gets this half's
+        float m = x[0];
+#pragma unroll
+        for (int r = 1; r < 16; ++r) m = fmaxf(m, x[r]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        got = mbar_wait_cl(smem_u32(&ms.m_free[sbi]), sph ^ 1u, a.wait_limit) && got;
+        if (par == 0 && got) st_async_b32(peer_mx + (sbi * kRows + rho) * 4, __float_as_uint(m), peer_m_full + 8 * sbi);
+        if (leader) mbar_arrive_expect_tx(smem_u32(&ms.m_full[sbi]), kRows * 4);
+        got = mbar_wait_cl(smem_u32(&ms.m_full[sbi]), sph, a.wait_limit) && got;
+        const float mt = fmaxf(m, ms.mx_recv[sbi][rho]);
+        __syncwarp();
+        if (lane == 0 && got) mbar_arrive_remote(peer_m_free + 8 * sbi);
+        // The exponentials use a running reference mu per row that only has to stay within e^kR of
+        // the true maximum; both CTAs see the same maxima, so they raise mu together.
+        float corr = 1.f;
+        if (mt > mu + kRescale) {
+          corr = (mu == -INFINITY) ? 0.f : ex2((mu - mt) * kLog2e);
+          mu = mt;
+        }
+        // O holds this item's earlier tiles: rescale this warp's rows (tcgen05.ld / st are
+        // warp-collective, so the whole warp takes part, rows that did not change by 1) once the
+        // previous tile's output MMAs are done
+        const bool resc = __any_sync(0xffffffffu, corr != 1.f) && p > it.p0;   // warp-uniform
+        if (resc) got = mbar_wait_cl(smem_u32(&ms.p_free), tph ^ 1u, a.wait_limit) && got;
+        const bool warp_got = __all_sync(0xffffffffu, got);
+        if (resc && warp_got) {
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < kHalf; c0 += 32) {
+            uint32_t ov[16];
+            tmem_ld16x64_x16(tq + c0, ov);
+            tmem_wait_ld();
+            reg_tie(ov);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+            tmem_st16x64_x16(tq + c0, ov);
+          }
+          tmem_wait_st();
+        }
+        lsum *= corr;
+        // probabilities and this thread's part of the row sum; a row with no visible token so far
+        // (mu = -inf) has only -inf logits, whose exponentials are 0 against any mu2
+        const float mu2 = mu == -INFINITY ? 0.f : mu * kLog2e;
+        float pr[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          pr[r] = ex2(fmaf(x[r], kLog2e, -mu2));
+          lsum += pr[r];
+        }
+        // bf16 pairs of consecutive tokens: the row's two threads swap half of their values, so that
+        // parity 0 holds tokens 0 .. 15 of the half and parity 1 tokens 16 .. 31
+        uint32_t w[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float send = par == 0 ? pr[r + 8] : pr[r];
+          const float got2 = __shfl_xor_sync(0xffffffffu, send, 2);
+          const __nv_bfloat162 b2 = par == 0 ? __floats2bfloat162_rn(pr[r], got2) : __floats2bfloat162_rn(got2, pr[r + 8]);
+          w[r] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        // the P tile is free once the previous tile's output MMAs are done in both CTAs
+        got = mbar_wait_cl(smem_u32(&ms.p_free), tph ^ 1u, a.wait_limit) && got;
+        if (got) {
+          uint8_t* pt = smem + P_OFF + crank * kPHalf;
+          *reinterpret_cast<uint4*>(pt + sw64(rho, par * 2)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(pt + sw64(rho, par * 2 + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
         }
         // rows of the page past the context: zero this CTA's latent half of them, so that 0 * (stale
         // bits, possibly NaN) cannot reach O through the output MMAs (the score MMAs are done with
         // the page: its s_full phase completed above)
-        const int nvalid_pg = min(kPage, it.L - p * kPage);
-        if (nvalid_pg < kPage) {
+        if (nvalid < kPage) {
           uint8_t* lat = smem + RING_OFF + cr.slot * SLOT_BYTES;
-          for (int e = threadIdx.x; e < (kPage - nvalid_pg) * 32; e += kMathWarps * 32) {
-            const int tok = nvalid_pg + (e >> 5), chunk = (e >> 3) & 3, unit = e & 7;
+          for (int e = threadIdx.x; e < (kPage - nvalid) * 32; e += kMathWarps * 32) {
+            const int tok = nvalid + (e >> 5), chunk = (e >> 3) & 3, unit = e & 7;
             *reinterpret_cast<uint4*>(lat + chunk * (kPage * 128) + tok * 128 + (unit << 4)) = make_uint4(0, 0, 0, 0);
           }
-          fence_proxy_async_smem();
         }
+        fence_proxy_async_smem();
+        if (bar_any(!got, 1, kMathWarps * 32)) { ok = false; break; }
+        if (leader) {
+          // this CTA's P half into the peer's tile; and the arm for the peer's half
+          mbar_arrive_expect_tx(smem_u32(&ms.pr_full), kPHalf);
+          bulk_copy_to_peer(peer_p + crank * kPHalf, sb + P_OFF + crank * kPHalf, kPHalf, peer_pr_full);
+        }
+        // the output MMAs also need the peer's half
+        carry = mbar_wait_cl(smem_u32(&ms.pr_full), tph, a.wait_limit);
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&ms.p_ready));
+        const bool warp_carry = __all_sync(0xffffffffu, carry);
+        if (lane == 0 && warp_carry) mbar_arrive(smem_u32(&ms.p_ready));
         cr.next();
         ++tile_n;
       }
       if (!ok) break;
-      // ---------------- epilogue of the item: O / l for every lane, lse for own rows
-      const uint32_t last = (uint32_t)((tile_n - 1) & 1);
-      bool got = mbar_wait_cl(smem_u32(&ms.p_free), last, a.wait_limit);
-      float linv = 0.f;
-      if (owner) {
-        ms.red[half][rl] = lpart;
-        named_bar_sync(bar_id, 128);
-        const float l = ms.red[0][rl] + ms.red[1][rl];
-        named_bar_sync(bar_id, 128);
-        linv = l > 0.f ? 1.f / l : 0.f;
-        if (half == 0) a.part_lse[(int64_t)it.slot * kRows + rho] = l > 0.f ? (mu + log2f(l)) * kLn2 : -INFINITY;
-        // 1 / l of these rows to the peer, once its senders have read the previous item's
-        if (leader) mbar_arrive_expect_tx(smem_u32(&ms.l_full), kOwnRows * 4);
-        got = mbar_wait_cl(smem_u32(&ms.l_free), (uint32_t)((n_item & 1) ^ 1), a.wait_limit) && got;
-        if (half == 0 && got) st_async_b32(peer_linv + rl * 4, __float_as_uint(linv), peer_l_full);
-      } else {
-        got = mbar_wait_cl(smem_u32(&ms.l_full), (uint32_t)(n_item & 1), a.wait_limit) && got;
-        linv = ms.linv_recv[rl];
-        __syncwarp();
-        if (lane == 0 && got) mbar_arrive_remote(peer_l_free);
+      // ---------------- epilogue of the item: O / l for every lane, lse
+      bool got = mbar_wait_cl(smem_u32(&ms.p_free), (uint32_t)((tile_n - 1) & 1), a.wait_limit) && carry;
+      const float lh = lsum + __shfl_xor_sync(0xffffffffu, lsum, 2);   // this CTA's token half of the row
+      got = mbar_wait_cl(smem_u32(&ms.l_free), (uint32_t)((n_item & 1) ^ 1), a.wait_limit) && got;
+      if (par == 0 && got) st_async_b32(peer_l + rho * 4, __float_as_uint(lh), peer_l_full);
+      if (leader) mbar_arrive_expect_tx(smem_u32(&ms.l_full), kRows * 4);
+      got = mbar_wait_cl(smem_u32(&ms.l_full), (uint32_t)(n_item & 1), a.wait_limit) && got;
+      const float l = lh + ms.l_recv[rho];
+      __syncwarp();
+      if (lane == 0 && got) mbar_arrive_remote(peer_l_free);
+      if (par == 0) {
+        ms.linv[rho] = l > 0.f ? 1.f / l : 0.f;
+        if (crank == 0) a.part_lse[(int64_t)it.slot * kRows + rho] = l > 0.f ? mu + logf(l) : -INFINITY;
       }
-      if (bar_any128(!got, bar_id)) { ok = false; break; }
+      if (bar_any(!got, 1, kMathWarps * 32)) { ok = false; break; }
       tc_fence_after();
-      float* po = a.part_o + ((int64_t)it.slot * kRows + rho) * kRkv + crank * kHalf + half * 128;
+      // read-out in the 32x32b layout: this warp takes every row of its quadrant, O columns
+      // [128 half, 128 half + 128)
+      const int orow = quad * 32 + lane;
+      const float linv = ms.linv[orow];
+      float* po = a.part_o + ((int64_t)it.slot * kRows + orow) * kRkv + crank * kHalf + half * 128;
 #pragma unroll
       for (int c0 = 0; c0 < 128; c0 += 16) {
         uint32_t ov[16];
-        tmem_ld16(tl + half * 128 + c0, ov);
+        tmem_ld16(tl32 + half * 128 + c0, ov);
         tmem_wait_ld();
         reg_tie(ov);
 #pragma unroll
@@ -597,10 +597,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                           __uint_as_float(ov[e + 2]) * linv, __uint_as_float(ov[e + 3]) * linv);
       }
       tc_fence_before();
-      __syncwarp();
+      named_bar_sync(1, kMathWarps * 32);              // ms.linv is read before the next item writes it
       if (lane == 0) mbar_arrive(smem_u32(&ms.o_empty));
       // the pair holding a segment's first split tells the merge kernel where its splits are
-      if (crank == 0 && warp == 0 && lane == 0 && it.p0 == 0) {
+      if (crank == 0 && threadIdx.x == 0 && it.p0 == 0) {
         const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota, sp.item_cost);
         a.seg_desc[it.b * a.ht_count + it.ht] = make_int2((it.b + sg.c0) * a.ht_count + it.ht, sg.nitems);
       }

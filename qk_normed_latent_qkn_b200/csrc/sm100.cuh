@@ -173,6 +173,16 @@ __device__ __forceinline__ void tmem_ld16x64_x16(uint32_t taddr, uint32_t (&v)[1
       : "r"(taddr));
 }
 
+// The store of the same 16x64b.x16 layout.
+__device__ __forceinline__ void tmem_st16x64_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x64b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Wait for outstanding TMEM loads; the registers are tied to the wait so that
 // no use of them can be scheduled before it.
@@ -243,6 +253,21 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// OR of a predicate over the `threads` threads that share named barrier `bar` (also a barrier for
+// them; every one of them must reach it).
+__device__ __forceinline__ bool bar_any(bool v, uint32_t bar, uint32_t threads) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(bar), "r"(threads)
+      : "memory");
+  return r != 0;
 }
 
 // OR of a predicate over the 128 threads that share named barrier `bar` (also a barrier for them).
@@ -364,16 +389,21 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void st_shared_remote_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
-// Arrive on an mbarrier of another CTA of the cluster (address from mapa_shared).
+// Arrive on an mbarrier of another CTA of the cluster (address from mapa_shared).  Relaxed: the
+// arrivals this is used for only say "this CTA has read what the other wrote" (the values read are
+// already in registers), so they order nothing and need not wait for this thread's earlier stores,
+// which a release at cluster scope would (remote stores still in flight included).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
-// try_wait with acquire at cluster scope: for phases completed by another CTA's arrivals or stores.
+// Non-blocking test with acquire at cluster scope: for phases completed by another CTA's arrivals
+// or stores.  (A try_wait may suspend the thread up to a time limit of its own; a phase that
+// another SM completes is then seen only when that limit runs out, so these waits poll.)
 __device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)

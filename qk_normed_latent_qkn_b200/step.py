@@ -27,11 +27,12 @@ class DecodeStep:
     NAMES = ("c", "k_rope", "slot", "pos", "q", "q_rope", "qpos", "block_table", "seq_lens")
 
     def __init__(self, session, batch: int, s_q: int, max_blocks: int, n_tok: int, kernel: int = KERNEL_AUTO,
-                 ak_mode: int = AK_CACHE):
+                 ak_mode: int = AK_CACHE, head_tile: int = 0):
         d = session.dims
         dt, dev, i32 = d.torch_dtype, session.device, torch.int32
         n_q = batch * s_q
         self.session, self.batch, self.s_q, self.kernel, self.ak_mode = session, batch, s_q, kernel, ak_mode
+        self.head_tile = head_tile
         shapes = {
             "c": ((n_tok, d.r_kv), dt), "k_rope": ((n_tok, d.d_rope), dt),
             "slot": ((n_tok,), i32), "pos": ((n_tok,), i32),
@@ -85,7 +86,8 @@ class DecodeStep:
                       s.w_k, s.key_gram, s.gamma_q, s.gamma_k, s.gamma_qr, s.gamma_kr, s.q_tilde, s.a_q,
                       s.q_rope_hat)
         decode(d, s.cache, s.q_tilde, s.a_q, s.q_rope_hat, di["block_table"], di["seq_lens"], self.s_q,
-               self.workspace, self.out, self.lse, ak_mode=self.ak_mode, kernel=self.kernel, step_writes_only=True)
+               self.workspace, self.out, self.lse, ak_mode=self.ak_mode, kernel=self.kernel, head_tile=self.head_tile,
+               step_writes_only=True)
         self._host_out_buf.copy_(self._dev_out_buf, non_blocking=True)
 
     def capture(self) -> None:

@@ -32,7 +32,8 @@ CASES = {
 
 
 def _decode(s, inp, **kw):
-    out, lse = s.decode(inp.block_table, inp.seq_lens, inp.wl.s_q, kernel=qkn.KERNEL_TCGEN05, **kw)
+    kw.setdefault("kernel", qkn.KERNEL_TCGEN05)
+    out, lse = s.decode(inp.block_table, inp.seq_lens, inp.wl.s_q, **kw)
     torch.cuda.synchronize()
     return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
 
@@ -48,6 +49,20 @@ def test_wait_that_runs_out_is_reported_and_the_next_decode_is_correct(name):
     o, lse = _decode(s, inp)
     assert s.device_status() == qkn.OK
     assert_close_to_oracle(inp, o, lse, what=f"{name} after a timeout")
+
+
+@pytest.mark.parametrize("name", ["large_mla_bf16", "grouped_mtp_bf16"])
+def test_wait_that_runs_out_on_the_cta_pair_kernel(name):
+    # 128-row tiles on CTA pairs: a timeout in one CTA of a pair must wind both down (the two
+    # exchange data every page) and leave the context usable
+    inp = make_inputs(CASES[name])
+    s = session_from_inputs(inp)
+    _decode(s, inp, head_tile=128, wait_limit=SHORT_WAIT, test_withhold_ak=True)
+    assert s.device_status() == qkn.ERR_TIMEOUT
+    s.clear_status()
+    o, lse = _decode(s, inp, head_tile=128)
+    assert s.device_status() == qkn.OK
+    assert_close_to_oracle(inp, o, lse, what=f"{name} on CTA pairs after a timeout")
 
 
 def test_timeout_twice_in_a_row_then_correct():

@@ -1,7 +1,7 @@
 """The CTA-pair decode (tiles of 128 query rows, latent split across the two
 CTAs of a cluster) against the fp64 oracle, through the C ABI (GPU).
 
-The 128-head and grouped two-token workloads take this kernel automatically;
+The kernel is taken when a caller asks for 128-row tiles (head_tile = 128);
 these cases pin its edges: page and tile boundaries with two query tokens and
 four KV groups, row counts that leave padding rows in a tile (96 rows, and
 160 rows = one full and one partial tile), plain-MLA mode (whose unnormalised
@@ -40,8 +40,8 @@ def test_pair_page_boundaries_two_tokens_four_groups():
     # 64 heads x 2 query tokens = one 128-row tile; lengths at and around page edges, and L = s_q
     wl = WORKLOADS["grouped_mtp_bf16"].with_(batch=8, seed=44)
     inp = make_inputs(wl, seq_lens=[2, 63, 64, 65, 127, 128, 129, 257])
-    s, o, lse = run_decode(inp, kernel=qkn.KERNEL_TCGEN05)
-    assert qkn.decode_kernel_for(s.dims, wl.s_q) == qkn.KERNEL_TCGEN05
+    s, o, lse = run_decode(inp, kernel=qkn.KERNEL_TCGEN05, head_tile=PAIR)
+    assert qkn.decode_kernel_for(s.dims, wl.s_q, head_tile=PAIR) == qkn.KERNEL_TCGEN05
     assert_close_to_oracle(inp, o, lse, what="pair boundaries")
 
 
