@@ -44,7 +44,7 @@ from typing import Iterable, Optional, Tuple
 import numpy as np
 
 __all__ = ["inv_rms", "rms_norm", "rope", "key_inv_rms", "rope_keys", "absorbed_query",
-           "sequence_logits", "decode", "decode_sequence"]
+           "sequence_logits", "decode", "decode_sequence", "up_project"]
 
 
 def inv_rms(x: np.ndarray, eps: float) -> np.ndarray:
@@ -196,3 +196,21 @@ def decode(inp, seqs: Optional[Iterable[int]] = None,
     for b in (range(B) if seqs is None else seqs):
         o[b], lse[b] = decode_sequence(inp, b, chunk)
     return o, lse
+
+
+def up_project(o_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
+    """Per-head value up-projection of the latent attention output.
+
+    The values of the absorbed path are the latents c_t themselves, so the
+    attention output lives in latent space; the value up-projection W^UV_h of
+    each head is applied once to that output instead of to every cached
+    token (GQLA summary, section 2, absorbed MQA route: the up-projections
+    move into the query and output projections).
+    ``o_lat`` is [..., H, r] and ``w_uv`` [H, r, d_v]; returns [..., H, d_v].
+    """
+    o = np.asarray(o_lat, dtype=np.float64)
+    w = np.asarray(w_uv, dtype=np.float64)
+    out = np.empty(o.shape[:-1] + (w.shape[2],))
+    for h in range(w.shape[0]):
+        out[..., h, :] = o[..., h, :] @ w[h]
+    return out

@@ -52,6 +52,7 @@ class Workload:
     rope_theta: float = 10000.0
     seed: int = 0
     block_size: int = BLOCK_SIZE
+    d_v: int = 128                         # per-head value width of the output up-projection
 
     @property
     def heads_per_group(self) -> int:
@@ -69,7 +70,7 @@ class Workload:
 # open (long-context and grouped cases), as in the large MLA case.
 WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", batch=1, s_q=1, heads=4, groups=1, r_kv=64, d_h=32,
-                         d_rope=16, context=256, paged=False, dtype="f32"),
+                         d_rope=16, context=256, paged=False, dtype="f32", d_v=32),
     "small_mla_bf16": Workload("small_mla_bf16", batch=16, s_q=1, heads=16, groups=1, r_kv=512,
                                d_h=128, d_rope=64, context=4096, paged=False, dtype="bf16"),
     "large_mla_bf16": Workload("large_mla_bf16", batch=32, s_q=1, heads=128, groups=1, r_kv=512,
@@ -122,6 +123,7 @@ class Inputs:
     gamma_k: np.ndarray         # [H, d_h]  head h's slice of its group's key norm weight
     gamma_qr: np.ndarray        # [H, d_R]
     gamma_kr: np.ndarray        # [d_R]     shared RoPE key norm weight
+    w_uv: np.ndarray            # [H, r, d_v] value up-projection W^UV_h of every head
 
     @property
     def total_tokens(self) -> int:
@@ -202,6 +204,8 @@ def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
     gamma_k = (1.0 + 0.1 * rng.standard_normal((wl.heads, wl.d_h), dtype=f32)).astype(f32)
     gamma_qr = (1.0 + 0.1 * rng.standard_normal((wl.heads, wl.d_rope), dtype=f32)).astype(f32)
     gamma_kr = (1.0 + 0.1 * rng.standard_normal(wl.d_rope, dtype=f32)).astype(f32)
+    # drawn last, so that every value above is the same with or without it
+    w_uv = rng.standard_normal((wl.heads, wl.r_kv, wl.d_v), dtype=f32) * f32(1.0 / np.sqrt(wl.r_kv))
 
     if wl.dtype == "bf16":
         c, k_rope, q, q_rope = (round_to_bf16(a) for a in (c, k_rope, q, q_rope))
@@ -211,4 +215,4 @@ def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
     return Inputs(wl=wl, seq_lens=lens, tok_off=tok_off, block_table=table, num_blocks=pool,
                   c=np.ascontiguousarray(c, f32), k_rope=np.ascontiguousarray(k_rope, f32),
                   q=q, q_rope=q_rope, w_k=w_k, gamma_q=gamma_q, gamma_k=gamma_k,
-                  gamma_qr=gamma_qr, gamma_kr=gamma_kr)
+                  gamma_qr=gamma_qr, gamma_kr=gamma_kr, w_uv=w_uv)

@@ -351,6 +351,40 @@ def check_permutation_invariance():
     np.testing.assert_allclose(lse1, lse0, rtol=1e-12)
 
 
+# --------------------------------------------------------------------------
+# 9. Output up-projection: applying W^UV_h once to the latent output equals
+#    attending over the per-token values c_t W^UV_h (GQLA summary, section 2,
+#    absorbed route: the up-projection moves to the output side).
+# --------------------------------------------------------------------------
+def check_up_projection_equals_explicit_values():
+    for wl in (TINY, TINY_MTP):
+        inp = make_inputs(wl.with_(d_v=3))
+        o_lat, _ = oracle.decode(inp)
+        got = oracle.up_project(o_lat, inp.w_uv)
+        for b in range(wl.batch):
+            c = inp.c[inp.sequence(b)].astype(np.float64)
+            l = oracle.sequence_logits(inp, b)                       # [s_q, H, L]
+            p = np.exp(l - l.max(-1, keepdims=True))
+            p /= p.sum(-1, keepdims=True)
+            for h in range(wl.heads):
+                v = c @ inp.w_uv[h].astype(np.float64)                 # values materialised per token
+                np.testing.assert_allclose(got[b, :, h], p[:, h] @ v, rtol=1e-11, atol=1e-13)
+
+
+def check_up_projection_selectors():
+    """W^UV_h picking latent columns (a column selection of the identity) returns exactly those columns."""
+    rng = np.random.default_rng(12)
+    H, r, d_v = 3, 7, 4
+    o = rng.standard_normal((2, 5, H, r))
+    w = np.zeros((H, r, d_v))
+    cols = [rng.permutation(r)[:d_v] for _ in range(H)]
+    for h in range(H):
+        w[h, cols[h], np.arange(d_v)] = 1.0
+    got = oracle.up_project(o, w)
+    for h in range(H):
+        assert np.array_equal(got[:, :, h], o[:, :, h][..., cols[h]])
+
+
 ALL_CHECKS = [
     check_absorbed_query_exact,
     check_absorbed_query_row_scale,
@@ -365,4 +399,6 @@ ALL_CHECKS = [
     check_brute_force_causal,
     check_rope_properties,
     check_permutation_invariance,
+    check_up_projection_equals_explicit_values,
+    check_up_projection_selectors,
 ]

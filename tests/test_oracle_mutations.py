@@ -30,6 +30,10 @@ MUTATIONS = {
     "row_scale_without_sigma": ("a_q = softmax_scale * inv_rms(q, eps)", "a_q = inv_rms(q, eps)"),
     "row_scale_half_width": ("a_q = softmax_scale * inv_rms(q, eps)",
                              "a_q = softmax_scale * inv_rms(q[..., ::2], eps)"),
+    "up_projection_wrong_head": ("out[..., h, :] = o[..., h, :] @ w[h]",
+                                 "out[..., h, :] = o[..., h, :] @ w[(h + 1) % w.shape[0]]"),
+    "up_projection_rows_reversed": ("out[..., h, :] = o[..., h, :] @ w[h]",
+                                    "out[..., h, :] = o[..., h, :] @ w[h][::-1]"),
 }
 
 
