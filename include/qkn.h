@@ -260,6 +260,35 @@ QKN_EXPORT qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, q
                       void* workspace, size_t ws_bytes, void* out, float* lse,
                       const qkn_decode_opts* opts, void* stream);
 
+/* qkn_decode_up — qkn_decode with the per-head value up-projection fused
+ * into the merge of the split-KV partials (GQLA summary, section 2, absorbed
+ * MQA route: on the absorbed path the values are the latents, and each head's
+ * up-projection W^UV_h is applied once to the latent attention output instead
+ * of to every cached token).  For query row i and head h:
+ *   out_v[i,h] = o_lat[i,h] W^UV_h,   lse[i,h] as in qkn_decode,
+ * o_lat[i,h] being qkn_decode's out[i,h]; o_lat is never written to memory.
+ *   Arguments are those of qkn_decode with out replaced by
+ *   w_uv   [H, r_kv, d_v] dtype, 16-byte aligned: W^UV_h = w_uv[h]
+ *   d_v    value head width: a multiple of 16
+ *   out_v  [batch, s_q, H, d_v] dtype (out), 16-byte aligned.
+ * The same workspace serves (qkn_decode_workspace_size).  The merged latent
+ * row is rounded to dtype before the product, as qkn_decode's out is; the
+ * product accumulates in fp32 and is rounded once.  A sequence whose length
+ * breaks its bound gets zero rows of out_v and lse = -inf, recorded as
+ * QKN_ERR_BOUNDS in the status word.
+ * Returns QKN_ERR_INVALID_ARG for a bad d_v or pointer, and
+ * QKN_ERR_UNSUPPORTED when r_kv > 512 or, in bf16, a head's W^UV_h and 32
+ * merged rows do not fit one CTA's shared memory
+ * (r_kv * (d_v + 8) * 2 + 32 * (r_kv + 8) * 2 + 512 bytes <= 227 KB, i.e.
+ * d_v <= 176 at r_kv = 512), before enqueuing anything. */
+QKN_EXPORT qkn_status qkn_decode_up(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode,
+                      const void* q_tilde, const float* a_q, const void* q_rope_hat,
+                      const int32_t* block_table, int32_t max_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t s_q,
+                      const void* w_uv, int32_t d_v,
+                      void* workspace, size_t ws_bytes, void* out_v, float* lse,
+                      const qkn_decode_opts* opts, void* stream);
+
 /* Size of the scratch array that qkn_decode_noalloc uses in place of a
  * caller-allocated workspace.  Every GPU that loads libqkn holds this much
  * device memory for the scratch until the process exits. */

@@ -26,7 +26,7 @@ KERNEL_AUTO, KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1, 2
 
 EXPORTED = ["qkn_append", "qkn_absorb_query", "qkn_decode_workspace_size", "qkn_workspace_init",
             "qkn_decode", "qkn_read_device_status", "qkn_decode_kernel_for", "qkn_status_string",
-            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb", "qkn_key_gram"]
+            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb", "qkn_key_gram", "qkn_decode_up"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "qkn_decode_workspace_size": (I32, [PD, I32, I32, I32, ctypes.POINTER(SZ)]),
         "qkn_workspace_init": (I32, [P, SZ, P]),
         "qkn_decode": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, SZ, P, P, PO, P]),
+        "qkn_decode_up": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, I32, P, SZ, P, P, PO, P]),
         "qkn_read_device_status": (I32, [P, P, ctypes.POINTER(I32)]),
         "qkn_decode_kernel_for": (I32, [PD, I32, PO]),
         "qkn_status_string": (ctypes.c_char_p, [I32]),
@@ -219,6 +220,22 @@ def decode(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_
                            _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens), batch, s_q,
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
                            ctypes.byref(opts), _stream(stream)), "qkn_decode")
+
+
+def decode_up(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_lens, s_q: int, w_uv,
+              workspace: torch.Tensor, out_v, lse, ak_mode: int = AK_CACHE, kernel: int = KERNEL_AUTO,
+              max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0, split_event=None, step_writes_only=False,
+              stream=None) -> None:
+    """The decode step with each head's value up-projection fused into the merge (see qkn_decode_up):
+    ``w_uv`` is [H, r_kv, d_v] in the storage dtype, ``out_v`` [batch, s_q, H, d_v]."""
+    batch = int(block_table.shape[0])
+    max_blocks = int(block_table.shape[1])
+    opts = _opts(kernel, max_ctas, head_tile, wait_limit, split_event, int(bool(step_writes_only)))
+    _check(_lib.qkn_decode_up(ctypes.byref(dims.c()), ctypes.byref(cache.c()), ak_mode, _ptr(q_tilde), _ptr(a_q),
+                              _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens), batch, s_q,
+                              _ptr(w_uv), int(w_uv.shape[-1]), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _ptr(out_v), _ptr(lse),
+                              ctypes.byref(opts), _stream(stream)), "qkn_decode_up")
 
 
 def decode_noalloc(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_lens, s_q: int, out, lse,

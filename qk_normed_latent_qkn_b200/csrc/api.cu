@@ -308,20 +308,37 @@ int32_t qkn_decode_kernel_for(const qkn_dims* dims, int32_t s_q, const qkn_decod
   return pick_kernel(dims, s_q, opts);
 }
 
-qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode, const void* q_tilde,
-                      const float* a_q, const void* q_rope_hat, const int32_t* block_table, int32_t max_blocks,
-                      const int32_t* seq_lens, int32_t batch, int32_t s_q, void* workspace, size_t ws_bytes,
-                      void* out, float* lse, const qkn_decode_opts* opts, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The value up-projection fused into the merge (qkn_decode_up), or none (qkn_decode).
+struct UpProj {
+  const void* w_uv;
+  int32_t d_v;
+  void* out_v;
+};
+
+// qkn_decode and qkn_decode_up: `out` is the latent output, or null when `up` is given.
+qkn_status decode_impl(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode, const void* q_tilde,
+                       const float* a_q, const void* q_rope_hat, const int32_t* block_table, int32_t max_blocks,
+                       const int32_t* seq_lens, int32_t batch, int32_t s_q, void* workspace, size_t ws_bytes,
+                       void* out, float* lse, const UpProj* up, const qkn_decode_opts* opts, void* stream) {
   qkn_status st = check_dims(dims);
   if (st != QKN_OK) return st;
   if ((st = check_cache(dims, cache)) != QKN_OK) return st;
   if (ak_mode != QKN_AK_CACHE && ak_mode != QKN_AK_ONE) return QKN_ERR_INVALID_ARG;
   if (batch < 0 || s_q < 1 || max_blocks < 1) return QKN_ERR_INVALID_ARG;
+  if (up && (up->d_v <= 0 || up->d_v % 16)) return QKN_ERR_INVALID_ARG;
   if (batch == 0) return QKN_OK;
-  if (!q_tilde || !a_q || !q_rope_hat || !block_table || !seq_lens || !workspace || !out || !lse)
+  if (!q_tilde || !a_q || !q_rope_hat || !block_table || !seq_lens || !workspace || !lse)
     return QKN_ERR_INVALID_ARG;
-  if (!aligned(q_tilde, 16) || !aligned(q_rope_hat, 16) || !aligned(workspace, 256) || !aligned(out, 16))
+  if (up ? (!up->w_uv || !up->out_v || !aligned(up->w_uv, 16) || !aligned(up->out_v, 16))
+         : (!out || !aligned(out, 16)))
     return QKN_ERR_INVALID_ARG;
+  if (!aligned(q_tilde, 16) || !aligned(q_rope_hat, 16) || !aligned(workspace, 256)) return QKN_ERR_INVALID_ARG;
+  if (up && !combine_up_supported(dims->dtype == QKN_BF16, dims->r_kv, up->d_v, batch * s_q))
+    return QKN_ERR_UNSUPPORTED;
   if (opts && (opts->max_ctas < 0 || opts->wait_limit < 0 ||
                (opts->head_tile && opts->head_tile != 16 && opts->head_tile != 32 && opts->head_tile != 64 &&
                 opts->head_tile != kPairRows)))
@@ -407,8 +424,39 @@ qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode 
   c.lse = lse;
   c.status = a.status;
   c.seg_desc = kernel == QKN_KERNEL_TCGEN05 ? a.seg_desc : nullptr;
-  e = launch_combine(c, bf16, cs);
+  if (up) {
+    CombineUpArgs u;
+    u.c = c;
+    u.w_uv = up->w_uv;
+    u.d_v = up->d_v;
+    u.out_v = up->out_v;
+    e = launch_combine_up(u, bf16, cs);
+  } else {
+    e = launch_combine(c, bf16, cs);
+  }
   return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+qkn_status qkn_decode(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode, const void* q_tilde,
+                      const float* a_q, const void* q_rope_hat, const int32_t* block_table, int32_t max_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t s_q, void* workspace, size_t ws_bytes,
+                      void* out, float* lse, const qkn_decode_opts* opts, void* stream) {
+  return decode_impl(dims, cache, ak_mode, q_tilde, a_q, q_rope_hat, block_table, max_blocks, seq_lens, batch, s_q,
+                     workspace, ws_bytes, out, lse, nullptr, opts, stream);
+}
+
+qkn_status qkn_decode_up(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode ak_mode, const void* q_tilde,
+                         const float* a_q, const void* q_rope_hat, const int32_t* block_table, int32_t max_blocks,
+                         const int32_t* seq_lens, int32_t batch, int32_t s_q, const void* w_uv, int32_t d_v,
+                         void* workspace, size_t ws_bytes, void* out_v, float* lse, const qkn_decode_opts* opts,
+                         void* stream) {
+  const UpProj up{w_uv, d_v, out_v};
+  return decode_impl(dims, cache, ak_mode, q_tilde, a_q, q_rope_hat, block_table, max_blocks, seq_lens, batch, s_q,
+                     workspace, ws_bytes, nullptr, lse, &up, opts, stream);
 }
 
 qkn_status qkn_read_device_status(const void* workspace, void* stream, int32_t* device_status) {

@@ -617,8 +617,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (pages_of(a.seq_lens[b], sp) != 0) continue;
       if (ts == 0) record_status(a.status, QKN_ERR_BOUNDS);
       for (int ht = ts; ht < a.ht_count; ht += kMathWarps * 32) a.seg_desc[b * a.ht_count + ht] = make_int2(0, 0);
+      // (no latent output when the merge applies the value up-projection: it writes those rows)
       uint4* ob = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * qrows * kRkv);
-      for (int64_t e = ts; e < (int64_t)qrows * kRkv / 8; e += kMathWarps * 32) ob[e] = make_uint4(0, 0, 0, 0);
+      for (int64_t e = ts; a.out && e < (int64_t)qrows * kRkv / 8; e += kMathWarps * 32) ob[e] = make_uint4(0, 0, 0, 0);
       for (int e = ts; e < qrows; e += kMathWarps * 32) a.lse[(int64_t)b * qrows + e] = -INFINITY;
     }
   }

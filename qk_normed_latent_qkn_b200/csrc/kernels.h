@@ -94,6 +94,15 @@ struct CombineArgs {
   const int2* seg_desc;      // per-segment (first slot, splits) from the tcgen05 kernel, or null
 };
 
+// Merge fused with the per-head value up-projection (combine_up.cu): c.out is not used; the merged
+// latent row of (query row i, head h) is multiplied by W^UV_h and written to out_v.
+struct CombineUpArgs {
+  CombineArgs c;
+  const void* w_uv;          // [H, r, d_v] in the storage type
+  int32_t d_v;
+  void* out_v;               // [batch, s_q, H, d_v] in the storage type
+};
+
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_key_gram(const float* w_k, float* gram, int groups, int r, int width, cudaStream_t st);
 // One launch for both (prep.cu) when the append can run as one launch and is a decode step's size.
@@ -102,6 +111,8 @@ cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, c
 cudaError_t launch_absorb(const AbsorbArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_decode_simt(const DecodeArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st);
+bool combine_up_supported(bool bf16, int r, int d_v, int n_q);
+cudaError_t launch_combine_up(const CombineUpArgs& u, bool bf16, cudaStream_t st);
 
 // tcgen05 decode (bf16 only).  Returns cudaErrorNotSupported for dims it
 // cannot take.

@@ -1,8 +1,9 @@
 """Device-resident decode state on top of the C ABI.
 
 A ``DecodeSession`` owns a paged cache, the key up-projection and norm
-weights, the absorbed queries and a decode workspace, and forwards to
-``qkn_append``, ``qkn_absorb_query`` and ``qkn_decode``.  It moves host
+weights, the value up-projection (optional), the absorbed queries and a
+decode workspace, and forwards to ``qkn_append``, ``qkn_absorb_query``,
+``qkn_decode`` and ``qkn_decode_up``.  It moves host
 arrays to the device and nothing else: all arithmetic runs in libqkn.
 """
 from __future__ import annotations
@@ -12,8 +13,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, append_absorb, decode, key_gram,
-               decode_workspace_size, read_device_status, workspace_init)
+from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, append_absorb, decode, decode_up,
+               key_gram, decode_workspace_size, read_device_status, workspace_init)
 
 
 def to_device(x, dtype: torch.dtype, device) -> torch.Tensor:
@@ -28,6 +29,7 @@ class DecodeSession:
         self.device = torch.device(device)
         self.cache = Cache(dims, num_blocks, device=self.device)
         self.w_k = self.key_gram = self.gamma_q = self.gamma_k = self.gamma_qr = self.gamma_kr = None
+        self.w_uv: Optional[torch.Tensor] = None
         self.q_tilde = self.a_q = self.q_rope_hat = None
         self.workspace: Optional[torch.Tensor] = None
 
@@ -42,6 +44,10 @@ class DecodeSession:
         self.gamma_k = to_device(gamma_k, f32, dev)
         self.gamma_qr = to_device(gamma_qr, f32, dev)
         self.gamma_kr = to_device(gamma_kr, f32, dev)
+
+    def load_value_weights(self, w_uv) -> None:
+        """W^UV [H, r_kv, d_v], kept in the storage dtype (the fused merge reads it every step)."""
+        self.w_uv = to_device(w_uv, self.dims.torch_dtype, self.device)
 
     # ------------------------------------------------------------ cache
     def append(self, c, k_rope_raw, slot, pos, chunk: int = 1 << 16) -> None:
@@ -109,6 +115,26 @@ class DecodeSession:
                split_event=split_event, step_writes_only=step_writes_only, test_withhold_ak=test_withhold_ak)
         return out, lse
 
+    def decode_up(self, block_table, seq_lens, s_q: int, out_v=None, lse=None, ak_mode: int = AK_CACHE,
+                  kernel: int = KERNEL_AUTO, max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0,
+                  split_event=None, step_writes_only: bool = False):
+        """The decode step with the value up-projection fused into the merge: o_v [batch, s_q, H, d_v]."""
+        d, dev = self.dims, self.device
+        if self.w_uv is None:
+            raise RuntimeError("decode_up needs load_value_weights first")
+        bt = to_device(block_table, torch.int32, dev)
+        sl = to_device(seq_lens, torch.int32, dev)
+        batch = bt.shape[0]
+        ws = self.ensure_workspace(batch, s_q)
+        if out_v is None:
+            out_v = torch.empty((batch, s_q, d.num_heads, self.w_uv.shape[-1]), dtype=d.torch_dtype, device=dev)
+        if lse is None:
+            lse = torch.empty((batch, s_q, d.num_heads), dtype=torch.float32, device=dev)
+        decode_up(d, self.cache, self.q_tilde, self.a_q, self.q_rope_hat, bt, sl, s_q, self.w_uv, ws, out_v, lse,
+                  ak_mode=ak_mode, kernel=kernel, max_ctas=max_ctas, head_tile=head_tile, wait_limit=wait_limit,
+                  split_event=split_event, step_writes_only=step_writes_only)
+        return out_v, lse
+
     def device_status(self) -> int:
         return read_device_status(self.workspace)
 
@@ -126,6 +152,7 @@ def session_from_inputs(inp, device="cuda", dtype=None) -> DecodeSession:
                 block_size=wl.block_size)
     s = DecodeSession(dims, inp.num_blocks, device=device)
     s.load_weights(inp.w_k, inp.gamma_q, inp.gamma_k, inp.gamma_qr, inp.gamma_kr)
+    s.load_value_weights(inp.w_uv)
     s.append(inp.c, inp.k_rope, inp.token_slots(), inp.token_positions())
     B, s_q = wl.batch, wl.s_q
     s.absorb(inp.q.reshape(B * s_q, wl.heads, wl.d_h), inp.q_rope.reshape(B * s_q, wl.heads, wl.d_rope),

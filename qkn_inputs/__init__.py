@@ -20,9 +20,10 @@ Value recipe (identical for every workload):
   * eps = 1e-6, RoPE base 10000.
 Draw order from one ``numpy.random.Generator(PCG64(seed))``: sequence lengths,
 block permutation, s_t, c, k^R, q, q^R, W^K, gamma_q, gamma_k, gamma_qR,
-gamma_kR.  Values are drawn in fp32 and, for bf16 workloads, the stored
-activations (c, k^R, q, q^R) are rounded once to bf16 (round to nearest even);
-weights and gammas stay fp32.
+gamma_kR, W^UV (value up-projection, N(0, 1/r_kv)).  Values are drawn in fp32
+and, for bf16 workloads, the stored activations (c, k^R, q, q^R) and W^UV
+(which the library reads in the storage type) are rounded once to bf16 (round
+to nearest even); the other weights and the gammas stay fp32.
 """
 from __future__ import annotations
 
@@ -208,7 +209,7 @@ def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
     w_uv = rng.standard_normal((wl.heads, wl.r_kv, wl.d_v), dtype=f32) * f32(1.0 / np.sqrt(wl.r_kv))
 
     if wl.dtype == "bf16":
-        c, k_rope, q, q_rope = (round_to_bf16(a) for a in (c, k_rope, q, q_rope))
+        c, k_rope, q, q_rope, w_uv = (round_to_bf16(a) for a in (c, k_rope, q, q_rope, w_uv))
     elif wl.dtype != "f32":
         raise ValueError(f"unknown dtype {wl.dtype}")
 

@@ -146,3 +146,27 @@ def test_append_absorb_validates_both_halves_before_any_launch():
     # negative counts
     assert lib.qkn_append_absorb(ctypes.byref(dims), ctypes.byref(cache), P, P, P, P, -1, P, P, P, 1,
                                  P, None, P, P, P, P, P, P, P, None) == qkn.ERR_INVALID_ARG
+
+
+def _decode_up(lib, dims, w_uv, d_v, out_v, batch=1):
+    cache = qkn._Cache(0x1000, 0x2000, 0x3000, 4)
+    return lib.qkn_decode_up(ctypes.byref(dims), ctypes.byref(cache), 0, 0x100, 0x100, 0x100, 0x100, 1, 0x100,
+                             batch, 1, w_uv, d_v, 0x100, 1 << 30, out_v, 0x100, None, None)
+
+
+def test_decode_up_validates_the_value_projection_before_any_launch():
+    lib = qkn.raw_library()
+    dims = DIMS.c()
+    for d_v in (0, -16, 8, 100):                 # d_v must be a positive multiple of 16
+        assert _decode_up(lib, dims, 0x100, d_v, 0x100) == qkn.ERR_INVALID_ARG
+    assert _decode_up(lib, dims, None, 128, 0x100) == qkn.ERR_INVALID_ARG       # no W^UV
+    assert _decode_up(lib, dims, 0x100, 128, None) == qkn.ERR_INVALID_ARG       # no output
+    assert _decode_up(lib, dims, 0x108, 128, 0x100) == qkn.ERR_INVALID_ARG      # misaligned W^UV
+    assert _decode_up(lib, dims, 0x100, 128, 0x104) == qkn.ERR_INVALID_ARG      # misaligned output
+    assert _decode_up(lib, dims, 0x100, 128, 0x100, batch=0) == qkn.OK          # empty batch: no-op
+    # W^UV_h and 32 merged rows must fit one CTA's shared memory: d_v = 176 is the widest at
+    # r_kv = 512 in bf16; r_kv above 512 is not taken
+    assert _decode_up(lib, dims, 0x100, 192, 0x100) == qkn.ERR_UNSUPPORTED
+    import dataclasses
+    wide = dataclasses.replace(DIMS, r_kv=1024).c()
+    assert _decode_up(lib, wide, 0x100, 64, 0x100) == qkn.ERR_UNSUPPORTED
