@@ -274,7 +274,7 @@ def oracle_throughput(inp, budget_s: float, max_seqs=None):
 def run_ours(args, world, rank, local):
     import torch
     import qk_normed_latent_qkn_b200 as qkn
-    from qk_normed_latent_qkn_b200.roofline import decode_step_cost
+    from qk_normed_latent_qkn_b200.roofline import decode_step_cost, merge_cost, split_counts
     from qk_normed_latent_qkn_b200.session import DecodeSession, session_from_inputs
     from qkn_inputs import WORKLOADS, make_inputs
 
@@ -309,11 +309,14 @@ def run_ours(args, world, rank, local):
         s.cache.k_rope.copy_(base.cache.k_rope)
         s.cache.a_k.copy_(base.cache.a_k)
         s.load_weights(base.w_k, base.gamma_q, base.gamma_k, base.gamma_qr, base.gamma_kr)
+        s.w_uv = base.w_uv.clone()             # its own W^UV, so that no copy finds it in L2
         sessions.append(s)
     dev_in = [{k: torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=types[k]) for k, v in
                host.items()} for _ in sessions]
     outs = [(torch.empty((B, s_q, H, wl.r_kv), dtype=dt, device=device),
              torch.empty((B, s_q, H), dtype=torch.float32, device=device)) for _ in sessions]
+    outs_v = [(torch.empty((B, s_q, H, wl.d_v), dtype=dt, device=device),
+               torch.empty((B, s_q, H), dtype=torch.float32, device=device)) for _ in sessions]
 
     evs = torch.cuda.Stream(device=device)
 
@@ -339,6 +342,11 @@ def run_ours(args, world, rank, local):
         s.decode(d["bt"], d["sl"], s_q, out=o, lse=l, ak_mode=ak_mode, kernel=kernel, split_event=split_event,
                  head_tile=args.head_tile)
 
+    def decode_up_only(i, split_event=None):
+        s, d, (ov, l) = sessions[i], dev_in[i], outs_v[i]
+        s.decode_up(d["bt"], d["sl"], s_q, out_v=ov, lse=l, kernel=kernel, split_event=split_event,
+                    head_tile=args.head_tile)
+
     ev = Events()
     stream = torch.cuda.Stream(device=device)
 
@@ -346,6 +354,7 @@ def run_ours(args, world, rank, local):
     for i in range(len(sessions)):
         step(i)
         step(i, ak_mode=qkn.AK_ONE)
+        decode_up_only(i)
     torch.cuda.synchronize(device)
     status = [s.device_status() for s in sessions]
     assert all(v == qkn.OK for v in status), f"device status {status}"
@@ -380,6 +389,17 @@ def run_ours(args, world, rank, local):
                     ev.record(e[2], stream.cuda_stream)
                 lst.append((g, e))
             over[mode] = lst
+        # decode-only graphs with the value up-projection fused into the merge: events before the
+        # split-KV kernel, between it and the fused merge, and after
+        up_graphs = []
+        for i in range(n_copies):
+            e = [ev.create() for _ in range(3)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                ev.record(e[0], stream.cuda_stream)
+                decode_up_only(i, split_event=e[1])
+                ev.record(e[2], stream.cuda_stream)
+            up_graphs.append((g, e))
     torch.cuda.synchronize(device)
 
     soak_graphs = graphs[:n_copies] if len(graphs) >= n_copies else graphs
@@ -442,7 +462,7 @@ def run_ours(args, world, rank, local):
     # overhead vs plain MLA: interleaved rounds of decode-only graphs; the same replays give the
     # split-KV kernel's launch duration for the roofline and the split + merge op
     per_mode = {qkn.AK_CACHE: [], qkn.AK_ONE: []}
-    op_only = []
+    op_only, merge_only, up_merge, up_op = [], [], [], []
     with torch.cuda.stream(stream):
         for _ in range(args.overhead_rounds):
             for mode in (qkn.AK_CACHE, qkn.AK_ONE):
@@ -452,6 +472,12 @@ def run_ours(args, world, rank, local):
                 per_mode[mode] += [ev.ms(e[0], e[1]) for _g, e in over[mode]]
                 if mode == qkn.AK_CACHE:
                     op_only += [ev.ms(e[0], e[2]) for _g, e in over[mode]]
+                    merge_only += [ev.ms(e[1], e[2]) for _g, e in over[mode]]
+            for g, _e in up_graphs:
+                g.replay()
+            stream.synchronize()
+            up_merge += [ev.ms(e[1], e[2]) for _g, e in up_graphs]
+            up_op += [ev.ms(e[0], e[2]) for _g, e in up_graphs]
     t_qkn = statistics.median(per_mode[qkn.AK_CACHE])
     t_mla = statistics.median(per_mode[qkn.AK_ONE])
     t_split_avg = statistics.mean(per_mode[qkn.AK_CACHE])
@@ -495,6 +521,14 @@ def run_ours(args, world, rank, local):
     op_only_avg = statistics.mean(op_only)
     tokens = world * B * s_q
     traffic = load_traffic(wl.name) if kernel_used == qkn.KERNEL_TCGEN05 else None
+    # the merge kernels' rooflines: partial rows read per the split schedule of this launch
+    rows_t, ncta_t, item_cost_t = schedule_shape(kernel_used, args.head_tile, s_q, H,
+                                                 torch.cuda.get_device_properties(device).multi_processor_count)
+    splits = split_counts(inp.seq_lens, s_q, inp.block_table.shape[1], -(-s_q * H // rows_t), ncta_t, item_cost_t)
+    elem = 2 if wl.dtype == "bf16" else 4
+    m_plain = merge_cost(splits, s_q, H, wl.r_kv, elem)
+    m_up = merge_cost(splits, s_q, H, wl.r_kv, elem, d_v=wl.d_v)
+    t_merge, t_up = statistics.mean(merge_only), statistics.mean(up_merge)
 
     line = None
     if rank == 0:
@@ -542,6 +576,22 @@ def run_ours(args, world, rank, local):
                          "decode_op_frac": cost.bytes / (op_only_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                     "frac": tflops / peaks["bf16_tflops"], "flops": cost.flops}},
+            "value_up": {
+                "d_v": wl.d_v, "op_us": statistics.mean(up_op) * 1e3, "merge_up_us": t_up * 1e3,
+                "merge_us": t_merge * 1e3,
+                "roofline": {"bound": "hbm", "achieved": m_up.bytes / (t_up * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": m_up.bytes / (t_up * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "algorithmic_bytes": m_up.bytes, "partial_bytes": m_up.partial_bytes,
+                             "weight_bytes": m_up.weight_bytes, "flops": m_up.flops},
+                "merge_roofline": {"bound": "hbm", "achieved": m_plain.bytes / (t_merge * 1e-3) / 1e9,
+                                   "frac": m_plain.bytes / (t_merge * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                   "algorithmic_bytes": m_plain.bytes},
+                "what": ("qkn_decode_up replayed alone in decode-only graphs (same rounds as the overhead "
+                         "figure): op_us = split-KV kernel + merge fused with the W^UV up-projection; "
+                         "merge_up_us = the fused merge kernel alone (event after the split-KV kernel); "
+                         "merge_us = qkn_decode's plain merge kernel, measured the same way; bytes = fp32 "
+                         "partial rows read per the split schedule + W^UV once + outputs written once"),
+            },
             "overhead_vs_mla": {"qkn_us": t_qkn * 1e3, "mla_us": t_mla * 1e3, "frac": t_qkn / t_mla - 1.0,
                                 "what": "decode split kernel, a_k cache vs a_k = 1, median of interleaved rounds"},
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
@@ -553,6 +603,18 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu,
         }
     return line
+
+
+def schedule_shape(kernel_used: int, head_tile: int, s_q: int, heads: int, sms: int):
+    """Row tile, schedule CTAs and item cost of the decode's split schedule for this launch (the C-ABI
+    layer's choice restated for cost accounting; 128-row tiles on CTA pairs count sms / 2 pairs)."""
+    import qk_normed_latent_qkn_b200 as qkn
+    if kernel_used != qkn.KERNEL_TCGEN05:
+        return 8, sms, 1
+    qrows = s_q * heads
+    rows = head_tile or (16 if qrows <= 16 else 32 if qrows <= 32 else 64)
+    ncta = sms // 2 if rows == 128 else sms
+    return rows, ncta, 3 if rows >= 64 else rows // 16
 
 
 # ----------------------------------------------------------------- reference arm (the oracle)

@@ -56,3 +56,56 @@ def decode_step_cost(seq_lens: Sequence[int], s_q: int, heads: int, groups: int,
         output_bytes=rows * (elem * r + 4),
         flops=pairs * heads * flops_per_token_row(r, d_rope),
     )
+
+
+# ----------------------------------------------------------------- the merge of the split-KV partials
+def split_counts(seq_lens: Sequence[int], s_q: int, max_blocks: int, ht_count: int, ncta: int,
+                 item_cost: int, block: int = 64) -> list:
+    """Splits (partial results) of each sequence's segments under the decode's split schedule.
+
+    Host restatement of the schedule for cost accounting: sequence b is item_cost + n(b) units
+    (n(b) pages; none for a rejected length), laid out one after another; the CTAs form
+    G = ncta // min(HT, ncta) groups, group g takes units [g Q, (g + 1) Q), Q = ceil(total / G); a
+    segment is split wherever a group boundary falls inside its pages.  Every row tile of a
+    sequence has the same count.
+    """
+    n = [0 if (int(L) < s_q or int(L) > max_blocks * block) else -(-int(L) // block) for L in seq_lens]
+    units = [x + item_cost if x > 0 else 0 for x in n]
+    total = sum(units)
+    hc = min(ht_count, ncta)
+    groups = max(1, ncta // max(hc, 1))
+    q = max(1, -(-total // groups))
+    out, u0 = [], 0
+    for nb, ub in zip(n, units):
+        if nb == 0:
+            out.append(0)
+        else:
+            pg0 = u0 + item_cost
+            out.append((pg0 + nb - 1) // q - pg0 // q + 1)
+        u0 += ub
+    return out
+
+
+@dataclasses.dataclass(frozen=True)
+class MergeCost:
+    partial_bytes: int     # fp32 partial rows and their lse, read once
+    weight_bytes: int      # W^UV (fused merge only), read once
+    output_bytes: int      # merged rows (or o_v) and lse, written once
+    flops: int             # the up-projection (fused merge only)
+
+    @property
+    def bytes(self) -> int:
+        return self.partial_bytes + self.weight_bytes + self.output_bytes
+
+
+def merge_cost(splits: Sequence[int], s_q: int, heads: int, r: int, elem: int = 2, d_v: int = 0) -> MergeCost:
+    """Bytes of the merge of one step: every query row reads its splits' fp32 partial row (4 r bytes)
+    and lse (4 bytes).  d_v = 0: the plain merge writes the latent row (elem r bytes) and lse.
+    d_v > 0: the merge fused with the value up-projection also reads W^UV once (heads r d_v elements)
+    and writes o_v (elem d_v bytes per row) and lse, at 2 r d_v FLOPs per row."""
+    rows_per_seq = s_q * heads
+    parts = sum(int(x) for x in splits) * rows_per_seq
+    rows = len(splits) * rows_per_seq
+    width = d_v if d_v else r
+    return MergeCost(partial_bytes=parts * (4 * r + 4), weight_bytes=heads * r * d_v * elem,
+                     output_bytes=rows * (elem * width + 4), flops=2 * rows * r * d_v)

@@ -107,3 +107,20 @@ def test_workspace_holds_the_slots():
             ht = -(-s_q * heads // rows)
             need = (batch * ht + ncta) * rows * (512 + 1) * 4        # partial O and lse, fp32
             assert ws >= need, (batch, s_q, heads, rows, ws, need)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_cost_accounting_split_counts_match_the_schedule(seed):
+    # the benchmark's merge byte count takes its split counts from roofline.split_counts: they must be
+    # the number of items each segment gets under the schedule's definition
+    from qk_normed_latent_qkn_b200.roofline import split_counts
+    rng = random.Random(1000 + seed)
+    batch, s_q, max_blocks = rng.randint(1, 40), rng.choice([1, 2]), rng.randint(1, 40)
+    lens = [rng.randint(s_q, max_blocks * BLOCK) if rng.random() > 0.1 else rng.choice([0, max_blocks * BLOCK + 1])
+            for _ in range(batch)]
+    ht_count, ncta, item_cost = rng.choice([1, 2, 3, 4, 16]), rng.choice([1, 2, 3, 5, 7, 64, 148]), rng.choice([0, 3])
+    items, _n, _starts, _q = schedule(lens, s_q, max_blocks, ht_count, ncta, item_cost)
+    counts = split_counts(lens, s_q, max_blocks, ht_count, ncta, item_cost)
+    for b in range(batch):
+        for ht in range(ht_count):
+            assert sum(1 for it in items if it[0] == b and it[1] == ht) == counts[b]
