@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(kRmsCols * kRmsSlices, 2) append_keyrms_kernel
   // dependents may launch only once everything before this kernel is complete (see prep.cu)
   pdl_wait();
   pdl_trigger();
-  keyrms_block<T, TT, FUSED>(a, blockIdx.x, blockIdx.y, blockIdx.z, reinterpret_cast<float*>(smem4));
+  __shared__ float rows[kRmsCols * kRmsSlices / 32][128];
+  keyrms_block<T, TT, FUSED>(a, blockIdx.x, blockIdx.y, blockIdx.z, reinterpret_cast<float*>(smem4), rows);
 }
 
 __global__ void append_finalize_kernel(AppendArgs a) {

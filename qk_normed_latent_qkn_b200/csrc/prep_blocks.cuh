@@ -96,8 +96,10 @@ constexpr int kRmsSlices = 32;
 // accumulator in ak_scratch and count themselves in, and the CTA whose count
 // completes a token writes a_k = 1 / sqrt(sum / width + eps) and returns the
 // accumulator and the count to zero.
+// `rows`: a 128-float buffer per warp (kRmsCols * kRmsSlices / 32 of them) for the copy column.
 template <typename T, int TT, bool FUSED>
-__device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by, int bz, float* smem) {
+__device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by, int bz, float* smem,
+                                             float (*rows)[128]) {
   float* cs = smem;                                               // [TT][r]
   float* zp = cs + TT * a.r;                                      // [kRmsSlices][TT][kRmsCols]
   const int g = bz;
@@ -110,7 +112,6 @@ __device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by
   const int nblk = (ncols + kRmsCols - 1) / kRmsCols;
   if constexpr (FUSED) {
     if (bx == nblk) {
-      __shared__ float rows[kRmsCols * kRmsSlices / 32][128];
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
       if (bz == 0)
         for (int i = warp; i < ntok; i += kRmsCols * kRmsSlices / 32) append_token<T>(a, t0 + i, lane, rows[warp]);
@@ -272,124 +273,115 @@ __device__ __forceinline__ void mma_tf32_m16n8k8(float (&d)[4], const uint32_t (
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Latent rows of W^K_{g,h} per absorption CTA of NW warps, and its shared memory.
-template <int NW>
-__host__ __device__ constexpr int absorb_rows() { return NW * 8; }
-inline size_t absorb_smem_bytes(int rows, int d_h) {
-  return ((size_t)rows * (d_h + 4) + (size_t)kAbsQ * (d_h + 4) + (size_t)d_h) * sizeof(float);
+// a_q and the rotated RoPE query of every query row of head h, one warp per row.
+template <typename T, int NW>
+__device__ __forceinline__ void absorb_head_rows(const AbsorbArgs& a, int h, float (*rows)[128]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < a.n_q; i += NW) absorb_row<T>(a, i, h, rows[warp], lane);
 }
 
-// CTA (h, y < last) of the absorption grid (H, ceil(r / KB) + 1), NW warps,
-// KB = 8 NW latent rows: stages its KB x d_h slice of W^K_{g,h} once, with
-// gamma_q * gamma_k folded into its columns, and computes q~[i, h, k] for its
-// latent rows k and every query row i, kAbsQ query rows per pass.  Warp w
-// takes 16 rows (w mod NW/2) and 16 query rows (w div NW/2) of a pass; lane
-// (rg, qg) = (lane % 8, lane / 8) takes rows rg, rg + 8 and query rows qg,
-// qg + 4, qg + 8, qg + 12 of those: per 4 columns of d_h it reads 2 W and 4
-// query vectors (16 bytes each) for 32 FMAs, and with row pitch d_h + 4 the
-// 8 distinct rows (and 4 distinct query rows) of one read fall in distinct
-// banks, so every read is one shared-memory wavefront.  The slice, the gamma
-// product and the first pass's queries are loaded in one round.  The CTA with
-// y == last produces a_q and the RoPE query of head h.
-template <typename T, int NW>
-__device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by, float* smem) {
-  constexpr int kThreadsAbs = NW * 32;
-  constexpr int KB = absorb_rows<NW>();
-  constexpr int kRowWarps = NW / 2;
-  static_assert(kRowWarps * 16 == KB && kAbsQ == 32, "warp tiling of the absorption CTA");
-  // bf16 storage: q~ is rounded to bf16 anyway, so the products run on the tensor cores in TF32
-  // (10-bit mantissa, fp32 accumulation); fp32 storage keeps fp32 FMAs
-  constexpr bool kTensor = std::is_same<T, __nv_bfloat16>::value;
-  const int pitch = a.d_h + 4;
-  float* wc = smem;                                        // [KB][d_h + 4]
-  float* sv = wc + KB * pitch;                             // [kAbsQ][d_h + 4]
-  float* g2 = sv + kAbsQ * pitch;                          // [d_h] gamma_q * gamma_k of head h
-  const int h = bx;
-  const int nkb = (a.r + KB - 1) / KB;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (by == nkb) {
-    __shared__ float rowbuf[NW][128];
-    for (int i = warp; i < a.n_q; i += NW) absorb_row<T>(a, i, h, rowbuf[warp], lane);
-    return;
-  }
-  const int kbase = by * KB;
-  const int ng = a.heads / a.groups;
-  const int g = h / ng, m = h - g * ng;
-  const int width = ng * a.d_h;
+// ---------------------------------------------------------------- absorption units
+// The absorption q~[i, h] = W^K_{g,h} (gamma_q[h] gamma_k[h] q[i, h]) as units (head h, KB = 8 NW
+// latent rows from kbase = kc KB), unit j = h ceil(r / KB) + kc, for CTAs of NW warps.  A unit's
+// slice of W^K_{g,h} (KB rows of d_h contiguous fp32 values) is copied raw with 16-byte cp.async
+// (no register staging) into a W buffer; gamma_q gamma_k is folded into the staged query rows
+// instead of into W (the same products in another order).  For bf16 storage the products run on
+// the tensor cores in TF32 (fp32 accumulation): the query rows are rounded to TF32, the raw W
+// values are truncated to it by the MMA (relative error below 2^-10, beside the bf16 rounding of
+// q~ at 2^-9); fp32 storage keeps fp32 FMAs.  a_q and the RoPE query of head h come from
+// absorb_head_rows, or from the kc == 0 unit.
+//
+// Shared memory (floats, row pitch d_h + 4 so that the 8 rows of a fragment read fall in distinct
+// banks): nbuf W buffers [KB][d_h + 4], the query rows [kAbsQ][d_h + 4], gamma_q gamma_k [d_h].
+template <int NW>
+__host__ __device__ constexpr int absorb_unit_rows() { return NW * 8; }
+template <int NW>
+inline size_t absorb_unit_floats(int d_h, int nbuf) {
+  return (size_t)(nbuf * absorb_unit_rows<NW>() + kAbsQ) * (d_h + 4) + d_h;
+}
+template <int NW>
+__host__ __device__ inline int absorb_units(int heads, int r) {
+  return heads * ((r + absorb_unit_rows<NW>() - 1) / absorb_unit_rows<NW>());
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  if (n > 0) asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Issue the copies of unit j's slice of W^K into `wb` and commit them as one group (every thread
+// commits, possibly an empty group).  Rows past r are not copied (their outputs are not stored).
+template <int NW>
+__device__ __forceinline__ void absorb_load_w(const AbsorbArgs& a, int j, float* wb) {
+  constexpr int KB = absorb_unit_rows<NW>(), kT = NW * 32;
+  const int nkc = (a.r + KB - 1) / KB;
+  const int h = j / nkc, kbase = (j - h * nkc) * KB;
+  const int ng = a.heads / a.groups, g = h / ng, m = h - g * ng;
+  const int width = ng * a.d_h, pitch = a.d_h + 4, dq = a.d_h / 4;
   const float* w = a.w_k + (int64_t)g * a.r * width + (int64_t)m * a.d_h;
-  const int dq = a.d_h / 4;
+  const int nrows = min(KB, a.r - kbase);
+  for (int e = threadIdx.x; e < nrows * dq; e += kT) {
+    const int rr = e / dq, d4 = e - rr * dq;
+    cp_async16(wb + rr * pitch + d4 * 4, w + (int64_t)(kbase + rr) * width + d4 * 4);
+  }
+  cp_async_commit();
+}
+
+// Zero the 4 pad columns of every W and query row once per kernel: the TF32 loop reads them when
+// d_h % 8 == 4, and the copies never write them.
+template <int NW>
+__device__ __forceinline__ void absorb_zero_pads(const AbsorbArgs& a, float* abs_smem, int nbuf) {
+  const int pitch = a.d_h + 4;
+  for (int rr = threadIdx.x; rr < nbuf * absorb_unit_rows<NW>() + kAbsQ; rr += NW * 32)
+    *reinterpret_cast<float4*>(abs_smem + rr * pitch + a.d_h) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Unit j with its W slice in `wb` (its copies committed as the older of at most `pending` + 1
+// outstanding groups of this thread).  Starts and ends with the CTA's query rows and gamma
+// buffers free; ends with a barrier, after which `wb` may be refilled.
+// `rows`: a 128-float buffer per warp, for the a_q / RoPE rows when the kc == 0 unit does them
+// (rows_too); otherwise absorb_head_rows does them separately.
+template <typename T, int NW>
+__device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const float* wb, float* sv, float* g2,
+                                            int pending, float (*rows)[128], bool rows_too) {
+  constexpr int kThreadsAbs = NW * 32;
+  constexpr int KB = absorb_unit_rows<NW>();
+  constexpr int kRowWarps = NW / 2;
+  static_assert(kRowWarps * 16 == KB && kAbsQ == 32, "warp tiling of the absorption unit");
+  constexpr bool kTensor = std::is_same<T, __nv_bfloat16>::value;
+  const int pitch = a.d_h + 4, dq = a.d_h / 4;
+  const int nkc = (a.r + KB - 1) / KB;
+  const int h = j / nkc, kc = j - h * nkc, kbase = kc * KB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const T* q = static_cast<const T*>(a.q);
   T* out = static_cast<T*>(a.q_tilde);
-  // stage query rows [i0, i0 + nq) of head h as fp32 (zeros past nq)
+  // stage query rows [i0, i0 + nq) of head h times gamma_q gamma_k (zeros past nq); g2 is ready
   auto stage_q = [&](int i0, int nq) {
-    constexpr int kB = 2;
-    for (int e0 = threadIdx.x; e0 < kAbsQ * dq; e0 += kB * kThreadsAbs) {
-      float4 v[kB];
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int e = e0 + u * kThreadsAbs;
-        const int qi = e / dq, d4 = e - qi * dq;
-        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (e < kAbsQ * dq && qi < nq) {
-          const T* src = q + ((int64_t)(i0 + qi) * a.heads + h) * a.d_h + d4 * 4;
-          v[u] = make_float4(to_f32(src[0]), to_f32(src[1]), to_f32(src[2]), to_f32(src[3]));
-        }
+    for (int e = threadIdx.x; e < kAbsQ * dq; e += kThreadsAbs) {
+      const int qi = e / dq, d4 = e - qi * dq;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (qi < nq) {
+        const T* src = q + ((int64_t)(i0 + qi) * a.heads + h) * a.d_h + d4 * 4;
+        const float4 gg = reinterpret_cast<const float4*>(g2)[d4];
+        v = make_float4(to_f32(src[0]) * gg.x, to_f32(src[1]) * gg.y, to_f32(src[2]) * gg.z, to_f32(src[3]) * gg.w);
+        if constexpr (kTensor) v = make_float4(round_tf32(v.x), round_tf32(v.y), round_tf32(v.z), round_tf32(v.w));
       }
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int e = e0 + u * kThreadsAbs;
-        if (e < kAbsQ * dq) {
-          const int qi = e / dq, d4 = e - qi * dq;
-          *reinterpret_cast<float4*>(sv + qi * pitch + d4 * 4) = v[u];
-        }
-      }
+      *reinterpret_cast<float4*>(sv + qi * pitch + d4 * 4) = v;
     }
   };
-  // the slice times the gamma product: all of a thread's loads go out before its first store
-  {
-    constexpr int kB = 8;
-    float4 wv[kB];
-    const int total = KB * dq;
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int e = threadIdx.x + u * kThreadsAbs;
-      const int rr = e / dq, d4 = e - rr * dq;
-      wv[u] = (e < total && kbase + rr < a.r)
-                  ? *reinterpret_cast<const float4*>(w + (int64_t)(kbase + rr) * width + d4 * 4)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float4 gq = make_float4(0.f, 0.f, 0.f, 0.f), gk = gq;
-    if ((int)threadIdx.x < dq) {
-      gq = *reinterpret_cast<const float4*>(a.gamma_q + h * a.d_h + threadIdx.x * 4);
-      gk = *reinterpret_cast<const float4*>(a.gamma_k + h * a.d_h + threadIdx.x * 4);
-    }
-    stage_q(0, min(kAbsQ, a.n_q));
-    // the 4 pad columns of every W and query row stay zero: the TF32 loop reads them when d_h % 8 == 4
-    for (int rr = threadIdx.x; rr < KB + kAbsQ; rr += kThreadsAbs)
-      *reinterpret_cast<float4*>(wc + rr * pitch + a.d_h) = make_float4(0.f, 0.f, 0.f, 0.f);
-    if ((int)threadIdx.x < dq)
-      reinterpret_cast<float4*>(g2)[threadIdx.x] = make_float4(gq.x * gk.x, gq.y * gk.y, gq.z * gk.z, gq.w * gk.w);
-    __syncthreads();
-    auto store_w = [&](int e, const float4& v) {
-      const int rr = e / dq, d4 = e - rr * dq;
-      const float4 gg = reinterpret_cast<const float4*>(g2)[d4];
-      float4 x = make_float4(v.x * gg.x, v.y * gg.y, v.z * gg.z, v.w * gg.w);
-      if constexpr (kTensor) x = make_float4(round_tf32(x.x), round_tf32(x.y), round_tf32(x.z), round_tf32(x.w));
-      *reinterpret_cast<float4*>(wc + rr * pitch + d4 * 4) = x;
-    };
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int e = threadIdx.x + u * kThreadsAbs;
-      if (e < total) store_w(e, wv[u]);
-    }
-    // d_h > 4 * kB * kThreadsAbs / KB: the rest of the slice, one vector at a time
-    for (int e = threadIdx.x + kB * kThreadsAbs; e < total; e += kThreadsAbs) {
-      const int rr = e / dq, d4 = e - rr * dq;
-      const float4 v = kbase + rr < a.r ? *reinterpret_cast<const float4*>(w + (int64_t)(kbase + rr) * width + d4 * 4)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      store_w(e, v);
-    }
+  if ((int)threadIdx.x < dq) {
+    const float4 gq = *reinterpret_cast<const float4*>(a.gamma_q + h * a.d_h + threadIdx.x * 4);
+    const float4 gk = *reinterpret_cast<const float4*>(a.gamma_k + h * a.d_h + threadIdx.x * 4);
+    reinterpret_cast<float4*>(g2)[threadIdx.x] = make_float4(gq.x * gk.x, gq.y * gk.y, gq.z * gk.z, gq.w * gk.w);
   }
+  __syncthreads();
+  stage_q(0, min(kAbsQ, a.n_q));
+  cp_async_wait_pending(pending);                        // this unit's W slice has landed
   const int rw = warp % kRowWarps, qw = warp / kRowWarps;
   for (int i0 = 0; i0 < a.n_q; i0 += kAbsQ) {
     const int nq = min(kAbsQ, a.n_q - i0);
@@ -403,9 +395,8 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
       // m16n8k8 TF32 products: A = 16 rows of the slice, B = 8 query rows, per 8 columns of d_h.
       // Fragments (lane = 4 gid + tig): A holds (row gid | gid + 8, column tig | tig + 4), B
       // (query row gid, column tig | tig + 4), D (row gid | gid + 8, query row 2 tig | 2 tig + 1).
-      // With row pitch d_h + 4 the 32 lanes of every fragment read hit 32 distinct banks.
       const int gid = lane >> 2, tig = lane & 3;
-      const float* wa = wc + (rw * 16 + gid) * pitch + tig;
+      const float* wa = wb + (rw * 16 + gid) * pitch + tig;
       const float* qb = sv + (qw * 16 + gid) * pitch + tig;
       float dacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 4
@@ -413,28 +404,27 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
         const uint32_t af[4] = {__float_as_uint(wa[d]), __float_as_uint(wa[8 * pitch + d]),
                                 __float_as_uint(wa[d + 4]), __float_as_uint(wa[8 * pitch + d + 4])};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint32_t bf[2] = {__float_as_uint(qb[j * 8 * pitch + d]), __float_as_uint(qb[j * 8 * pitch + d + 4])};
-          mma_tf32_m16n8k8(dacc[j], af, bf);
+        for (int jj = 0; jj < 2; ++jj) {
+          const uint32_t bf[2] = {__float_as_uint(qb[jj * 8 * pitch + d]), __float_as_uint(qb[jj * 8 * pitch + d + 4])};
+          mma_tf32_m16n8k8(dacc[jj], af, bf);
         }
       }
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int jj = 0; jj < 2; ++jj) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int row = rw * 16 + gid + (e >> 1) * 8;
-          const int qi = qw * 16 + j * 8 + 2 * tig + (e & 1);
+          const int qi = qw * 16 + jj * 8 + 2 * tig + (e & 1);
           if (qi < nq && kbase + row < a.r)
-            out[((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase + row] = from_f32<T>(dacc[j][e]);
+            out[((int64_t)(i0 + qi) * a.heads + h) * a.r + kbase + row] = from_f32<T>(dacc[jj][e]);
         }
       }
     } else {
-      // fp32 storage keeps fp32 FMAs: lane (rg, qg) = (lane % 8, lane / 8) takes rows rg, rg + 8
-      // of the warp's 16 and query rows qg, qg + 4, qg + 8, qg + 12: per 4 columns of d_h 2 W and
-      // 4 query vectors (16 bytes each, one wavefront per read) for 32 FMAs
+      // fp32 FMAs: lane (rg, qg) = (lane % 8, lane / 8) takes rows rg, rg + 8 of the warp's 16 and
+      // query rows qg, qg + 4, qg + 8, qg + 12: per 4 columns of d_h 2 W and 4 query vectors
       const int rg = lane & 7, qg = lane >> 3;
       const int k0 = rw * 16 + rg;
-      const float* wrow0 = wc + k0 * pitch;
+      const float* wrow0 = wb + k0 * pitch;
       const float* wrow1 = wrow0 + 8 * pitch;
       const float* qrow = sv + (qw * 16 + qg) * pitch;
       float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -460,6 +450,11 @@ __device__ __forceinline__ void absorb_block(const AbsorbArgs& a, int bx, int by
       }
     }
   }
+  if (kc == 0 && rows_too) {
+    // a_q and the rotated RoPE query of head h, one warp per query row
+    for (int i = warp; i < a.n_q; i += NW) absorb_row<T>(a, i, h, rows[warp], lane);
+  }
+  __syncthreads();
 }
 
 }  // namespace qkn
