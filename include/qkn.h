@@ -142,6 +142,15 @@ typedef struct {
                               MMAs in flight are waited for, tensor memory is freed) and the merge
                               writes no partial it cannot vouch for.  It exercises the timeout path
                               without faulting or hanging the GPU.  Ignored with QKN_AK_ONE.  0 in use. */
+  const int32_t* vis_end;  /* optional DEVICE array [batch]: where each sequence ends for the causal
+                              limit, in this call's token numbering (token t of sequence b is the
+                              t-th token of the pages block_table[b] lists).  Query j of sequence b
+                              sees the tokens t <= vis_end[b] - s_q + j among the seq_lens[b] tokens
+                              the call covers.  For a call that covers only part of a sequence's
+                              pages (context parallelism: block_table[b] starts at the slice's first
+                              page and seq_lens[b] counts the slice's tokens), vis_end[b] is the
+                              sequence's length counted from that first page, so the limit stays the
+                              whole sequence's.  NULL (default): vis_end = seq_lens. */
 } qkn_decode_opts;
 
 /* qkn_key_gram — G_g = W^K_g (W^K_g)^T for every group g, the r_kv x r_kv
@@ -322,6 +331,24 @@ QKN_EXPORT qkn_status qkn_decode_noalloc(const qkn_dims* dims, const qkn_cache* 
                       const int32_t* seq_lens, int32_t batch, int32_t s_q,
                       void* out, float* lse, int32_t* device_status,
                       const qkn_decode_opts* opts, void* stream);
+
+/* qkn_merge_partials — merge partial decode results of the same query rows.
+ * For context-parallel decoding (each rank decodes a slice of every
+ * sequence's pages, with qkn_decode_opts.vis_end, and the ranks' outputs
+ * are all-gathered) the slices' results combine by the same identity as the
+ * split-KV merge: for every row
+ *   lse = log sum_p exp(lse_p),   out = sum_p exp(lse_p - lse) parts[p]
+ * (the softmax over the union of the slices' tokens; QKN summary, decode-logit
+ * equation, whose softmax runs over all cached tokens).
+ *   parts     [n_parts, rows, r_kv] dtype, 16-byte aligned (each part as
+ *             qkn_decode writes out: normalised over the part's tokens)
+ *   lse_parts [n_parts, rows] fp32 (-inf: the part saw no token of the row)
+ *   out       [rows, r_kv] dtype, 16-byte aligned; lse [rows] fp32
+ * rows = batch * s_q * num_heads.  A row with no visible token in any part
+ * gets zeros and lse = -inf.  Returns QKN_ERR_INVALID_ARG for n_parts < 1,
+ * rows < 0 or a missing or misaligned pointer; rows == 0 is a no-op. */
+QKN_EXPORT qkn_status qkn_merge_partials(const qkn_dims* dims, int32_t n_parts, int64_t rows, const void* parts,
+                      const float* lse_parts, void* out, float* lse, void* stream);
 
 /* Synchronise `stream`, then read the workspace status word into *device_status
  * (a qkn_status value; QKN_OK if no kernel recorded an error).  The word is

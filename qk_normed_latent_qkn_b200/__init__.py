@@ -26,7 +26,8 @@ KERNEL_AUTO, KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1, 2
 
 EXPORTED = ["qkn_append", "qkn_absorb_query", "qkn_decode_workspace_size", "qkn_workspace_init",
             "qkn_decode", "qkn_read_device_status", "qkn_decode_kernel_for", "qkn_status_string",
-            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb", "qkn_key_gram", "qkn_decode_up"]
+            "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb", "qkn_key_gram", "qkn_decode_up",
+            "qkn_merge_partials"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -51,7 +52,8 @@ class _Cache(ctypes.Structure):
 class _Opts(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("max_ctas", ctypes.c_int32), ("head_tile", ctypes.c_int32),
                 ("wait_limit", ctypes.c_int64), ("split_event", ctypes.c_void_p),
-                ("step_writes_only", ctypes.c_int32), ("test_withhold_ak", ctypes.c_int32)]
+                ("step_writes_only", ctypes.c_int32), ("test_withhold_ak", ctypes.c_int32),
+                ("vis_end", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -69,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "qkn_decode": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, SZ, P, P, PO, P]),
         "qkn_decode_up": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, I32, P, SZ, P, P, PO, P]),
         "qkn_read_device_status": (I32, [P, P, ctypes.POINTER(I32)]),
+        "qkn_merge_partials": (I32, [PD, I32, I64, P, P, P, P, P]),
         "qkn_decode_kernel_for": (I32, [PD, I32, PO]),
         "qkn_status_string": (ctypes.c_char_p, [I32]),
         "qkn_version": (I32, []),
@@ -150,8 +153,9 @@ def _stream(stream) -> Optional[int]:
 
 
 def _opts(kernel=KERNEL_AUTO, max_ctas=0, head_tile=0, wait_limit=0, split_event=None, step_writes_only=0,
-          test_withhold_ak=0) -> _Opts:
-    return _Opts(kernel, max_ctas, head_tile, wait_limit, split_event, step_writes_only, test_withhold_ak)
+          test_withhold_ak=0, vis_end=None) -> _Opts:
+    return _Opts(kernel, max_ctas, head_tile, wait_limit, split_event, step_writes_only, test_withhold_ak,
+                 vis_end)
 
 
 # ----------------------------------------------------------------- calls
@@ -209,13 +213,14 @@ def decode_kernel_for(dims: Dims, s_q: int, kernel=KERNEL_AUTO, head_tile=0) -> 
 def decode(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_table, seq_lens, s_q: int,
            workspace: torch.Tensor, out, lse, ak_mode: int = AK_CACHE, kernel: int = KERNEL_AUTO,
            max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0, split_event=None, step_writes_only=False,
-           test_withhold_ak=False, stream=None) -> None:
+           test_withhold_ak=False, vis_end=None, stream=None) -> None:
     """One decode step over the cache (see qkn_decode).  ``split_event`` is a raw cudaEvent_t handle;
-    ``step_writes_only`` and ``test_withhold_ak`` are the qkn_decode_opts fields of those names."""
+    ``step_writes_only``, ``test_withhold_ak`` and ``vis_end`` (a device int32 tensor [batch] or None)
+    are the qkn_decode_opts fields of those names."""
     batch = int(block_table.shape[0])
     max_blocks = int(block_table.shape[1])
     opts = _opts(kernel, max_ctas, head_tile, wait_limit, split_event, int(bool(step_writes_only)),
-                 int(bool(test_withhold_ak)))
+                 int(bool(test_withhold_ak)), _ptr(vis_end))
     _check(_lib.qkn_decode(ctypes.byref(dims.c()), ctypes.byref(cache.c()), ak_mode, _ptr(q_tilde), _ptr(a_q),
                            _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens), batch, s_q,
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
@@ -249,6 +254,15 @@ def decode_noalloc(dims: Dims, cache: Cache, q_tilde, a_q, q_rope_hat, block_tab
                                    _ptr(a_q), _ptr(q_rope_hat), _ptr(block_table), max_blocks, _ptr(seq_lens),
                                    batch, s_q, _ptr(out), _ptr(lse), _ptr(device_status), ctypes.byref(opts),
                                    _stream(stream)), "qkn_decode_noalloc")
+
+
+def merge_partials(dims: Dims, parts, lse_parts, out, lse, stream=None) -> None:
+    """Merge partial results of the same rows (see qkn_merge_partials): ``parts`` [n_parts, ..., r_kv] in the
+    storage dtype, ``lse_parts`` [n_parts, ...] fp32; ``out`` / ``lse`` take the row shape."""
+    n_parts = int(parts.shape[0])
+    rows = int(lse_parts[0].numel())
+    _check(_lib.qkn_merge_partials(ctypes.byref(dims.c()), n_parts, rows, _ptr(parts), _ptr(lse_parts), _ptr(out),
+                                   _ptr(lse), _stream(stream)), "qkn_merge_partials")
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:

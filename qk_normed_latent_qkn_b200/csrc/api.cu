@@ -394,6 +394,7 @@ qkn_status decode_impl(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mode
   a.seg_desc = reinterpret_cast<int2*>(ws + w.desc_off);
   a.step_writes_only = (opts && opts->step_writes_only) ? 1 : 0;
   a.withhold_ak = (opts && opts->test_withhold_ak) ? 1 : 0;
+  a.vis_end = opts ? opts->vis_end : nullptr;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const bool bf16 = dims->dtype == QKN_BF16;
@@ -457,6 +458,19 @@ qkn_status qkn_decode_up(const qkn_dims* dims, const qkn_cache* cache, qkn_ak_mo
   const UpProj up{w_uv, d_v, out_v};
   return decode_impl(dims, cache, ak_mode, q_tilde, a_q, q_rope_hat, block_table, max_blocks, seq_lens, batch, s_q,
                      workspace, ws_bytes, nullptr, lse, &up, opts, stream);
+}
+
+qkn_status qkn_merge_partials(const qkn_dims* dims, int32_t n_parts, int64_t rows, const void* parts,
+                              const float* lse_parts, void* out, float* lse, void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (n_parts < 1 || rows < 0) return QKN_ERR_INVALID_ARG;
+  if (rows == 0) return QKN_OK;
+  if (rows > INT32_MAX) return QKN_ERR_INVALID_ARG;   // grid x of row groups
+  if (!parts || !lse_parts || !out || !lse || !aligned(parts, 16) || !aligned(out, 16)) return QKN_ERR_INVALID_ARG;
+  cudaError_t e = launch_merge_parts(parts, lse_parts, n_parts, rows, dims->r_kv, out, lse, dims->dtype == QKN_BF16,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
 }
 
 qkn_status qkn_read_device_status(const void* workspace, void* stream, int32_t* device_status) {

@@ -233,7 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return true;
       };
       if (waited && !issue_q()) { ok = false; break; }
-      const int first_new_page = (it.L - a.s_q) / kPage;
+      const int first_new_page = ((a.vis_end ? a.vis_end[it.b] : it.L) - a.s_q) / kPage;
       for (int pb = it.p0; pb < it.p1 && ok; pb += 32) {
         if (pb > it.p0) mine = (pb + lane < it.p1) ? row[pb + lane] : 0;
         if (mine < 0 || mine >= a.num_blocks) {
@@ -397,7 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int j = valid ? rg / a.heads : 0;
       const int grp = (valid ? rg - j * a.heads : 0) / ng;
       const float aq = valid ? a.a_q[(int64_t)it.b * qrows + rg] : 0.f;
-      const int qlim = valid ? it.L - a.s_q + j : -1;
+      const int qlim = valid ? (a.vis_end ? a.vis_end[it.b] : it.L) - a.s_q + j : -1;
       float mu = -INFINITY, lsum = 0.f;               // reference and this thread's part of the row sum
       // A wait that runs out makes `got` false; the math warps leave together, at the next vote
       // over all 256 of them (every named barrier of the loop is such a vote), never at a barrier

@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(kSimtRows * 32) decode_simt_kernel(DecodeArgs 
     const int j = valid ? rho / a.heads : 0;
     const int h = valid ? rho - j * a.heads : 0;
     const int grp = h / ng;
-    const int32_t qpos = it.L - a.s_q + j;
+    const int32_t qpos = (a.vis_end ? a.vis_end[it.b] : it.L) - a.s_q + j;
     const int64_t qrow = (int64_t)it.b * qrows + (valid ? rho : 0);
 
     float qv[NK], ov[NK];

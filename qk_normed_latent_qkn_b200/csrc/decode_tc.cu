@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         return true;
       };
       if (waited && !issue_q()) { ok = false; break; }
-      const int first_new_page = (it.L - a.s_q) / kPage;   // pages from here on hold this step's tokens
+      // pages from here on hold this step's tokens
+      const int first_new_page = ((a.vis_end ? a.vis_end[it.b] : it.L) - a.s_q) / kPage;
       for (int pb = it.p0; pb < it.p1 && ok; pb += 32) {
         // 32 block-table entries per warp-wide load
         if (pb > it.p0) mine = (pb + lane < it.p1) ? row[pb + lane] : 0;
@@ -543,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const int sl = cb + pm(t);
         ms.aq2[sl] = valid ? a.a_q[(int64_t)it.b * qrows + rho] * kLog2e : 0.f;
         ms.grp[sl] = h / ng;
-        ms.qlim[sl] = valid ? it.L - a.s_q + j : -1;
+        ms.qlim[sl] = valid ? (a.vis_end ? a.vis_end[it.b] : it.L) - a.s_q + j : -1;
         ms.mu[sl] = -INFINITY;
       }
       named_bar_sync(gbar, kGroupThreads);

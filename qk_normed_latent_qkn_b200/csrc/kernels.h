@@ -78,6 +78,7 @@ struct DecodeArgs {
   int2* seg_desc;            // [batch * ht_count]
   int32_t step_writes_only;  // qkn_decode_opts.step_writes_only: read inputs and old pages before the wait
   int32_t withhold_ak;       // qkn_decode_opts.test_withhold_ak (tests of the timeout path)
+  const int32_t* vis_end;    // qkn_decode_opts.vis_end: per sequence, the causal limit's end (null: seq_lens)
 };
 
 struct CombineArgs {
@@ -111,6 +112,9 @@ cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, c
 cudaError_t launch_absorb(const AbsorbArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_decode_simt(const DecodeArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st);
+// Merge n_parts normalised partial outputs of the same rows (merge_parts.cu).
+cudaError_t launch_merge_parts(const void* parts, const float* lse_parts, int n_parts, int64_t rows, int r,
+                               void* out, float* lse, bool bf16, cudaStream_t st);
 bool combine_up_supported(bool bf16, int r, int d_v, int n_q);
 cudaError_t launch_combine_up(const CombineUpArgs& u, bool bf16, cudaStream_t st);
 

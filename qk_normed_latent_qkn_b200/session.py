@@ -100,7 +100,7 @@ class DecodeSession:
 
     def decode(self, block_table, seq_lens, s_q: int, out=None, lse=None, ak_mode: int = AK_CACHE,
                kernel: int = KERNEL_AUTO, max_ctas: int = 0, head_tile: int = 0, wait_limit: int = 0,
-               split_event=None, step_writes_only: bool = False, test_withhold_ak: bool = False):
+               split_event=None, step_writes_only: bool = False, test_withhold_ak: bool = False, vis_end=None):
         d, dev = self.dims, self.device
         bt = to_device(block_table, torch.int32, dev)
         sl = to_device(seq_lens, torch.int32, dev)
@@ -112,7 +112,8 @@ class DecodeSession:
             lse = torch.empty((batch, s_q, d.num_heads), dtype=torch.float32, device=dev)
         decode(d, self.cache, self.q_tilde, self.a_q, self.q_rope_hat, bt, sl, s_q, ws, out, lse,
                ak_mode=ak_mode, kernel=kernel, max_ctas=max_ctas, head_tile=head_tile, wait_limit=wait_limit,
-               split_event=split_event, step_writes_only=step_writes_only, test_withhold_ak=test_withhold_ak)
+               split_event=split_event, step_writes_only=step_writes_only, test_withhold_ak=test_withhold_ak,
+               vis_end=None if vis_end is None else to_device(vis_end, torch.int32, dev))
         return out, lse
 
     def decode_up(self, block_table, seq_lens, s_q: int, out_v=None, lse=None, ak_mode: int = AK_CACHE,
