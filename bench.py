@@ -543,15 +543,11 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "batch_per_gpu": B, "s_q": s_q, "heads": H, "groups": wl.groups,
-                       "r_kv": wl.r_kv, "d_h": wl.d_h, "d_rope": wl.d_rope,
-                       "context": list(wl.context) if isinstance(wl.context, tuple) else wl.context,
-                       "cached_tokens_per_gpu": int(inp.seq_lens.sum()), "paged": wl.paged,
-                       "kernel": {qkn.KERNEL_TCGEN05: "tcgen05", qkn.KERNEL_SIMT: "simt"}.get(kernel_used),
-                       "head_tile": args.head_tile or "auto",
-                       "l2": f"{n_copies} rotating cache copies, {n_copies * cache_bytes / 2**20:.0f} MiB "
-                             f"(L2 {l2 / 2**20:.0f} MiB)", "step_launch": "CUDA graph per step",
-                       "parallelism": f"replicas x{world}"},
+            "config": dict(workload_config(wl, inp, world),
+                           kernel={qkn.KERNEL_TCGEN05: "tcgen05", qkn.KERNEL_SIMT: "simt"}.get(kernel_used),
+                           head_tile=args.head_tile or "auto",
+                           l2=f"{n_copies} rotating cache copies, {n_copies * cache_bytes / 2**20:.0f} MiB "
+                              f"(L2 {l2 / 2**20:.0f} MiB)", step_launch="CUDA graph per step"),
             "breakdown_us": {"append_absorb": statistics.median(prep_ms) * 1e3,
                              "decode_split": statistics.median(split_ms) * 1e3,
                              "combine": statistics.median(combine_ms) * 1e3,
@@ -618,6 +614,15 @@ def schedule_shape(kernel_used: int, head_tile: int, s_q: int, heads: int, sms: 
 
 
 # ----------------------------------------------------------------- reference arm (the oracle)
+def workload_config(wl, inp, world: int) -> dict:
+    """The workload part of the JSON line's config, the same for both arms."""
+    return {"workload": wl.name, "batch_per_gpu": wl.batch, "s_q": wl.s_q, "heads": wl.heads, "groups": wl.groups,
+            "r_kv": wl.r_kv, "d_h": wl.d_h, "d_rope": wl.d_rope,
+            "context": list(wl.context) if isinstance(wl.context, tuple) else wl.context,
+            "cached_tokens_per_gpu": int(inp.seq_lens.sum()), "paged": wl.paged,
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return None
@@ -639,7 +644,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.heads},
+        "config": dict(workload_config(wl, inp, world), sample="one whole sequence per step"),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"one sequence of {wl.name} per step (explicit keys, fp64 numpy)"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
