@@ -67,7 +67,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five decode workloads.  d_h = 128 where the workload statement leaves it
+# The five decode workloads and a prefill workload.  d_h = 128 where the workload statement leaves it
 # open (long-context and grouped cases), as in the large MLA case.
 WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", batch=1, s_q=1, heads=4, groups=1, r_kv=64, d_h=32,
@@ -82,8 +82,12 @@ WORKLOADS = {
     "grouped_mtp_bf16": Workload("grouped_mtp_bf16", batch=8, s_q=2, heads=64, groups=4,
                                  r_kv=512, d_h=128, d_rope=64, context=(4096, 65536),
                                  paged=True, dtype="bf16"),
+    # attention forward over whole sequences (prefill / training-time forward): every token is a
+    # query, causal (s_q = context)
+    "prefill_mla_bf16": Workload("prefill_mla_bf16", batch=2, s_q=2048, heads=16, groups=1, r_kv=512,
+                                 d_h=128, d_rope=64, context=2048, paged=True, dtype="bf16"),
 }
-WORKLOAD_ORDER = ["tiny_f32", "small_mla_bf16", "large_mla_bf16", "long_ctx_bf16",
+WORKLOAD_ORDER = ["tiny_f32", "small_mla_bf16", "large_mla_bf16", "long_ctx_bf16", "prefill_mla_bf16",
                   "grouped_mtp_bf16"]
 
 
