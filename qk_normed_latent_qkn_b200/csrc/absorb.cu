@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(kAbsWarps * 32, 1) absorb_kernel(const __grid_
   float* smem = reinterpret_cast<float*>(smem4);
   float (*rows)[128] = reinterpret_cast<float (*)[128]>(smem);
   float* absm = smem + kAbsWarps * 128;
-  const int pitch = p.a.d_h + 4;
+  const int pitch = absorb_pitch(p.a.d_h);
   const int wstride = (p.nbuf - 1) * KB * pitch;        // second W buffer (the first when nbuf == 1)
   float* sv = absm + p.nbuf * KB * pitch;
   float* g2 = sv + kAbsQ * pitch;

@@ -10,7 +10,9 @@
 // global memory:
 //   o_lat[i, h] = sum_s exp(lse_s - lse) o_s,  lse[i, h] = log sum_s exp(lse_s),
 //   o_v[i, h] = o_lat[i, h] W^UV_h.
-// One CTA per (head h, kRows query rows i = b s_q + j):
+// One CTA per (head h, kRows query rows i = b s_q + j, group of d_v / G output columns); G > 1
+// only when heads x row blocks would leave SMs idle (each column group merges the same rows, the
+// repeated partial reads coming from L2, and loads only its columns of W^UV_h):
 //   1. bf16 storage: W^UV_h goes to shared memory by cp.async while the merge
 //      runs (issued before the wait for the decode, which never writes it);
 //   2. the merge: each warp takes rows in turn, every lane owning 16-byte
@@ -110,17 +112,18 @@ __global__ void __launch_bounds__(kUpThreads, 1) combine_up_kernel(const Combine
   const int n_q = a.batch * a.s_q;
   const int nrows = min(kRows, n_q - i0);                 // rows of this CTA that exist
   const int r = a.r, dv = u.d_v;
+  const int dvc = dv / u.col_groups, n_lo = (int)blockIdx.z * dvc;   // this CTA's output columns
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const UpLayout L = up_layout(kTensor, kRows, r, dv);
+  const UpLayout L = up_layout(kTensor, kRows, r, dvc);
   T* ws = reinterpret_cast<T*>(up_smem + L.w_off);
   T* os = reinterpret_cast<T*>(up_smem + L.o_off);
   int64_t* first_s = reinterpret_cast<int64_t*>(up_smem + L.misc_off);
   int* nitems_s = reinterpret_cast<int*>(up_smem + L.misc_off + (size_t)kRows * 8);
-  const T* w = static_cast<const T*>(u.w_uv) + (int64_t)h * r * dv;
+  const T* w = static_cast<const T*>(u.w_uv) + (int64_t)h * r * dv + n_lo;   // column n_lo of W^UV_h
 
   // ---- 1. W^UV_h into shared memory, in flight during the merge
   if constexpr (kTensor) {
-    const int cpr = dv / 8;                               // 16-byte chunks per row of W^UV_h
+    const int cpr = dvc / 8;                              // 16-byte chunks per row of the columns
     const uint32_t wbase = smem_u32(ws);
     for (int c = threadIdx.x; c < r * cpr; c += kUpThreads) {
       const int k = c / cpr, n8 = c - k * cpr;
@@ -236,7 +239,8 @@ __global__ void __launch_bounds__(kUpThreads, 1) combine_up_kernel(const Combine
       if (v < nvec)
         store_row4<T>(orow + v * 4, make_float4(acc[t].x * inv, acc[t].y * inv, acc[t].z * inv, acc[t].w * inv));
     }
-    if (lane == 0 && rr < nrows) a.lse[(int64_t)(i0 + rr) * a.heads + h] = den > 0.f ? m + logf(den) : -INFINITY;
+    if (lane == 0 && rr < nrows && blockIdx.z == 0)
+      a.lse[(int64_t)(i0 + rr) * a.heads + h] = den > 0.f ? m + logf(den) : -INFINITY;
   }
   if constexpr (kTensor) cp_async_wait_all();
   __syncthreads();
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) combine_up_kernel(const Combine
   // ---- 3. o_v = o_lat W^UV_h for the CTA's rows
   T* out = static_cast<T*>(u.out_v);
   const int64_t ostride = (int64_t)a.heads * dv;          // between consecutive query rows of o_v
-  T* out0 = out + ((int64_t)i0 * a.heads + h) * dv;
+  T* out0 = out + ((int64_t)i0 * a.heads + h) * dv + n_lo;
   if constexpr (kTensor) {
     // Task = (group of kMt m-tiles of 16 rows, pair of n-tiles of 8 columns); kRows / 16 / kMt = 2
     // groups, so 2 d_v / 16 tasks over the 16 warps.  Fragments (lane = 4 gid + tig): A rows gid and
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) combine_up_kernel(const Combine
     // gid + 8, columns 2 tig, 2 tig + 1.
     constexpr int kMt = kRows / 32;
     const int gid = lane >> 2, tig = lane & 3;
-    const int npairs = dv / 16;
+    const int npairs = dvc / 16;
     const uint32_t obase = smem_u32(os), wbase = smem_u32(ws);
     for (int task = warp; task < 2 * npairs; task += kUpWarps) {
       const int mg = task / npairs, np = task - mg * npairs;
@@ -288,9 +292,9 @@ __global__ void __launch_bounds__(kUpThreads, 1) combine_up_kernel(const Combine
           }
     }
   } else {
-    // fp32: thread t takes outputs e = t, t + 512, ... as (row e / d_v, column e % d_v)
-    for (int e = threadIdx.x; e < nrows * dv; e += kUpThreads) {
-      const int rr = e / dv, n = e - rr * dv;
+    // fp32: thread t takes outputs e = t, t + 512, ... as (row e / dvc, column e % dvc)
+    for (int e = threadIdx.x; e < nrows * dvc; e += kUpThreads) {
+      const int rr = e / dvc, n = e - rr * dvc;
       const float* orow = reinterpret_cast<const float*>(os) + (size_t)rr * L.opitch;
       const float* wc = reinterpret_cast<const float*>(w) + n;
       float acc = 0.f;
@@ -303,13 +307,29 @@ __global__ void __launch_bounds__(kUpThreads, 1) combine_up_kernel(const Combine
 constexpr int kMaxUpSmem = 227 * 1024;
 
 template <typename T, int kRows>
-cudaError_t launch_up_t(const CombineUpArgs& u, cudaStream_t st) {
-  const UpLayout L = up_layout(std::is_same<T, __nv_bfloat16>::value, kRows, u.c.r, u.d_v);
+cudaError_t launch_up_t(CombineUpArgs u, cudaStream_t st) {
   static PerDeviceOnce attrs;
   cudaError_t e = once_per_device(attrs, [] { return set_smem_attrs(combine_up_kernel<T, kRows>, kMaxUpSmem); });
   if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   const int n_q = u.c.batch * u.c.s_q;
-  const dim3 grid((unsigned)u.c.heads, (unsigned)((n_q + kRows - 1) / kRows));
+  const int ctas = u.c.heads * ((n_q + kRows - 1) / kRows);
+  // column groups repeat the merge of the CTA's rows (from L2) for every group, which costs more
+  // than it gains unless the grid leaves most SMs idle: below a quarter of the SMs, the fewest
+  // groups (a divisor of d_v / 16) that reach half of them (measured: 16 heads x 16 rows 14.4 ->
+  // 12.3 us; 64 and 128 heads slower with groups)
+  const int pairs = u.d_v / 16;
+  int g = 1;
+  while (4 * ctas < sms && g < pairs && 2 * ctas * g < sms) {
+    ++g;
+    while (pairs % g) ++g;
+  }
+  u.col_groups = g;
+  const UpLayout L = up_layout(std::is_same<T, __nv_bfloat16>::value, kRows, u.c.r, u.d_v / g);
+  const dim3 grid((unsigned)u.c.heads, (unsigned)((n_q + kRows - 1) / kRows), (unsigned)g);
   return launch_chained(combine_up_kernel<T, kRows>, grid, dim3(kUpThreads), L.total, st, u);
 }
 

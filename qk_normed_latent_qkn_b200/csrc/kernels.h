@@ -102,6 +102,7 @@ struct CombineUpArgs {
   const void* w_uv;          // [H, r, d_v] in the storage type
   int32_t d_v;
   void* out_v;               // [batch, s_q, H, d_v] in the storage type
+  int32_t col_groups;        // output column groups per (head, row block); set by the launcher
 };
 
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);

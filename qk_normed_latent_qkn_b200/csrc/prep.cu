@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(const __grid_cons
   }
   bid -= p.ab.heads;
   constexpr int KB = absorb_unit_rows<kPrepWarps>();
-  const int pitch = p.ab.d_h + 4;
+  const int pitch = absorb_pitch(p.ab.d_h);
   float* sv = work + KB * pitch;
   absorb_zero_pads<kPrepWarps>(p.ab, work, 1);
   absorb_load_w<kPrepWarps>(p.ab, bid, work);

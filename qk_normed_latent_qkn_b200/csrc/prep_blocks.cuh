@@ -291,13 +291,16 @@ __device__ __forceinline__ void absorb_head_rows(const AbsorbArgs& a, int h, flo
 // q~ at 2^-9); fp32 storage keeps fp32 FMAs.  a_q and the RoPE query of head h come from
 // absorb_head_rows, or from the kc == 0 unit.
 //
-// Shared memory (floats, row pitch d_h + 4 so that the 8 rows of a fragment read fall in distinct
-// banks): nbuf W buffers [KB][d_h + 4], the query rows [kAbsQ][d_h + 4], gamma_q gamma_k [d_h].
+// Shared memory (floats): nbuf W buffers [KB][pitch], the query rows [kAbsQ][pitch], gamma_q gamma_k
+// [d_h].  The row pitch is the smallest p >= d_h + 4 with p = 8 (mod 32): the TF32 products read a
+// fragment's two K values as one 8-byte pair (below), and with that pitch the 16 threads of each
+// half-warp (rows gid < 4, pairs 2 tig) hit 32 distinct banks; the 4 pad columns stay zero.
+__host__ __device__ inline int absorb_pitch(int d_h) { return d_h + 4 + (((8 - (d_h + 4)) % 32) + 32) % 32; }
 template <int NW>
 __host__ __device__ constexpr int absorb_unit_rows() { return NW * 8; }
 template <int NW>
 inline size_t absorb_unit_floats(int d_h, int nbuf) {
-  return (size_t)(nbuf * absorb_unit_rows<NW>() + kAbsQ) * (d_h + 4) + d_h;
+  return (size_t)(nbuf * absorb_unit_rows<NW>() + kAbsQ) * absorb_pitch(d_h) + d_h;
 }
 template <int NW>
 __host__ __device__ inline int absorb_units(int heads, int r) {
@@ -322,12 +325,19 @@ __device__ __forceinline__ void absorb_load_w(const AbsorbArgs& a, int j, float*
   const int nkc = (a.r + KB - 1) / KB;
   const int h = j / nkc, kbase = (j - h * nkc) * KB;
   const int ng = a.heads / a.groups, g = h / ng, m = h - g * ng;
-  const int width = ng * a.d_h, pitch = a.d_h + 4, dq = a.d_h / 4;
+  const int width = ng * a.d_h, pitch = absorb_pitch(a.d_h), dq = a.d_h / 4;
   const float* w = a.w_k + (int64_t)g * a.r * width + (int64_t)m * a.d_h;
   const int nrows = min(KB, a.r - kbase);
-  for (int e = threadIdx.x; e < nrows * dq; e += kT) {
-    const int rr = e / dq, d4 = e - rr * dq;
-    cp_async16(wb + rr * pitch + d4 * 4, w + (int64_t)(kbase + rr) * width + d4 * 4);
+  if (kT % dq == 0) {
+    // each thread keeps one 16-byte column of the slice and walks its rows
+    const int d4 = threadIdx.x % dq, rstep = kT / dq;
+    for (int rr = threadIdx.x / dq; rr < nrows; rr += rstep)
+      cp_async16(wb + rr * pitch + d4 * 4, w + (int64_t)(kbase + rr) * width + d4 * 4);
+  } else {
+    for (int e = threadIdx.x; e < nrows * dq; e += kT) {
+      const int rr = e / dq, d4 = e - rr * dq;
+      cp_async16(wb + rr * pitch + d4 * 4, w + (int64_t)(kbase + rr) * width + d4 * 4);
+    }
   }
   cp_async_commit();
 }
@@ -336,7 +346,7 @@ __device__ __forceinline__ void absorb_load_w(const AbsorbArgs& a, int j, float*
 // d_h % 8 == 4, and the copies never write them.
 template <int NW>
 __device__ __forceinline__ void absorb_zero_pads(const AbsorbArgs& a, float* abs_smem, int nbuf) {
-  const int pitch = a.d_h + 4;
+  const int pitch = absorb_pitch(a.d_h);
   for (int rr = threadIdx.x; rr < nbuf * absorb_unit_rows<NW>() + kAbsQ; rr += NW * 32)
     *reinterpret_cast<float4*>(abs_smem + rr * pitch + a.d_h) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -354,7 +364,7 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
   constexpr int kRowWarps = NW / 2;
   static_assert(kRowWarps * 16 == KB && kAbsQ == 32, "warp tiling of the absorption unit");
   constexpr bool kTensor = std::is_same<T, __nv_bfloat16>::value;
-  const int pitch = a.d_h + 4, dq = a.d_h / 4;
+  const int pitch = absorb_pitch(a.d_h), dq = a.d_h / 4;
   const int nkc = (a.r + KB - 1) / KB;
   const int h = j / nkc, kc = j - h * nkc, kbase = kc * KB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -363,7 +373,7 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
   // stage query rows [i0, i0 + nq) of head h times gamma_q gamma_k (zeros past nq); g2 is ready
   auto stage_q = [&](int i0, int nq) {
     for (int e = threadIdx.x; e < kAbsQ * dq; e += kThreadsAbs) {
-      const int qi = e / dq, d4 = e - qi * dq;
+      const int qi = (dq == 32) ? (e >> 5) : e / dq, d4 = e - qi * dq;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (qi < nq) {
         const T* src = q + ((int64_t)(i0 + qi) * a.heads + h) * a.d_h + d4 * 4;
@@ -393,19 +403,25 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
     if (qw * 16 >= nq) continue;                           // no query rows for this warp (warp-uniform)
     if constexpr (kTensor) {
       // m16n8k8 TF32 products: A = 16 rows of the slice, B = 8 query rows, per 8 columns of d_h.
-      // Fragments (lane = 4 gid + tig): A holds (row gid | gid + 8, column tig | tig + 4), B
-      // (query row gid, column tig | tig + 4), D (row gid | gid + 8, query row 2 tig | 2 tig + 1).
+      // Fragments (lane = 4 gid + tig): A holds (row gid | gid + 8, K index tig | tig + 4), B
+      // (query row gid, K index tig | tig + 4), D (row gid | gid + 8, query row 2 tig | 2 tig + 1).
+      // K index tig carries column d + 2 tig of d_h and K index tig + 4 column d + 2 tig + 1 (the same
+      // map on A and B, so the 8 products of a step are those of columns d .. d + 7): each thread
+      // reads a fragment's two values as one 8-byte pair.
       const int gid = lane >> 2, tig = lane & 3;
-      const float* wa = wb + (rw * 16 + gid) * pitch + tig;
-      const float* qb = sv + (qw * 16 + gid) * pitch + tig;
+      const float* wa = wb + (rw * 16 + gid) * pitch + 2 * tig;
+      const float* qb = sv + (qw * 16 + gid) * pitch + 2 * tig;
       float dacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 4
       for (int d = 0; d < a.d_h; d += 8) {
-        const uint32_t af[4] = {__float_as_uint(wa[d]), __float_as_uint(wa[8 * pitch + d]),
-                                __float_as_uint(wa[d + 4]), __float_as_uint(wa[8 * pitch + d + 4])};
+        const float2 w0 = *reinterpret_cast<const float2*>(wa + d);
+        const float2 w1 = *reinterpret_cast<const float2*>(wa + 8 * pitch + d);
+        const uint32_t af[4] = {__float_as_uint(w0.x), __float_as_uint(w1.x), __float_as_uint(w0.y),
+                                __float_as_uint(w1.y)};
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const uint32_t bf[2] = {__float_as_uint(qb[jj * 8 * pitch + d]), __float_as_uint(qb[jj * 8 * pitch + d + 4])};
+          const float2 q2 = *reinterpret_cast<const float2*>(qb + jj * 8 * pitch + d);
+          const uint32_t bf[2] = {__float_as_uint(q2.x), __float_as_uint(q2.y)};
           mma_tf32_m16n8k8(dacc[jj], af, bf);
         }
       }
