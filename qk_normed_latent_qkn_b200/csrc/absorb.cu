@@ -56,7 +56,7 @@ template <typename T>
 cudaError_t launch_absorb_t(const AbsorbArgs& a, cudaStream_t st) {
   AbsorbLaunch p;
   p.a = a;
-  p.units = absorb_units<kAbsWarps>(a.heads, a.r);
+  p.units = absorb_units<kAbsWarps>(a.heads, a.r, a.n_q);
   const size_t rows_floats = (size_t)kAbsWarps * 128;
   size_t floats = rows_floats + absorb_unit_floats<kAbsWarps>(a.d_h, 2);
   p.nbuf = 2;

@@ -69,7 +69,7 @@ cudaError_t launch_prep(const AppendArgs& ap, const AbsorbArgs& ab, bool bf16, c
   p.append_x = (ap.ncols + kRmsCols - 1) / kRmsCols + 1;
   p.append_y = (ap.n_tok + kPrepTT - 1) / kPrepTT;
   p.append_ctas = p.append_x * p.append_y * ap.groups;
-  const int64_t ctas = (int64_t)p.append_ctas + ab.heads + absorb_units<kPrepWarps>(ab.heads, ab.r);
+  const int64_t ctas = (int64_t)p.append_ctas + ab.heads + absorb_units<kPrepWarps>(ab.heads, ab.r, ab.n_q);
   const size_t app = (size_t)kPrepTT * ap.r + (size_t)kRmsSlices * kPrepTT * kRmsCols;
   const size_t abs1 = absorb_unit_floats<kPrepWarps>(ab.d_h, 1);
   const size_t smem = ((size_t)kPrepWarps * 128 + (app > abs1 ? app : abs1)) * sizeof(float);

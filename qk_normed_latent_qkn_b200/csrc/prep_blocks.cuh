@@ -282,7 +282,9 @@ __device__ __forceinline__ void absorb_head_rows(const AbsorbArgs& a, int h, flo
 
 // ---------------------------------------------------------------- absorption units
 // The absorption q~[i, h] = W^K_{g,h} (gamma_q[h] gamma_k[h] q[i, h]) as units (head h, KB = 8 NW
-// latent rows from kbase = kc KB), unit j = h ceil(r / KB) + kc, for CTAs of NW warps.  A unit's
+// latent rows from kbase = kc KB, query rows [qb QB, (qb + 1) QB)), unit
+// j = (h ceil(r / KB) + kc) ceil(n_q / QB) + qb, for CTAs of NW warps (the units that share a W
+// slice are consecutive, so the later copies of it come from L2).  A unit's
 // slice of W^K_{g,h} (KB rows of d_h contiguous fp32 values) is copied raw with 16-byte cp.async
 // (no register staging) into a W buffer; gamma_q gamma_k is folded into the staged query rows
 // instead of into W (the same products in another order).  For bf16 storage the products run on
@@ -302,9 +304,10 @@ template <int NW>
 inline size_t absorb_unit_floats(int d_h, int nbuf) {
   return (size_t)(nbuf * absorb_unit_rows<NW>() + kAbsQ) * absorb_pitch(d_h) + d_h;
 }
+constexpr int kAbsQB = 128;      // query rows per absorption unit (in passes of kAbsQ)
 template <int NW>
-__host__ __device__ inline int absorb_units(int heads, int r) {
-  return heads * ((r + absorb_unit_rows<NW>() - 1) / absorb_unit_rows<NW>());
+__host__ __device__ inline int absorb_units(int heads, int r, int n_q) {
+  return heads * ((r + absorb_unit_rows<NW>() - 1) / absorb_unit_rows<NW>()) * ((n_q + kAbsQB - 1) / kAbsQB);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -322,8 +325,9 @@ __device__ __forceinline__ void cp_async_wait_pending(int n) {
 template <int NW>
 __device__ __forceinline__ void absorb_load_w(const AbsorbArgs& a, int j, float* wb) {
   constexpr int KB = absorb_unit_rows<NW>(), kT = NW * 32;
-  const int nkc = (a.r + KB - 1) / KB;
-  const int h = j / nkc, kbase = (j - h * nkc) * KB;
+  const int nkc = (a.r + KB - 1) / KB, nqb = (a.n_q + kAbsQB - 1) / kAbsQB;
+  const int hk = j / nqb;
+  const int h = hk / nkc, kbase = (hk - h * nkc) * KB;
   const int ng = a.heads / a.groups, g = h / ng, m = h - g * ng;
   const int width = ng * a.d_h, pitch = absorb_pitch(a.d_h), dq = a.d_h / 4;
   const float* w = a.w_k + (int64_t)g * a.r * width + (int64_t)m * a.d_h;
@@ -365,8 +369,10 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
   static_assert(kRowWarps * 16 == KB && kAbsQ == 32, "warp tiling of the absorption unit");
   constexpr bool kTensor = std::is_same<T, __nv_bfloat16>::value;
   const int pitch = absorb_pitch(a.d_h), dq = a.d_h / 4;
-  const int nkc = (a.r + KB - 1) / KB;
-  const int h = j / nkc, kc = j - h * nkc, kbase = kc * KB;
+  const int nkc = (a.r + KB - 1) / KB, nqb = (a.n_q + kAbsQB - 1) / kAbsQB;
+  const int hk = j / nqb, qb = j - hk * nqb;
+  const int h = hk / nkc, kc = hk - h * nkc, kbase = kc * KB;
+  const int q_lo = qb * kAbsQB, q_hi = min(a.n_q, q_lo + kAbsQB);   // this unit's query rows
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const T* q = static_cast<const T*>(a.q);
   T* out = static_cast<T*>(a.q_tilde);
@@ -390,12 +396,12 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
     reinterpret_cast<float4*>(g2)[threadIdx.x] = make_float4(gq.x * gk.x, gq.y * gk.y, gq.z * gk.z, gq.w * gk.w);
   }
   __syncthreads();
-  stage_q(0, min(kAbsQ, a.n_q));
+  stage_q(q_lo, min(kAbsQ, q_hi - q_lo));
   cp_async_wait_pending(pending);                        // this unit's W slice has landed
   const int rw = warp % kRowWarps, qw = warp / kRowWarps;
-  for (int i0 = 0; i0 < a.n_q; i0 += kAbsQ) {
-    const int nq = min(kAbsQ, a.n_q - i0);
-    if (i0 > 0) {
+  for (int i0 = q_lo; i0 < q_hi; i0 += kAbsQ) {
+    const int nq = min(kAbsQ, q_hi - i0);
+    if (i0 > q_lo) {
       __syncthreads();                                     // the previous pass is done with sv
       stage_q(i0, nq);
     }
@@ -468,7 +474,7 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
   }
   if (kc == 0 && rows_too) {
     // a_q and the rotated RoPE query of head h, one warp per query row
-    for (int i = warp; i < a.n_q; i += NW) absorb_row<T>(a, i, h, rows[warp], lane);
+    for (int i = q_lo + warp; i < q_hi; i += NW) absorb_row<T>(a, i, h, rows[warp], lane);
   }
   __syncthreads();
 }
