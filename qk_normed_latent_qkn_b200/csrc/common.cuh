@@ -117,6 +117,13 @@ struct SchedParams {
   int32_t ht_count;     // query-row tiles per sequence (HT)
   int32_t ncta;
   int32_t item_cost;    // units without pages at the start of every sequence
+  // Decode kernels only (0 / null elsewhere): with heads and the rows per tile known, an item ends at
+  // the last page its tile's rows can see (the causal limit of the tile's last query row), so that
+  // the row tiles of a long chunk of queries (a prefill) skip the pages past their limit.  Such an
+  // item may have no pages at all; it still takes its slot (zero output, lse = -inf).
+  int32_t heads = 0;
+  int32_t rows = 0;
+  const int32_t* vis_end = nullptr;
 };
 
 __device__ __forceinline__ int32_t pages_of(int32_t L, const SchedParams& p) {
@@ -238,6 +245,12 @@ __device__ __forceinline__ bool sched_next(Cursor& cur, const SchedParams& p, in
       it.L = p.seq_lens[cur.b];
       it.slot = (cur.b + cur.group) * p.ht_count + cur.ht;
       it.seg_u0 = s0;
+      if (p.heads > 0) {
+        const int32_t jmax = min(p.s_q - 1, (cur.ht * p.rows + p.rows - 1) / p.heads);
+        const int32_t last = (p.vis_end ? p.vis_end[cur.b] : it.L) - p.s_q + jmax;   // last visible token
+        const int32_t lim = last >= 0 ? last / kBlockSize + 1 : 0;
+        if (it.p1 > lim) it.p1 = lim > it.p0 ? lim : it.p0;
+      }
       cur.ht += cur.hstep;                       // this CTA's next row tile of the same pages
       if (cur.ht < p.ht_count) return true;
     }

@@ -144,7 +144,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t crank = cluster_ctarank();            // c: this CTA's latent half and row half
   const uint32_t prank = crank ^ 1u;
   const int pair = blockIdx.x >> 1;                    // the schedule's unit of work is the pair
-  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost};
+  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost,
+                       a.heads, a.rows, a.vis_end};
   const int qrows = a.s_q * a.heads;
   const int G = a.groups;
 
@@ -334,8 +335,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int64_t tile_n = 0;
     int n_item = 0;
     while (ok && sched_next(cur, sp, pair, it)) {
+      // once per item, pages or not, so that the barrier is never more than one phase ahead
+      if (!mbar_wait_warp(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
       for (int p = it.p0; p < it.p1 && ok; ++p) {
-        if (p == it.p0 && !mbar_wait_warp(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
         if (!mbar_wait_warp(smem_u32(&ms.p_ready), (uint32_t)(tile_n & 1), a.wait_limit)) { ok = false; break; }
         tc_fence_after();
         const uint64_t slot = (uint64_t)((cr.slot * SLOT_BYTES) >> 4);
@@ -564,7 +566,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------- epilogue of the item: O / l for every lane, lse
-      bool got = mbar_wait_cl(smem_u32(&ms.p_free), (uint32_t)((tile_n - 1) & 1), a.wait_limit) && carry;
+      bool got = (tile_n == 0 || mbar_wait_cl(smem_u32(&ms.p_free), (uint32_t)((tile_n - 1) & 1), a.wait_limit)) && carry;
       const float lh = lsum + __shfl_xor_sync(0xffffffffu, lsum, 2);   // this CTA's token half of the row
       got = mbar_wait_cl(smem_u32(&ms.l_free), (uint32_t)((n_item & 1) ^ 1), a.wait_limit) && got;
       if (par == 0 && got) st_async_b32(peer_l + rho * 4, __float_as_uint(lh), peer_l_full);
@@ -590,11 +592,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld16(tl32 + half * 128 + c0, ov);
         tmem_wait_ld();
         reg_tie(ov);
+        // a row with no visible token in the item writes zeros, whatever the TMEM holds
 #pragma unroll
         for (int e = 0; e < 16; e += 4)
           *reinterpret_cast<float4*>(po + c0 + e) =
-              make_float4(__uint_as_float(ov[e]) * linv, __uint_as_float(ov[e + 1]) * linv,
-                          __uint_as_float(ov[e + 2]) * linv, __uint_as_float(ov[e + 3]) * linv);
+              linv > 0.f ? make_float4(__uint_as_float(ov[e]) * linv, __uint_as_float(ov[e + 1]) * linv,
+                                       __uint_as_float(ov[e + 2]) * linv, __uint_as_float(ov[e + 3]) * linv)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       tc_fence_before();
       named_bar_sync(1, kMathWarps * 32);              // ms.linv is read before the next item writes it

@@ -23,7 +23,8 @@ __global__ void __launch_bounds__(kSimtRows * 32) decode_simt_kernel(DecodeArgs 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
-  SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost};
+  SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost,
+                 a.heads, a.rows, a.vis_end};
   if (warp == 0) {
     Cursor c = sched_begin(sp, blockIdx.x);
     if (lane == 0) cur_s = c;

@@ -202,7 +202,9 @@ __device__ __forceinline__ bool group_any(bool v, uint32_t bar) {
   return r != 0;
 }
 
-template <int R, bool AK_ONE>
+// SKIP: long chunks of queries (a prefill): an item ends at the last page its tile's rows can see,
+// so an item may have no pages (separate instantiation, so that the decode's code is unchanged).
+template <int R, bool AK_ONE, bool SKIP>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TcMaps maps) {
   using C = Cfg<R>;
   constexpr int NS = C::NS, NKR = C::NKR;
@@ -215,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
   MiscT& ms = *reinterpret_cast<MiscT*>(smem + C::MISC_OFF);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost};
+  const SchedParams sp{a.seq_lens, a.batch, a.s_q, a.max_blocks, a.ht_count, a.ncta, a.item_cost,
+                       SKIP ? a.heads : 0, a.rows, a.vis_end};
   const int qrows = a.s_q * a.heads;
   const int G = a.groups;
 
@@ -441,9 +444,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
     int n_item = 0;
     bool ok = true;
     while (ok && sched_next(cur, sp, blockIdx.x, it)) {
+      // O^T of the previous item must have been read out before it is overwritten; with empty items
+      // possible it is waited once per item, pages or not, so that the barrier is never more than one
+      // phase ahead
+      if (SKIP && !mbar_wait_warp(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
       for (int p = it.p0; p < it.p1 && ok; ++p) {
-        // O^T of the previous item must have been read out before it is overwritten
-        if (p == it.p0 && !mbar_wait_warp(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+        if (!SKIP && p == it.p0 && !mbar_wait_warp(smem_u32(&ms.o_empty), (n_item & 1) ^ 1, a.wait_limit)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait_warp(smem_u32(&ms.p_full[pb.slot]), pb.phase, a.wait_limit)) { ok = false; break; }
         tc_fence_after();
         const uint64_t bP = dP + (uint64_t)(kr.slot * (kKrBytes >> 4));
@@ -736,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       bool got = true;
       if (t == 0) {
         if (tile_n > 1) got = pv_wait(tile_n - 2);
-        got = got && pv_wait(tile_n - 1);
+        if (!SKIP || tile_n > 0) got = got && pv_wait(tile_n - 1);   // (an empty first item has no tiles)
       }
       if (!group_all(got, gbar)) { ok = false; break; }
       tc_fence_after();
@@ -761,7 +770,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
           reg_tie(ov);
 #pragma unroll
           for (int e = 0; e < kOcols; ++e)
-            po[(int64_t)(c0 + e) * kRkv + m * 128 + t] = __uint_as_float(ov[e]) * ms.linv[c0 + e];
+            // (with empty items, a row with no visible token writes zeros, whatever the TMEM holds)
+            if constexpr (SKIP)
+              po[(int64_t)(c0 + e) * kRkv + m * 128 + t] =
+                  ms.linv[c0 + e] > 0.f ? __uint_as_float(ov[e]) * ms.linv[c0 + e] : 0.f;
+            else
+              po[(int64_t)(c0 + e) * kRkv + m * 128 + t] = __uint_as_float(ov[e]) * ms.linv[c0 + e];
         }
       }
       tc_fence_before();
@@ -890,15 +904,22 @@ TmapCache& tmap_cache() {
   return c;
 }
 
-template <int R, bool AK_ONE>
-cudaError_t launch_tc(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) {
+template <int R, bool AK_ONE, bool SKIP>
+cudaError_t launch_tc3(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) {
   static PerDeviceOnce attrs;
   cudaError_t e = once_per_device(attrs, [] {
-    return cudaFuncSetAttribute(decode_tc_kernel<R, AK_ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(decode_tc_kernel<R, AK_ONE, SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Cfg<R>::SMEM);
   });
   if (e != cudaSuccess) return e;
-  return launch_chained(decode_tc_kernel<R, AK_ONE>, dim3(a.ncta), dim3(kThreads), Cfg<R>::SMEM, st, a, maps);
+  return launch_chained(decode_tc_kernel<R, AK_ONE, SKIP>, dim3(a.ncta), dim3(kThreads), Cfg<R>::SMEM, st, a, maps);
+}
+
+// Page skipping pays only when a tile's rows span many query positions: more query rows per
+// sequence than two tiles (s_q > 2 at 64 heads per tile) is a chunk of a prefill.
+template <int R, bool AK_ONE>
+cudaError_t launch_tc(const DecodeArgs& a, const TcMaps& maps, cudaStream_t st) {
+  return a.s_q * a.heads > 2 * R ? launch_tc3<R, AK_ONE, true>(a, maps, st) : launch_tc3<R, AK_ONE, false>(a, maps, st);
 }
 
 }  // namespace
