@@ -749,6 +749,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       }
       if (!group_all(got, gbar)) { ok = false; break; }
       tc_fence_after();
+      // A query chunk's segment that one CTA holds whole (long chunks: every CTA group covers whole
+      // sequences) is written straight to the output, and its descriptor says "no splits" so that the
+      // merge leaves it alone; not when the merge applies the value up-projection (no output here).
+      bool direct = false;
+      if constexpr (SKIP) {
+        if (a.out != nullptr && it.p0 == 0)
+          direct = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota, sp.item_cost).nitems == 1;
+      }
       reduce_store(lpart, false);
       named_bar_sync(gbar, kGroupThreads);
       if (t < NH) {
@@ -756,10 +764,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
         const int sl = cb + pm(t);
         const float l = ms.red[0][sl] + ms.red[1][sl] + ms.red[2][sl] + ms.red[3][sl];
         ms.linv[c] = l > 0.f ? 1.f / l : 0.f;
-        a.part_lse[(int64_t)it.slot * R + c] = l > 0.f ? (ms.mu[sl] + log2f(l)) * kLn2 : -INFINITY;
+        const float lse_c = l > 0.f ? (ms.mu[sl] + log2f(l)) * kLn2 : -INFINITY;
+        if (!direct) {
+          a.part_lse[(int64_t)it.slot * R + c] = lse_c;
+        } else if (it.ht * R + c < qrows) {
+          a.lse[(int64_t)it.b * qrows + it.ht * R + c] = lse_c;
+        }
       }
       named_bar_sync(gbar, kGroupThreads);
       float* po = a.part_o + (int64_t)it.slot * R * kRkv;
+      __nv_bfloat16* pd = static_cast<__nv_bfloat16*>(a.out) + ((int64_t)it.b * qrows + it.ht * R) * kRkv;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
 #pragma unroll
@@ -771,11 +785,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
 #pragma unroll
           for (int e = 0; e < kOcols; ++e)
             // (with empty items, a row with no visible token writes zeros, whatever the TMEM holds)
-            if constexpr (SKIP)
-              po[(int64_t)(c0 + e) * kRkv + m * 128 + t] =
-                  ms.linv[c0 + e] > 0.f ? __uint_as_float(ov[e]) * ms.linv[c0 + e] : 0.f;
-            else
+            if constexpr (SKIP) {
+              const float v = ms.linv[c0 + e] > 0.f ? __uint_as_float(ov[e]) * ms.linv[c0 + e] : 0.f;
+              if (!direct)
+                po[(int64_t)(c0 + e) * kRkv + m * 128 + t] = v;
+              else if (it.ht * R + c0 + e < qrows)
+                pd[(int64_t)(c0 + e) * kRkv + m * 128 + t] = __float2bfloat16_rn(v);
+            } else {
               po[(int64_t)(c0 + e) * kRkv + m * 128 + t] = __uint_as_float(ov[e]) * ms.linv[c0 + e];
+            }
         }
       }
       tc_fence_before();
@@ -783,7 +801,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const DecodeArgs
       // the CTA holding a segment's first split tells the merge kernel where its splits are
       if (threadIdx.x == 0 && it.p0 == 0) {
         const SegSplit sg = seg_split(it.seg_u0, pages_of(it.L, sp), cur.quota, sp.item_cost);
-        a.seg_desc[it.b * a.ht_count + it.ht] = make_int2((it.b + sg.c0) * a.ht_count + it.ht, sg.nitems);
+        a.seg_desc[it.b * a.ht_count + it.ht] =
+            direct ? make_int2(0, 0) : make_int2((it.b + sg.c0) * a.ht_count + it.ht, sg.nitems);
       }
       ++n_item;
     }

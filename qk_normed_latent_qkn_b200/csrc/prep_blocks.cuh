@@ -291,7 +291,7 @@ __device__ __forceinline__ void absorb_head_rows(const AbsorbArgs& a, int h, flo
 // the tensor cores in TF32 (fp32 accumulation): the query rows are rounded to TF32, the raw W
 // values are truncated to it by the MMA (relative error below 2^-10, beside the bf16 rounding of
 // q~ at 2^-9); fp32 storage keeps fp32 FMAs.  a_q and the RoPE query of head h come from
-// absorb_head_rows, or from the kc == 0 unit.
+// absorb_head_rows, or from the units of each query block.
 //
 // Shared memory (floats): nbuf W buffers [KB][pitch], the query rows [kAbsQ][pitch], gamma_q gamma_k
 // [d_h].  The row pitch is the smallest p >= d_h + 4 with p = 8 (mod 32): the TF32 products read a
@@ -358,8 +358,9 @@ __device__ __forceinline__ void absorb_zero_pads(const AbsorbArgs& a, float* abs
 // Unit j with its W slice in `wb` (its copies committed as the older of at most `pending` + 1
 // outstanding groups of this thread).  Starts and ends with the CTA's query rows and gamma
 // buffers free; ends with a barrier, after which `wb` may be refilled.
-// `rows`: a 128-float buffer per warp, for the a_q / RoPE rows when the kc == 0 unit does them
-// (rows_too); otherwise absorb_head_rows does them separately.
+// `rows`: a 128-float buffer per warp, for the a_q / RoPE rows when the units do them (rows_too:
+// the units of a query block share its rows, unit kc taking every ceil(r / KB)-th one); otherwise
+// absorb_head_rows does them separately.
 template <typename T, int NW>
 __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const float* wb, float* sv, float* g2,
                                             int pending, float (*rows)[128], bool rows_too) {
@@ -472,9 +473,9 @@ __device__ __forceinline__ void absorb_unit(const AbsorbArgs& a, int j, const fl
       }
     }
   }
-  if (kc == 0 && rows_too) {
+  if (rows_too) {
     // a_q and the rotated RoPE query of head h, one warp per query row
-    for (int i = q_lo + warp; i < q_hi; i += NW) absorb_row<T>(a, i, h, rows[warp], lane);
+    for (int i = q_lo + kc + warp * nkc; i < q_hi; i += NW * nkc) absorb_row<T>(a, i, h, rows[warp], lane);
   }
   __syncthreads();
 }
