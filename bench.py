@@ -58,6 +58,9 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--soak-seconds", type=float, default=1.0, help="load window around the timed steps for clocks")
     p.add_argument("--overhead-rounds", type=int, default=5)
+    p.add_argument("--cp-emulate", type=int, default=0,
+                   help="also time a context-parallel decode over this many ranks, emulated on one GPU "
+                        "(every rank's slice decode and the merge of the partials; one GPU only)")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -601,6 +604,8 @@ def run_ours(args, world, rank, local):
             "clocks": sampler.summary(window),
             "cpu_baseline": cpu,
         }
+        if args.cp_emulate > 1 and world == 1:
+            line["context_parallel_emulated"] = cp_emulate(args.cp_emulate, base, inp, device, ev, stream)
         if tensor_bound:
             # the step's intensity is above the ridge (every query row sees most of its sequence): the
             # binding roof is the bf16 tensor peak; algorithmic FLOPs count the causal (query, key) pairs
@@ -625,6 +630,74 @@ def schedule_shape(kernel_used: int, head_tile: int, s_q: int, heads: int, sms: 
 
 
 # ----------------------------------------------------------------- reference arm (the oracle)
+def cp_emulate(world: int, base, inp, device, ev, stream, rounds: int = 10) -> dict:
+    """Context-parallel decode over `world` ranks, timed on one GPU: each rank's slice decode (its
+    page slices of every sequence, qkn_decode with vis_end) replayed alone, and the merge of the
+    stacked partials (qkn_merge_partials).  The step on `world` GPUs is estimated as the slowest
+    rank's slice + an all-gather of the partials at the pool's measured NVLink peer-copy bandwidth
+    + the merge; the all-gather is not run here."""
+    import torch
+    import qk_normed_latent_qkn_b200 as qkn
+    from qk_normed_latent_qkn_b200 import context_parallel as cp
+    wl = inp.wl
+    B, s_q, H, r = wl.batch, wl.s_q, wl.heads, wl.r_kv
+    dt = base.dims.torch_dtype
+    ws = base.ensure_workspace(B, s_q)
+    outs = torch.empty((world, B, s_q, H, r), dtype=dt, device=device)
+    lses = torch.empty((world, B, s_q, H), dtype=torch.float32, device=device)
+    out = torch.empty((B, s_q, H, r), dtype=dt, device=device)
+    lse = torch.empty((B, s_q, H), dtype=torch.float32, device=device)
+    views = []
+    for k in range(world):
+        bt, lens, ve = cp.rank_view(inp.block_table, inp.seq_lens, k, world)
+        views.append([torch.from_numpy(x).to(device) for x in (bt, lens, ve)])
+    graphs = []
+    with torch.cuda.stream(stream):
+        for k in range(world):
+            bt, lens, ve = views[k]
+            e = [ev.create() for _ in range(2)]
+            g = torch.cuda.CUDAGraph()
+            # eager first (first-call set-up), then captured
+            qkn.decode(base.dims, base.cache, base.q_tilde, base.a_q, base.q_rope_hat, bt, lens, s_q, ws, outs[k],
+                       lses[k], vis_end=ve)
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                ev.record(e[0], stream.cuda_stream)
+                qkn.decode(base.dims, base.cache, base.q_tilde, base.a_q, base.q_rope_hat, bt, lens, s_q, ws,
+                           outs[k], lses[k], vis_end=ve)
+                ev.record(e[1], stream.cuda_stream)
+            graphs.append((g, e))
+        qkn.merge_partials(base.dims, outs, lses, out, lse)
+        em = [ev.create() for _ in range(2)]
+        gm = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gm, stream=stream, capture_error_mode="relaxed"):
+            ev.record(em[0], stream.cuda_stream)
+            qkn.merge_partials(base.dims, outs, lses, out, lse)
+            ev.record(em[1], stream.cuda_stream)
+    torch.cuda.synchronize(device)
+    slice_ms = [[] for _ in range(world)]
+    merge_ms = []
+    with torch.cuda.stream(stream):
+        for _ in range(rounds):
+            for k, (g, e) in enumerate(graphs):
+                g.replay()
+                stream.synchronize()
+                slice_ms[k].append(ev.ms(e[0], e[1]))
+            gm.replay()
+            stream.synchronize()
+            merge_ms.append(ev.ms(em[0], em[1]))
+    assert base.device_status() == qkn.OK
+    part_bytes = B * s_q * H * (r * outs.element_size() + 4)
+    peer_gbs = 770.0                                  # measured NVLink peer copy, GB/s per direction
+    gather_us = part_bytes * (world - 1) / (peer_gbs * 1e9) * 1e6
+    slices = [statistics.median(v) * 1e3 for v in slice_ms]
+    merge_us = statistics.median(merge_ms) * 1e3
+    return {"world": world, "slice_us": slices, "merge_us": merge_us, "gather_bytes_per_rank": part_bytes,
+            "gather_us_estimate": gather_us, "step_us_estimate": max(slices) + gather_us + merge_us,
+            "what": ("each rank's slice decode (split-KV + merge of its own slices) and the merge of the "
+                     "ranks' partials, timed on one GPU (CUDA events, decode-only graphs); the all-gather "
+                     "is estimated at the measured 770 GB/s NVLink peer copy, not run")}
+
+
 def workload_config(wl, inp, world: int) -> dict:
     """The workload part of the JSON line's config, the same for both arms."""
     return {"workload": wl.name, "batch_per_gpu": wl.batch, "s_q": wl.s_q, "heads": wl.heads, "groups": wl.groups,
