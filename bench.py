@@ -649,7 +649,7 @@ def cp_emulate(world: int, base, inp, device, ev, stream, rounds: int = 10) -> d
     lse = torch.empty((B, s_q, H), dtype=torch.float32, device=device)
     views = []
     for k in range(world):
-        bt, lens, ve = cp.rank_view(inp.block_table, inp.seq_lens, k, world)
+        bt, lens, ve = cp.rank_view(inp.block_table, inp.seq_lens, k, world, s_q)
         views.append([torch.from_numpy(x).to(device) for x in (bt, lens, ve)])
     graphs = []
     with torch.cuda.stream(stream):

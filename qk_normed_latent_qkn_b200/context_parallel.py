@@ -12,8 +12,9 @@ on GPUs.  Host logic only: every arithmetic step runs in libqkn.
 
 Slices: sequence b has ``n_b = ceil(L_b / 64)`` pages; rank k of W takes
 pages ``[floor(n_b k / W), floor(n_b (k + 1) / W))``.  Every slice must hold
-at least ``s_q`` tokens, so ``n_b >= 2 W`` is required (each slice then
-spans at least two pages).
+at least ``s_q`` tokens (the decode's length check): ``n_b >= 2 W`` pages per
+sequence, so that each slice spans at least two pages, and enough of them for
+a longer query chunk.
 """
 from __future__ import annotations
 
@@ -27,7 +28,7 @@ from . import merge_partials
 BLOCK = 64
 
 
-def page_slices(seq_lens, world: int) -> np.ndarray:
+def page_slices(seq_lens, world: int, s_q: int = 1) -> np.ndarray:
     """[world, B, 2] int64: the page range (lo, hi) of each rank for each sequence."""
     lens = np.asarray(seq_lens, dtype=np.int64)
     n = (lens + BLOCK - 1) // BLOCK
@@ -38,15 +39,19 @@ def page_slices(seq_lens, world: int) -> np.ndarray:
                          f"sequence (shortest: {int(n.min())})")
     k = np.arange(world + 1, dtype=np.int64)[:, None]
     bounds = (n[None, :] * k) // world                  # [world + 1, B]
-    return np.stack([bounds[:-1], bounds[1:]], axis=-1)
+    sl = np.stack([bounds[:-1], bounds[1:]], axis=-1)
+    tokens = np.minimum(lens[None, :], sl[..., 1] * BLOCK) - sl[..., 0] * BLOCK
+    if np.any(tokens < s_q):
+        raise ValueError(f"a slice over {world} ranks would hold fewer than s_q = {s_q} tokens")
+    return sl
 
 
-def rank_view(block_table, seq_lens, rank: int, world: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+def rank_view(block_table, seq_lens, rank: int, world: int, s_q: int = 1) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """The decode inputs of one rank: its block table (each row starts at the slice's first page),
     its token counts and the causal limit's end in the slice's numbering (vis_end)."""
     bt = np.asarray(block_table, dtype=np.int32)
     lens = np.asarray(seq_lens, dtype=np.int64)
-    sl = page_slices(lens, world)[rank]                 # [B, 2]
+    sl = page_slices(lens, world, s_q)[rank]            # [B, 2]
     width = int((sl[:, 1] - sl[:, 0]).max())
     out = np.zeros((bt.shape[0], width), dtype=np.int32)
     for b, (lo, hi) in enumerate(sl):
@@ -58,7 +63,7 @@ def rank_view(block_table, seq_lens, rank: int, world: int) -> Tuple[np.ndarray,
 
 def slice_decode(session, block_table, seq_lens, s_q: int, rank: int, world: int, **kw):
     """This rank's partial result (out [B, s_q, H, r], lse [B, s_q, H]) for its page slices."""
-    bt, lens, vis_end = rank_view(block_table, seq_lens, rank, world)
+    bt, lens, vis_end = rank_view(block_table, seq_lens, rank, world, s_q)
     return session.decode(bt, lens, s_q, vis_end=vis_end, **kw)
 
 

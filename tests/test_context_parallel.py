@@ -33,6 +33,8 @@ def test_slices_partition_every_sequence(world):
 def test_too_short_sequences_are_refused():
     with pytest.raises(ValueError):
         cp.page_slices([64 * 7], 4)                          # 7 pages < 2 x 4
+    with pytest.raises(ValueError):
+        cp.page_slices([64 * 8], 4, s_q=200)                 # slices of 128 tokens < s_q
 
 
 def test_rank_view():

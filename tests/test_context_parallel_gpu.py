@@ -99,3 +99,12 @@ def test_merge_kernel_against_its_definition():
     assert (o[7] == 0).all() and np.isneginf(lse.cpu().numpy()[7])
     lg = lse.cpu().numpy()
     assert np.abs(lg[ok] - lref[ok]).max() <= 1e-4
+
+
+def test_context_parallel_over_a_prefill_chunk():
+    # 200 new tokens per sequence after a history, over 2 ranks: the decode skips each row tile's
+    # invisible pages counting from vis_end, and whole segments go straight to each rank's output
+    inp = make_inputs(WORKLOADS["prefill_mla_bf16"].with_(batch=2, s_q=200, context=(900, 1500), seed=95))
+    s = session_from_inputs(inp)
+    o, lse = _cp_decode(s, inp, 2)
+    assert_close_to_oracle(inp, o, lse, what="prefill chunk over 2 ranks")

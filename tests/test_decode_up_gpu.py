@@ -134,3 +134,13 @@ def test_full_size_headline_workload_sampled():
     order = np.argsort(inp.seq_lens)
     sample = sorted({int(order[0]), int(order[len(order) // 2]), int(order[-1])})
     _assert_up_close(inp, o_v, lse, seqs=sample, what="large_mla_bf16 full size")
+
+
+def test_decode_up_after_a_prefill_chunk():
+    # long query chunk: the decode's row tiles skip their invisible pages (items that may be empty
+    # write zero partials with lse = -inf) and the fused merge applies W^UV to the merged rows
+    inp = make_inputs(WORKLOADS["prefill_mla_bf16"].with_(batch=2, s_q=150, context=(300, 700), seed=77))
+    s = session_from_inputs(inp)
+    o_v, lse = _run_up(s, inp)
+    assert s.device_status() == qkn.OK
+    _assert_up_close(inp, o_v, lse, what="prefill chunk")
