@@ -317,6 +317,25 @@ def check_brute_force_causal():
             assert abs(lse[0, j, h] - (mx + math.log(s))) < 1e-12
 
 
+def check_prefill_rows_are_prefix_decodes():
+    # a whole sequence as queries (s_q = L): query j sits at position j and sees tokens 0 .. j, so
+    # its output is the one-query decode of the length-(j + 1) prefix, and query 0 returns c_0
+    import dataclasses
+    L = 7
+    wl = TINY.with_(name="pin_prefill", batch=1, s_q=L, context=L, seed=11)
+    inp = make_inputs(wl)
+    o, lse = oracle.decode(inp)
+    np.testing.assert_allclose(o[0, 0], np.broadcast_to(inp.c[0], o[0, 0].shape), rtol=0, atol=1e-14)
+    for j in range(L):
+        pre = dataclasses.replace(
+            inp, wl=wl.with_(s_q=1, context=j + 1), seq_lens=np.array([j + 1], dtype=np.int32),
+            tok_off=np.array([0, j + 1]), c=inp.c[:j + 1], k_rope=inp.k_rope[:j + 1],
+            q=inp.q[:, j:j + 1], q_rope=inp.q_rope[:, j:j + 1])
+        oj, lj = oracle.decode(pre)
+        np.testing.assert_allclose(o[0, j], oj[0, 0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lse[0, j], lj[0, 0], rtol=1e-12, atol=1e-14)
+
+
 # --------------------------------------------------------------------------
 # 7. RoPE: a rotation whose inner products depend on relative position only.
 # --------------------------------------------------------------------------
@@ -397,6 +416,7 @@ ALL_CHECKS = [
     check_identical_tokens_return_that_token,
     check_against_library_attention,
     check_brute_force_causal,
+    check_prefill_rows_are_prefix_decodes,
     check_rope_properties,
     check_permutation_invariance,
     check_up_projection_equals_explicit_values,
