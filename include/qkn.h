@@ -190,6 +190,9 @@ QKN_EXPORT qkn_status qkn_append(const qkn_dims* dims, const qkn_cache* cache,
                       const int32_t* slot, const int32_t* pos, int32_t n_tok,
                       const float* w_k, const float* key_gram, const float* gamma_kr,
                       void* stream);
+/* (qkn_append, qkn_append_absorb: a token whose slot id lies outside
+ * [0, num_blocks * block_size) is skipped: nothing of it is written, so that a
+ * bad id cannot write outside the pool.) */
 
 /* qkn_absorb_query — fold the static norm weights into the query
  * (technical summary, Metodología item 1 and the decode-logit equation).

@@ -178,6 +178,7 @@ qkn_status append_args(const qkn_dims* dims, const qkn_cache* cache, const void*
   a->groups = dims->num_groups;
   a->width = (dims->num_heads / dims->num_groups) * dims->d_h;
   a->ncols = key_gram ? dims->r_kv : a->width;
+  a->n_slots = (int64_t)cache->num_blocks * kBlockSize;
   a->eps = dims->eps;
   a->rope_theta = dims->rope_theta;
   a->freq = rope_freqs(dims);

@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(256) append_copy_kernel(const __grid_constant_
   if (warp >= a.n_tok) return;
   append_token<T>(a, warp, lane, buf[threadIdx.x >> 5]);
   const int64_t slot = a.slot[warp];
+  if (slot < 0 || slot >= a.n_slots) return;       // outside the pool: the token is skipped
   for (int g = lane; g < a.groups; g += 32) a.a_k[slot * a.groups + g] = 0.f;
 }
 
@@ -57,7 +58,9 @@ __global__ void append_finalize_kernel(AppendArgs a) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n_tok * a.groups) return;
   const int t = i / a.groups, g = i - t * a.groups;
-  float* p = a.a_k + (int64_t)a.slot[t] * a.groups + g;
+  const int64_t slot = a.slot[t];
+  if (slot < 0 || slot >= a.n_slots) return;
+  float* p = a.a_k + slot * a.groups + g;
   *p = 1.0f / sqrtf(*p / (float)a.width + a.eps);
 }
 
@@ -162,8 +165,9 @@ __global__ void __launch_bounds__(kGThreads) keystat_gemm_kernel(const __grid_co
     }
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (tx == 0 && t < ntok) {
-      const int64_t idx = (int64_t)a.slot[t0 + t] * a.groups + g;
+    const int64_t s_t = t < ntok ? (int64_t)a.slot[t0 + t] : -1;
+    if (tx == 0 && t < ntok && s_t >= 0 && s_t < a.n_slots) {
+      const int64_t idx = s_t * a.groups + g;
       if constexpr (FUSED) {
         float* accp = reinterpret_cast<float*>(a.ak_scratch + 2 * idx);
         unsigned int* cnt = a.ak_scratch + 2 * idx + 1;

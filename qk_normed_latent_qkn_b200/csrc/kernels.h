@@ -29,6 +29,7 @@ struct AppendArgs {
   const float* gamma_kr;   // [d_rope]
   int32_t n_tok, r, d_rope, groups, width;   // width = n_g * d_h
   int32_t ncols;           // columns of the key-statistic matrix: r with key_gram, else width
+  int64_t n_slots;         // cache slots (num_blocks * block_size): a token whose slot is outside is skipped
   float eps, rope_theta;
   RopeFreqs freq;
 };

@@ -18,6 +18,7 @@ namespace qkn {
 template <typename T>
 __device__ __forceinline__ void append_token(const AppendArgs& a, int i, int lane, float* row) {
   const int64_t slot = a.slot[i];
+  if (slot < 0 || slot >= a.n_slots) return;        // outside the pool: the token is skipped
   const int32_t pos = a.pos[i];
   // latent row: 16-byte vectors (rows are a multiple of 16 bytes)
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(a.c_new) + (int64_t)i * a.r);
@@ -197,8 +198,9 @@ __device__ __forceinline__ void keyrms_block(const AppendArgs& a, int bx, int by
     float v = (n < ncols) ? z * (gram ? cs[t * a.r + n] : z) : 0.f;
 #pragma unroll
     for (int o = kRmsCols / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (col == 0 && t < ntok) {
-      const int64_t i = (int64_t)a.slot[t0 + t] * a.groups + g;
+    const int64_t s_t = t < ntok ? (int64_t)a.slot[t0 + t] : -1;
+    if (col == 0 && t < ntok && s_t >= 0 && s_t < a.n_slots) {
+      const int64_t i = s_t * a.groups + g;
       if constexpr (FUSED) {
         float* acc = reinterpret_cast<float*>(a.ak_scratch + 2 * i);
         unsigned int* cnt = a.ak_scratch + 2 * i + 1;

@@ -9,6 +9,8 @@
   the oracle.
 - A block id outside the pool: the kernels clamp it to block 0 and record
   QKN_ERR_BOUNDS; the other sequences' results are unaffected.
+- A slot id outside the pool in an append: the token is skipped in every
+  append path (one launch, three launches, the GEMM form for many tokens).
 """
 import numpy as np
 import pytest
@@ -91,3 +93,43 @@ def test_block_id_out_of_range_is_clamped_and_reported(kernel):
     l = lse.cpu().numpy().astype(np.float64)
     # the other sequences read only their own pages
     assert_close_to_oracle(inp, o, l, seqs=range(1, inp.wl.batch), what="sequences without the bad id")
+
+
+@pytest.mark.parametrize("n_bad, scratch", [(4, True), (4, False), (300, True)],
+                         ids=["one-launch", "three-launch", "gemm-path"])
+def test_append_skips_slots_outside_the_pool(n_bad, scratch):
+    # new tokens for the free slots at the end of each sequence's last page, mixed with tokens whose
+    # slot ids lie outside the pool (negative, and past its end): those are skipped, nothing is
+    # written outside the pool, and the valid tokens get their latent rows and a_k
+    import oracle
+    inp = make_inputs(CASES["grouped_mtp_bf16"])
+    s = session_from_inputs(inp)
+    if not scratch:
+        s.cache.ak_scratch = None                       # the three-launch append
+    pool = inp.num_blocks * 64
+    free = []
+    for b in range(inp.wl.batch):
+        L = int(inp.seq_lens[b])
+        last = int(inp.block_table[b, (L - 1) // 64])
+        free += [last * 64 + t for t in range(L % 64, 64)] if L % 64 else []
+    free = np.array(free[:6], dtype=np.int32)
+    assert free.size > 0
+    bad = np.array([-1 - k if k % 2 == 0 else pool + k for k in range(n_bad)], dtype=np.int32)
+    slots = np.concatenate([free, bad])
+    rng = np.random.default_rng(8)
+    n = slots.size
+    c = rng.standard_normal((n, inp.wl.r_kv)).astype(np.float32)
+    kr = rng.standard_normal((n, inp.wl.d_rope)).astype(np.float32)
+    pos = np.arange(n, dtype=np.int32)
+    a_k_before = s.cache.a_k.clone()
+    s.append(c, kr, slots, pos)
+    torch.cuda.synchronize()
+    a_k = s.cache.a_k.reshape(-1, inp.wl.groups).cpu().numpy()
+    lat = s.cache.latent.reshape(pool, -1).float().cpu().numpy()
+    c_bf16 = torch.from_numpy(c).to(torch.bfloat16).float().numpy()
+    ref = oracle.key_inv_rms(c_bf16[:free.size].astype(np.float64), inp.w_k, inp.wl.eps)
+    np.testing.assert_allclose(a_k[free], ref, rtol=2e-5)
+    assert (lat[free] == c_bf16[:free.size]).all()
+    # every other slot of the pool keeps its a_k
+    others = torch.from_numpy(np.setdiff1d(np.arange(pool), free)).to(s.cache.a_k.device)
+    assert torch.equal(s.cache.a_k.reshape(-1, inp.wl.groups)[others], a_k_before.reshape(-1, inp.wl.groups)[others])
