@@ -29,6 +29,16 @@ Readings of points the pages leave open:
   * values are the unnormalised latents c_t; the output lives in latent space;
   * a query sees the keys whose position is <= its own position.
 
+The GQA route of GQLA (section 2, "Ruta GQA") is here too: the latent is
+expanded once per token into one key head and one value head per KV group,
+and decode is ordinary grouped-query attention over those cached keys and
+values.  Readings: the group's key is RMS-normalised over its d_h columns
+after the up-projection with the group's gamma_k (the QK-Normed key norm,
+with one key head per group); the RoPE block and the queries as above; the
+output is the value-space o_v [s_q, H, d_v].  Sparse GQLA (section 2, "GQLA
+Disperso") is read as: every (query token, KV group) pair attends only to
+a given list of its visible tokens, the n_g heads of the group sharing it.
+
 Pins (tests/test_oracle_pins.py): exact absorbed == explicit equality in
 rational arithmetic; invariance of the logits to rescaling c_t; softmax rows
 summing to 1; closed forms (one token, zero queries, identical tokens); a
@@ -44,7 +54,9 @@ from typing import Iterable, Optional, Tuple
 import numpy as np
 
 __all__ = ["inv_rms", "rms_norm", "rope", "key_inv_rms", "rope_keys", "absorbed_query",
-           "sequence_logits", "decode", "decode_sequence", "up_project"]
+           "sequence_logits", "decode", "decode_sequence", "up_project", "group_keys",
+           "group_values",
+           "gqa_logits", "gqa_decode_sequence", "gqa_decode"]
 
 
 def inv_rms(x: np.ndarray, eps: float) -> np.ndarray:
@@ -214,3 +226,104 @@ def up_project(o_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     for h in range(w.shape[0]):
         out[..., h, :] = o[..., h, :] @ w[h]
     return out
+
+
+def group_keys(c: np.ndarray, w_uk: np.ndarray, gamma_k: np.ndarray, eps: float) -> np.ndarray:
+    """Keys of the GQA route: k_{t,g} = RMSNorm(c_t W^UK_g) gamma_k[g] over the group's d_h columns.
+
+    The latent expanded into one key head per KV group, which that route
+    caches (GQLA summary, section 2, "Ruta GQA"), normalised after its
+    up-projection as the QK-Normed key is (technical summary, "Planteamiento
+    del Problema").  ``c`` [T, r], ``w_uk`` [g, r, d_h], ``gamma_k`` [g, d_h];
+    returns [T, g, d_h].
+    """
+    c = np.asarray(c, dtype=np.float64)
+    wk = np.asarray(w_uk, dtype=np.float64)
+    return np.stack([rms_norm(c @ wk[g], np.asarray(gamma_k[g], np.float64), eps) for g in range(wk.shape[0])],
+                    axis=1)
+
+
+def group_values(c: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
+    """Values of the GQA route: v_{t,g} = c_t W^UV_g (GQLA summary, section 2, "Ruta GQA").
+
+    ``c`` [T, r], ``w_uv`` [g, r, d_v]; returns [T, g, d_v].
+    """
+    c = np.asarray(c, dtype=np.float64)
+    wv = np.asarray(w_uv, dtype=np.float64)
+    return np.stack([c @ wv[g] for g in range(wv.shape[0])], axis=1)
+
+
+def gqa_logits(inp, b: int, w_uk: np.ndarray, gamma_k: np.ndarray,
+               selection: Optional[np.ndarray] = None) -> np.ndarray:
+    """Logits of grouped-query attention over the expanded keys of sequence b, [s_q, H, L].
+
+    l[j, h, t] = sigma * (RMSNorm(q_jh) . k_{t,g(h)} + RoPE(RMSNorm(q^R_jh)) . RoPE(RMSNorm(k^R_t))),
+    g(h) = h // n_g; -inf where key t sits after query j, and, with ``selection``
+    ([s_q, g, K] token positions, -1 = none), where t is not listed for (j, g(h))
+    (GQLA summary, section 2, "Ruta GQA" and "GQLA Disperso").
+    """
+    wl = inp.wl
+    sl = inp.sequence(b)
+    c = np.asarray(inp.c[sl], dtype=np.float64)
+    L = c.shape[0]
+    qpos = inp.query_positions()[b]
+    H, ng = wl.heads, wl.heads_per_group
+    k = group_keys(c, w_uk, gamma_k, wl.eps)                                       # [L, g, d_h]
+    qh = rms_norm(inp.q[b], inp.gamma_q, wl.eps)                                   # [s_q, H, d_h]
+    qrh = rope(rms_norm(inp.q_rope[b], inp.gamma_qr, wl.eps), pos=qpos[:, None], theta=wl.rope_theta)
+    krh = rope_keys(inp.k_rope[sl], inp.gamma_kr, np.arange(L), wl.eps, wl.rope_theta)
+    grp = np.arange(H) // ng
+    logits = np.einsum("jhd,thd->jht", qh, k[:, grp, :]) + np.einsum("jhd,td->jht", qrh, krh)
+    logits *= wl.softmax_scale
+    visible = np.arange(L)[None, :] <= qpos[:, None]                               # [s_q, L]
+    mask = np.broadcast_to(visible[:, None, :], logits.shape).copy()
+    if selection is not None:
+        listed = np.zeros((wl.s_q, wl.groups, L), dtype=bool)
+        for j in range(wl.s_q):
+            for g in range(wl.groups):
+                idx = np.asarray(selection[j, g])
+                idx = idx[(idx >= 0) & (idx < L)]
+                listed[j, g, idx] = True
+        mask &= listed[:, grp, :]
+    logits[~mask] = -np.inf
+    return logits
+
+
+def gqa_decode_sequence(inp, b: int, w_uk: np.ndarray, gamma_k: np.ndarray, w_uv: np.ndarray,
+                        selection: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax over the listed / visible tokens, then the weighted sum of the group's values.
+
+    Returns (o_v [s_q, H, d_v], lse [s_q, H]) for sequence b; a row with no
+    token gives zeros and lse = -inf.
+    """
+    wl = inp.wl
+    c = np.asarray(inp.c[inp.sequence(b)], dtype=np.float64)
+    v = group_values(c, w_uv)                                                      # [L, g, d_v]
+    l = gqa_logits(inp, b, w_uk, gamma_k, selection)
+    m = l.max(axis=-1, keepdims=True)
+    has = np.isfinite(m)
+    e = np.exp(l - np.where(has, m, 0.0))
+    s = e.sum(axis=-1, keepdims=True)
+    p = np.where(has, e / np.where(has, s, 1.0), 0.0)
+    lse = np.where(has, m + np.log(np.where(has, s, 1.0)), -np.inf)[..., 0]
+    grp = np.arange(wl.heads) // wl.heads_per_group
+    o = np.einsum("jht,thd->jhd", p, v[:, grp, :])
+    return o, lse
+
+
+def gqa_decode(inp, w_uk: np.ndarray, gamma_k: np.ndarray, w_uv: np.ndarray,
+               seqs: Optional[Iterable[int]] = None,
+               selection: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """GQA-route decode outputs for the listed sequences (all by default).
+
+    ``selection`` [B, s_q, g, K] selects sparse attention.  Returns
+    (o_v [B, s_q, H, d_v], lse [B, s_q, H]); rows of sequences not listed are NaN.
+    """
+    wl = inp.wl
+    B = wl.batch
+    o = np.full((B, wl.s_q, wl.heads, w_uv.shape[2]), np.nan)
+    lse = np.full((B, wl.s_q, wl.heads), np.nan)
+    for b in (range(B) if seqs is None else seqs):
+        o[b], lse[b] = gqa_decode_sequence(inp, b, w_uk, gamma_k, w_uv,
+                                           None if selection is None else selection[b])
+    return o, lse

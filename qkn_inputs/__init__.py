@@ -20,7 +20,16 @@ Value recipe (identical for every workload):
   * eps = 1e-6, RoPE base 10000.
 Draw order from one ``numpy.random.Generator(PCG64(seed))``: sequence lengths,
 block permutation, s_t, c, k^R, q, q^R, W^K, gamma_q, gamma_k, gamma_qR,
-gamma_kR, W^UV (value up-projection, N(0, 1/r_kv)).  Values are drawn in fp32
+gamma_kR, W^UV (value up-projection, N(0, 1/r_kv)).
+
+Tied groups (``Workload.tied_groups``): the GQLA parameterisation, where the
+up-projections are indexed by KV group rather than by head ("GQLA", section
+2, Arquitectura): one key head W^UK_g [r, d_h] with its norm weight
+gamma_k,g [d_h] and one value head W^UV_g [r, d_v] per group.  They are drawn
+with the group's shape in the same order, then laid out per head (W^K_g as
+n_g copies of W^UK_g side by side, gamma_k and W^UV repeated over the
+group's heads), so that the per-head arrays describe the same model and the
+absorbed route reads them unchanged.  Values are drawn in fp32
 and, for bf16 workloads, the stored activations (c, k^R, q, q^R) and W^UV
 (which the library reads in the storage type) are rounded once to bf16 (round
 to nearest even); the other weights and the gammas stay fp32.
@@ -54,6 +63,7 @@ class Workload:
     seed: int = 0
     block_size: int = BLOCK_SIZE
     d_v: int = 128                         # per-head value width of the output up-projection
+    tied_groups: bool = False              # one key head and one value head per KV group (GQLA)
 
     @property
     def heads_per_group(self) -> int:
@@ -86,9 +96,13 @@ WORKLOADS = {
     # query, causal (s_q = context)
     "prefill_mla_bf16": Workload("prefill_mla_bf16", batch=2, s_q=2048, heads=16, groups=1, r_kv=512,
                                  d_h=128, d_rope=64, context=2048, paged=True, dtype="bf16"),
+    # GQLA's configuration for its GQA route (h_q = 128, g = 8, so h_q / g = 16, with a two-token
+    # MTP step): keys and values expanded per group; the context mix of the large MLA case
+    "gqla_gqa_bf16": Workload("gqla_gqa_bf16", batch=32, s_q=2, heads=128, groups=8, r_kv=512, d_h=128,
+                              d_rope=64, context=(1024, 32768), paged=True, dtype="bf16", tied_groups=True),
 }
 WORKLOAD_ORDER = ["tiny_f32", "small_mla_bf16", "large_mla_bf16", "long_ctx_bf16", "prefill_mla_bf16",
-                  "grouped_mtp_bf16"]
+                  "grouped_mtp_bf16", "gqla_gqa_bf16"]
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
@@ -159,6 +173,15 @@ class Inputs:
     def sequence(self, b: int) -> slice:
         return slice(int(self.tok_off[b]), int(self.tok_off[b + 1]))
 
+    def group_weights(self) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+        """The per-group weights of a tied-groups workload, in the group layout:
+        W^UK [g, r, d_h], gamma_k [g, d_h], W^UV [g, r, d_v] (slices of the per-head arrays)."""
+        if not self.wl.tied_groups:
+            raise ValueError("group weights exist only for a tied-groups workload")
+        ng = self.wl.heads_per_group
+        return (np.ascontiguousarray(self.w_k[:, :, :self.wl.d_h]), np.ascontiguousarray(self.gamma_k[::ng]),
+                np.ascontiguousarray(self.w_uv[::ng]))
+
 
 def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
                 seq_lens: Optional[Sequence[int]] = None) -> Inputs:
@@ -204,13 +227,20 @@ def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
     q = rng.standard_normal((B, wl.s_q, wl.heads, wl.d_h), dtype=f32)
     q_rope = rng.standard_normal((B, wl.s_q, wl.heads, wl.d_rope), dtype=f32)
     ng = wl.heads_per_group
-    w_k = rng.standard_normal((wl.groups, wl.r_kv, ng * wl.d_h), dtype=f32) * f32(1.0 / np.sqrt(wl.r_kv))
+    kh = 1 if wl.tied_groups else ng                    # key heads drawn per group
+    vh = wl.groups if wl.tied_groups else wl.heads      # value heads drawn
+    w_k = rng.standard_normal((wl.groups, wl.r_kv, kh * wl.d_h), dtype=f32) * f32(1.0 / np.sqrt(wl.r_kv))
     gamma_q = (1.0 + 0.1 * rng.standard_normal((wl.heads, wl.d_h), dtype=f32)).astype(f32)
-    gamma_k = (1.0 + 0.1 * rng.standard_normal((wl.heads, wl.d_h), dtype=f32)).astype(f32)
+    gamma_k = (1.0 + 0.1 * rng.standard_normal((wl.groups * kh, wl.d_h), dtype=f32)).astype(f32)
     gamma_qr = (1.0 + 0.1 * rng.standard_normal((wl.heads, wl.d_rope), dtype=f32)).astype(f32)
     gamma_kr = (1.0 + 0.1 * rng.standard_normal(wl.d_rope, dtype=f32)).astype(f32)
     # drawn last, so that every value above is the same with or without it
-    w_uv = rng.standard_normal((wl.heads, wl.r_kv, wl.d_v), dtype=f32) * f32(1.0 / np.sqrt(wl.r_kv))
+    w_uv = rng.standard_normal((vh, wl.r_kv, wl.d_v), dtype=f32) * f32(1.0 / np.sqrt(wl.r_kv))
+    if wl.tied_groups:
+        # lay the group's single key and value head out over its n_g query heads
+        w_k = np.ascontiguousarray(np.tile(w_k, (1, 1, ng)))
+        gamma_k = np.ascontiguousarray(np.repeat(gamma_k, ng, axis=0))
+        w_uv = np.ascontiguousarray(np.repeat(w_uv, ng, axis=0))
 
     if wl.dtype == "bf16":
         c, k_rope, q, q_rope, w_uv = (round_to_bf16(a) for a in (c, k_rope, q, q_rope, w_uv))
@@ -221,3 +251,27 @@ def make_inputs(wl: Union[str, Workload], seed: Optional[int] = None,
                   c=np.ascontiguousarray(c, f32), k_rope=np.ascontiguousarray(k_rope, f32),
                   q=q, q_rope=q_rope, w_k=w_k, gamma_q=gamma_q, gamma_k=gamma_k,
                   gamma_qr=gamma_qr, gamma_kr=gamma_kr, w_uv=w_uv)
+
+
+def make_selection(inp: Inputs, k: int, seed: int = 0) -> np.ndarray:
+    """Token selections for sparse attention over the GQA route: [B, s_q, g, k] int32.
+
+    For query token j of sequence b and KV group g, ``k`` distinct positions drawn uniformly
+    without replacement from the tokens that query can see (positions 0 .. L_b - s_q + j), in
+    random order; when fewer are visible, all of them, then -1 (no token) in the remaining
+    entries.  Drawn from ``numpy.random.Generator(PCG64(seed))``, one draw per (b, j, g) in
+    that order.
+    """
+    wl = inp.wl
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = np.full((wl.batch, wl.s_q, wl.groups, k), -1, dtype=np.int32)
+    qpos = inp.query_positions()
+    for b in range(wl.batch):
+        for j in range(wl.s_q):
+            n = int(qpos[b, j]) + 1
+            for g in range(wl.groups):
+                if n <= k:
+                    out[b, j, g, :n] = rng.permutation(n)
+                else:
+                    out[b, j, g] = rng.choice(n, size=k, replace=False)
+    return out

@@ -18,7 +18,7 @@ import numpy as np
 import torch
 
 import oracle
-from qkn_inputs import Workload, make_inputs
+from qkn_inputs import Workload, make_inputs, make_selection
 
 TINY = Workload("pin_tiny", batch=2, s_q=1, heads=4, groups=2, r_kv=8, d_h=4, d_rope=4,
                 context=(5, 19), paged=True, dtype="f32", seed=3)
@@ -404,6 +404,138 @@ def check_up_projection_selectors():
         assert np.array_equal(got[:, :, h], o[:, :, h][..., cols[h]])
 
 
+# --------------------------------------------------------------------------
+# 10. The GQA route (GQLA summary, section 2, "Ruta GQA"): keys and values
+#     expanded per group, grouped-query attention over them.  Sparse GQLA
+#     ("GQLA Disperso"): each (query token, group) attends to a token list.
+# --------------------------------------------------------------------------
+TINY_GQLA = Workload("pin_gqla", batch=2, s_q=2, heads=6, groups=2, r_kv=8, d_h=4, d_rope=4,
+                     context=(5, 19), paged=True, dtype="f32", seed=13, d_v=3, tied_groups=True)
+
+
+def check_gqa_route_equals_absorbed_route():
+    """With one key and one value head per group, the two routes over the same weights agree
+    (GQLA summary, section 2: two algebraically equivalent decode routes over the same parameters)."""
+    for wl in (TINY_GQLA, TINY_GQLA.with_(s_q=1, seed=14)):
+        inp = make_inputs(wl)
+        o_gqa, lse_gqa = oracle.gqa_decode(inp, *inp.group_weights())
+        o_lat, lse = oracle.decode(inp)
+        np.testing.assert_allclose(o_gqa, oracle.up_project(o_lat, inp.w_uv), rtol=1e-11, atol=1e-13)
+        np.testing.assert_allclose(lse_gqa, lse, rtol=1e-12, atol=1e-12)
+
+
+def _gqa_group_weights(wl, seed):
+    rng = np.random.default_rng(seed)
+    w_uk = rng.standard_normal((wl.groups, wl.r_kv, wl.d_h)) / math.sqrt(wl.r_kv)
+    gamma_k = 1.0 + 0.1 * rng.standard_normal((wl.groups, wl.d_h))
+    w_uv = rng.standard_normal((wl.groups, wl.r_kv, wl.d_v)) / math.sqrt(wl.r_kv)
+    return w_uk, gamma_k, w_uv
+
+
+def check_gqa_against_library_attention():
+    """torch fp64 grouped-query scaled_dot_product_attention on keys and values this check forms."""
+    wl = TINY_GQLA.with_(tied_groups=False, seed=15)
+    inp = make_inputs(wl)
+    w_uk, gamma_k, w_uv = _gqa_group_weights(wl, 16)
+    o_ref, lse_ref = oracle.gqa_decode(inp, w_uk, gamma_k, w_uv)
+    sigma = 1.0 / math.sqrt(wl.d_h + wl.d_rope)
+    for b in range(wl.batch):
+        sl = inp.sequence(b)
+        c = torch.tensor(inp.c[sl], dtype=torch.float64)
+        L = c.shape[0]
+        z = torch.einsum("tr,grd->gtd", c, torch.tensor(w_uk))
+        k = z / torch.sqrt((z * z).mean(-1, keepdim=True) + wl.eps) * torch.tensor(gamma_k)[:, None, :]
+        v = torch.einsum("tr,grd->gtd", c, torch.tensor(w_uv))
+        krs = inp.k_rope[sl].astype(np.float64)
+        kr = torch.tensor(np.stack([_rotate_complex(
+            krs[t] * inp.gamma_kr.astype(np.float64) / math.sqrt(float(np.mean(krs[t] ** 2)) + wl.eps),
+            t, wl.rope_theta) for t in range(L)]))
+        qv = torch.tensor(inp.q[b], dtype=torch.float64)
+        qn = qv / torch.sqrt((qv * qv).mean(-1, keepdim=True) + wl.eps) * torch.tensor(inp.gamma_q, dtype=torch.float64)
+        qr = np.empty((wl.s_q, wl.heads, wl.d_rope))
+        for j in range(wl.s_q):
+            for h in range(wl.heads):
+                x = inp.q_rope[b, j, h].astype(np.float64)
+                qr[j, h] = _rotate_complex(x * inp.gamma_qr[h].astype(np.float64) / math.sqrt(float(np.mean(x * x)) + wl.eps),
+                                           L - wl.s_q + j, wl.rope_theta)
+        qcat = torch.cat([qn, torch.tensor(qr)], -1).permute(1, 0, 2)                # [H, s_q, d]
+        kcat = torch.cat([k, kr.unsqueeze(0).expand(wl.groups, L, wl.d_rope)], -1)  # [g, L, d]
+        mask = (torch.arange(L)[None, :] <= (L - wl.s_q + torch.arange(wl.s_q))[:, None])
+        out = torch.nn.functional.scaled_dot_product_attention(qcat, kcat, v, attn_mask=mask, scale=sigma,
+                                                               enable_gqa=True)     # [H, s_q, d_v]
+        np.testing.assert_allclose(o_ref[b], out.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+
+
+def check_gqa_single_token_returns_value():
+    wl = TINY_GQLA.with_(s_q=1, context=1, seed=17)
+    inp = make_inputs(wl, seq_lens=[1, 1])
+    w_uk, gamma_k, w_uv = _gqa_group_weights(wl, 18)
+    o, _ = oracle.gqa_decode(inp, w_uk, gamma_k, w_uv)
+    ng = wl.heads // wl.groups
+    for b in range(wl.batch):
+        c0 = inp.c[inp.sequence(b)][0].astype(np.float64)
+        for h in range(wl.heads):
+            want = [sum(c0[i] * w_uv[h // ng, i, d] for i in range(wl.r_kv)) for d in range(wl.d_v)]
+            np.testing.assert_allclose(o[b, 0, h], want, rtol=1e-12, atol=1e-14)
+
+
+def check_gqa_sparse_full_selection_equals_dense():
+    """Listing every visible token, in any order, is dense attention."""
+    inp = make_inputs(TINY_GQLA)
+    wts = inp.group_weights()
+    sel = make_selection(inp, 32, seed=19)
+    o_s, lse_s = oracle.gqa_decode(inp, *wts, selection=sel)
+    o_d, lse_d = oracle.gqa_decode(inp, *wts)
+    np.testing.assert_allclose(o_s, o_d, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse_s, lse_d, rtol=1e-12, atol=1e-14)
+    none = np.full_like(sel, -1)
+    o_n, lse_n = oracle.gqa_decode(inp, *wts, selection=none)
+    assert (o_n == 0).all() and np.isneginf(lse_n).all()
+
+
+def check_gqa_sparse_brute_force():
+    """Plain Python loops over a three-token selection per (query token, group)."""
+    wl = Workload("pin_sparse", batch=1, s_q=2, heads=4, groups=2, r_kv=3, d_h=2, d_rope=2,
+                  context=9, paged=False, dtype="f32", eps=0.25, seed=21, d_v=2, tied_groups=True)
+    inp = make_inputs(wl)
+    w_uk, gamma_k, w_uv = inp.group_weights()
+    sel = make_selection(inp, 3, seed=22)
+    o, lse = oracle.gqa_decode(inp, w_uk, gamma_k, w_uv, selection=sel)
+    L, r, ng = 9, 3, 2
+    c = [[float(inp.c[t, i]) for i in range(r)] for t in range(L)]
+    sigma = 1.0 / math.sqrt(wl.d_h + wl.d_rope)
+
+    def rmsinv(v):
+        return 1.0 / math.sqrt(sum(x * x for x in v) / len(v) + wl.eps)
+
+    def rot(v, pos):   # d = 2: one pair, frequency 1
+        return [v[0] * math.cos(pos) - v[1] * math.sin(pos), v[1] * math.cos(pos) + v[0] * math.sin(pos)]
+
+    for j in range(2):
+        qpos = L - 2 + j
+        for h in range(4):
+            g = h // ng
+            toks = [int(t) for t in sel[0, j, g] if t >= 0]
+            logits, vals = [], []
+            for t in toks:
+                z = [sum(c[t][i] * float(w_uk[g, i, d]) for i in range(r)) for d in range(2)]
+                key = [z[d] * rmsinv(z) * float(gamma_k[g, d]) for d in range(2)]
+                qv = [float(x) for x in inp.q[0, j, h]]
+                qn = [qv[d] * rmsinv(qv) * float(inp.gamma_q[h, d]) for d in range(2)]
+                kr = [float(x) for x in inp.k_rope[t]]
+                krn = rot([kr[d] * rmsinv(kr) * float(inp.gamma_kr[d]) for d in range(2)], t)
+                qr = [float(x) for x in inp.q_rope[0, j, h]]
+                qrn = rot([qr[d] * rmsinv(qr) * float(inp.gamma_qr[h, d]) for d in range(2)], qpos)
+                logits.append(sigma * (sum(a * b for a, b in zip(qn, key)) + sum(a * b for a, b in zip(qrn, krn))))
+                vals.append([sum(c[t][i] * float(w_uv[g, i, d]) for i in range(r)) for d in range(2)])
+            mx = max(logits)
+            ex = [math.exp(x - mx) for x in logits]
+            s = sum(ex)
+            want = [sum(ex[n] / s * vals[n][d] for n in range(len(toks))) for d in range(2)]
+            np.testing.assert_allclose(o[0, j, h], want, rtol=1e-12, atol=1e-14)
+            assert abs(lse[0, j, h] - (mx + math.log(s))) < 1e-12
+
+
 ALL_CHECKS = [
     check_absorbed_query_exact,
     check_absorbed_query_row_scale,
@@ -421,4 +553,9 @@ ALL_CHECKS = [
     check_permutation_invariance,
     check_up_projection_equals_explicit_values,
     check_up_projection_selectors,
+    check_gqa_route_equals_absorbed_route,
+    check_gqa_against_library_attention,
+    check_gqa_single_token_returns_value,
+    check_gqa_sparse_full_selection_equals_dense,
+    check_gqa_sparse_brute_force,
 ]
