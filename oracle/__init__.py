@@ -273,7 +273,10 @@ def gqa_logits(inp, b: int, w_uk: np.ndarray, gamma_k: np.ndarray,
     qrh = rope(rms_norm(inp.q_rope[b], inp.gamma_qr, wl.eps), pos=qpos[:, None], theta=wl.rope_theta)
     krh = rope_keys(inp.k_rope[sl], inp.gamma_kr, np.arange(L), wl.eps, wl.rope_theta)
     grp = np.arange(H) // ng
-    logits = np.einsum("jhd,thd->jht", qh, k[:, grp, :]) + np.einsum("jhd,td->jht", qrh, krh)
+    logits = np.empty((wl.s_q, H, L))
+    for g in range(wl.groups):                       # the group's n_g heads share its key head
+        logits[:, g * ng:(g + 1) * ng] = np.einsum("jmd,td->jmt", qh[:, g * ng:(g + 1) * ng], k[:, g, :])
+    logits = logits + np.einsum("jhd,td->jht", qrh, krh)
     logits *= wl.softmax_scale
     visible = np.arange(L)[None, :] <= qpos[:, None]                               # [s_q, L]
     mask = np.broadcast_to(visible[:, None, :], logits.shape).copy()
@@ -306,8 +309,10 @@ def gqa_decode_sequence(inp, b: int, w_uk: np.ndarray, gamma_k: np.ndarray, w_uv
     s = e.sum(axis=-1, keepdims=True)
     p = np.where(has, e / np.where(has, s, 1.0), 0.0)
     lse = np.where(has, m + np.log(np.where(has, s, 1.0)), -np.inf)[..., 0]
-    grp = np.arange(wl.heads) // wl.heads_per_group
-    o = np.einsum("jht,thd->jhd", p, v[:, grp, :])
+    ng = wl.heads_per_group
+    o = np.empty((wl.s_q, wl.heads, v.shape[2]))
+    for g in range(wl.groups):                       # ... and its value head
+        o[:, g * ng:(g + 1) * ng] = np.einsum("jmt,td->jmd", p[:, g * ng:(g + 1) * ng], v[:, g, :])
     return o, lse
 
 

@@ -34,15 +34,15 @@ MUTATIONS = {
                                  "out[..., h, :] = o[..., h, :] @ w[(h + 1) % w.shape[0]]"),
     "up_projection_rows_reversed": ("out[..., h, :] = o[..., h, :] @ w[h]",
                                     "out[..., h, :] = o[..., h, :] @ w[h][::-1]"),
-    "gqa_key_group_of_head": ("grp = np.arange(H) // ng", "grp = np.arange(H) % wl.groups"),
-    "gqa_value_group_shifted": ("v[:, grp, :])", "v[:, (grp + 1) % wl.groups, :])"),
+    "gqa_key_group_of_head": ("qh[:, g * ng:(g + 1) * ng], k[:, g, :])", "qh[:, g * ng:(g + 1) * ng], k[:, (g + 1) % wl.groups, :])"),
+    "gqa_value_group_shifted": ("v[:, g, :])", "v[:, (g + 1) % wl.groups, :])"),
     "gqa_key_gamma_dropped": ("rms_norm(c @ wk[g], np.asarray(gamma_k[g], np.float64), eps)",
                               "rms_norm(c @ wk[g], 1.0, eps)"),
     "gqa_key_unnormalised": ("rms_norm(c @ wk[g], np.asarray(gamma_k[g], np.float64), eps)",
                              "(c @ wk[g]) * np.asarray(gamma_k[g], np.float64)"),
     "gqa_values_from_keys_weight": ("np.stack([c @ wv[g] for g in range(wv.shape[0])], axis=1)",
                                     "np.stack([c @ wv[g][::-1] for g in range(wv.shape[0])], axis=1)"),
-    "gqa_rope_dropped": ('k[:, grp, :]) + np.einsum("jhd,td->jht", qrh, krh)', "k[:, grp, :])"),
+    "gqa_rope_dropped": ('logits = logits + np.einsum("jhd,td->jht", qrh, krh)', "pass"),
     "gqa_causal_off_by_one": ("visible = np.arange(L)[None, :] <= qpos[:, None]",
                               "visible = np.arange(L)[None, :] < qpos[:, None]"),
     "gqa_selection_of_group_zero": ("idx = np.asarray(selection[j, g])", "idx = np.asarray(selection[j, 0])"),
