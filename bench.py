@@ -58,6 +58,9 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--soak-seconds", type=float, default=1.0, help="load window around the timed steps for clocks")
     p.add_argument("--overhead-rounds", type=int, default=5)
+    p.add_argument("--route", choices=["absorbed", "gqa"], default="absorbed",
+                   help="decode route: the absorbed latent decode, or GQLA's GQA route over keys and values "
+                        "expanded per group (workloads with one key and one value head per group)")
     p.add_argument("--cp-emulate", type=int, default=0,
                    help="also time a context-parallel decode over this many ranks, emulated on one GPU "
                         "(every rank's slice decode and the merge of the partials; one GPU only)")
@@ -617,6 +620,214 @@ def run_ours(args, world, rank, local):
     return line
 
 
+def run_gqa(args, world, rank, local):
+    """GQLA's GQA route: per step, the step's new tokens expanded into the per-group cache
+    (qkn_gqa_append) and the dense decode (qkn_gqa_decode: split-KV kernel, then the merge)."""
+    import torch
+    import qk_normed_latent_qkn_b200 as qkn
+    from qk_normed_latent_qkn_b200.roofline import gqa_step_cost
+    from qk_normed_latent_qkn_b200.session import GqaSession, gqa_session_from_inputs
+    from qkn_inputs import make_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = rank_workload(args.workload, rank)
+    if not wl.tied_groups or wl.dtype != "bf16":
+        raise SystemExit("--route gqa needs a bf16 workload with one key and one value head per group")
+    inp = make_inputs(wl)
+    B, s_q, H = wl.batch, wl.s_q, wl.heads
+    last = np.concatenate([np.arange(inp.tok_off[b + 1] - s_q, inp.tok_off[b + 1]) for b in range(B)])
+    host = {"c": inp.c[last], "kr": inp.k_rope[last], "slot": inp.token_slots()[last],
+            "pos": inp.token_positions()[last], "q": inp.q, "qr": inp.q_rope, "bt": inp.block_table,
+            "sl": inp.seq_lens}
+    types = {"c": torch.bfloat16, "kr": torch.bfloat16, "slot": torch.int32, "pos": torch.int32,
+             "q": torch.bfloat16, "qr": torch.bfloat16, "bt": torch.int32, "sl": torch.int32}
+
+    base = gqa_session_from_inputs(inp, device=device)
+    cache_bytes = sum(t.numel() * t.element_size() for t in (base.cache.k, base.cache.v, base.cache.k_rope))
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    n_copies = max(1, min(16, math.ceil(3 * l2 / cache_bytes))) if cache_bytes < 2 * l2 else 1
+    sessions = [base]
+    for _ in range(n_copies - 1):
+        s = GqaSession(base.dims, inp.num_blocks, wl.d_v, device=device)
+        for dst, src in ((s.cache.k, base.cache.k), (s.cache.v, base.cache.v), (s.cache.k_rope, base.cache.k_rope)):
+            dst.copy_(src)
+        s.load_weights(base.w_uk, base.gamma_k, base.w_uv.clone(), base.gamma_q, base.gamma_qr, base.gamma_kr)
+        sessions.append(s)
+    dev_in = [{k: torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=types[k]) for k, v in
+               host.items()} for _ in sessions]
+    outs = [(torch.empty((B, s_q, H, wl.d_v), dtype=torch.bfloat16, device=device),
+             torch.empty((B, s_q, H), dtype=torch.float32, device=device)) for _ in sessions]
+    wss = [s.ensure_workspace(B, s_q) for s in sessions]
+    ev = Events()
+    stream = torch.cuda.Stream(device=device)
+
+    def append(i):
+        s, d = sessions[i], dev_in[i]
+        qkn.gqa_append(s.dims, s.cache, d["c"], d["kr"], d["slot"], d["pos"], s.w_uk, s.gamma_k, s.w_uv, s.gamma_kr)
+
+    def decode(i):
+        s, d, (o, l) = sessions[i], dev_in[i], outs[i]
+        qkn.gqa_decode(s.dims, s.cache, d["q"], d["qr"], s.gamma_q, s.gamma_qr, d["bt"], d["sl"], s_q, wss[i], o, l)
+
+    for i in range(n_copies):
+        append(i)
+        decode(i)
+    torch.cuda.synchronize(device)
+    assert all(s.device_status() == qkn.OK for s in sessions)
+
+    total = args.warmup + args.steps
+    graphs, op_graphs, bd_graphs = [], [], []
+    with torch.cuda.stream(stream):
+        for k in range(total):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                append(k % n_copies)
+                decode(k % n_copies)
+            graphs.append(g)
+        for i in range(n_copies):
+            e = [ev.create() for _ in range(2)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                ev.record(e[0], stream.cuda_stream)
+                decode(i)
+                ev.record(e[1], stream.cuda_stream)
+            op_graphs.append((g, e))
+            e = [ev.create() for _ in range(3)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+                ev.record(e[0], stream.cuda_stream)
+                append(i)
+                ev.record(e[1], stream.cuda_stream)
+                decode(i)
+                ev.record(e[2], stream.cuda_stream)
+            bd_graphs.append((g, e))
+    torch.cuda.synchronize(device)
+
+    def soak(seconds):
+        t_end = time.perf_counter() + seconds
+        with torch.cuda.stream(stream):
+            while time.perf_counter() < t_end:
+                for g in graphs[:n_copies]:
+                    g.replay()
+                stream.synchronize()
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    w0 = time.perf_counter()
+    with sampler:
+        soak(args.soak_seconds)
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup):
+                graphs[k].replay()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for k in range(args.warmup, total):
+                graphs[k].replay()
+            t1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        soak(args.soak_seconds)
+    window = time.perf_counter() - w0
+    value, step_ms = job_throughput(B * s_q, world, t0.elapsed_time(t1), args.steps, device)
+
+    op_ms, app_ms, dec_ms = [], [], []
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.overhead_rounds)):
+            for g, e in op_graphs:
+                g.replay()
+                stream.synchronize()
+                op_ms.append(ev.ms(e[0], e[1]))
+            for g, e in bd_graphs:
+                g.replay()
+                stream.synchronize()
+                app_ms.append(ev.ms(e[0], e[1]))
+                dec_ms.append(ev.ms(e[1], e[2]))
+
+    # end to end through the public API from pinned host buffers: copy-in, append, decode, copy-out of
+    # o_v and lse, synchronize, every step
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(types[k]).pin_memory() for k, v in host.items()}
+    o_host = torch.empty(outs[0][0].shape, dtype=torch.bfloat16).pin_memory()
+    l_host = torch.empty(outs[0][1].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = o_host.numel() * 2 + l_host.numel() * 4
+
+    def e2e_step(k):
+        i = k % n_copies
+        for key, t in pinned.items():
+            dev_in[i][key].copy_(t, non_blocking=True)
+        append(i)
+        decode(i)
+        o_host.copy_(outs[i][0], non_blocking=True)
+        l_host.copy_(outs[i][1], non_blocking=True)
+        torch.cuda.synchronize(device)
+
+    for k in range(args.warmup):
+        e2e_step(k)
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(args.steps):
+        e2e_step(k)
+    e1.record()
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device) / args.steps
+    assert all(s.device_status() == qkn.OK for s in sessions)
+
+    cost = gqa_step_cost(inp.seq_lens, s_q, H, wl.groups, wl.d_h, wl.d_rope, wl.d_v)
+    peaks, peak_src = load_peaks()
+    t_op = statistics.mean(op_ms)
+    achieved = cost.bytes / (t_op * 1e-3) / 1e9
+    tflops = cost.flops / (t_op * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        wts = inp.group_weights()
+        done, c0 = 0, time.perf_counter()
+        for b in range(B):
+            oracle.gqa_decode_sequence(inp, b, *wts)
+            done += 1
+            if time.perf_counter() - c0 >= args.cpu_seconds:
+                break
+        el = time.perf_counter() - c0
+        cpu = {"value": done * s_q / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{done} of {B} sequences of the workload ({done * s_q} query tokens, "
+                         f"{int(inp.seq_lens[:done].sum())} cached tokens) in {el:.1f} s, fp64 numpy, GQA route"}
+    tokens = world * B * s_q
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(wl, inp, world), route="gqa", d_v=wl.d_v,
+                       l2=f"{n_copies} rotating cache copies, {n_copies * cache_bytes / 2**20:.0f} MiB "
+                          f"(L2 {l2 / 2**20:.0f} MiB)", step_launch="CUDA graph per step"),
+        "breakdown_us": {"gqa_append": statistics.median(app_ms) * 1e3,
+                         "gqa_decode_op": statistics.median(dec_ms) * 1e3,
+                         "what": "expansion of the step's new tokens / split-KV decode + merge, from separate "
+                                 "graphs with an event between the stages"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "intensity_flop_per_byte": cost.flops / cost.bytes,
+                     "algorithmic_bytes": cost.bytes, "peak_source": f"{peak_src} HBM copy bandwidth",
+                     "kernel": ("GQA decode op (split-KV kernel + merge of its partials): mean duration over "
+                                "%d replays of decode-only graphs, CUDA events on the launching stream" % len(op_ms)),
+                     "duration_us": t_op * 1e3,
+                     "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": tflops / peaks["bf16_tflops"], "flops": cost.flops}},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "per step: copy-in from pinned host buffers, qkn_gqa_append, qkn_gqa_decode, copy-out of "
+                        "o_v and lse to pinned host buffers, synchronize"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": sampler.summary(window),
+        "cpu_baseline": cpu,
+    }
+
+
 def schedule_shape(kernel_used: int, head_tile: int, s_q: int, heads: int, sms: int):
     """Row tile, schedule CTAs and item cost of the decode's split schedule for this launch (the C-ABI
     layer's choice restated for cost accounting; 128-row tiles on CTA pairs count sms / 2 pairs)."""
@@ -719,7 +930,10 @@ def run_reference(args, world, rank):
     for k in range(args.warmup + args.steps):
         b = k % wl.batch
         t0 = time.perf_counter()
-        oracle.decode_sequence(inp, b)
+        if args.route == "gqa":
+            oracle.gqa_decode_sequence(inp, b, *inp.group_weights())
+        else:
+            oracle.decode_sequence(inp, b)
         if k >= args.warmup:
             times.append(time.perf_counter() - t0)
     per_tok = statistics.mean(times) / wl.s_q
@@ -728,7 +942,8 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(workload_config(wl, inp, world), sample="one whole sequence per step"),
+        "config": dict(workload_config(wl, inp, world), sample="one whole sequence per step",
+                       **({"route": "gqa", "d_v": wl.d_v} if args.route == "gqa" else {})),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"one sequence of {wl.name} per step (explicit keys, fp64 numpy)"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -753,7 +968,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
-        line = run_ours(args, world, rank, local)
+        line = (run_gqa if args.route == "gqa" else run_ours)(args, world, rank, local)
     finally:
         if world > 1:
             dist.destroy_process_group()

@@ -353,6 +353,98 @@ QKN_EXPORT qkn_status qkn_decode_noalloc(const qkn_dims* dims, const qkn_cache* 
 QKN_EXPORT qkn_status qkn_merge_partials(const qkn_dims* dims, int32_t n_parts, int64_t rows, const void* parts,
                       const float* lse_parts, void* out, float* lse, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * The GQA route of GQLA ("GQLA", section 2, "Ruta GQA") and its sparse form
+ * ("GQLA Disperso").  Under GQLA's parameterisation the up-projections are
+ * indexed by KV group: one key head W^UK_g [r_kv, d_h] with its norm weight
+ * gamma_k[g] and one value head W^UV_g [r_kv, d_v] per group, shared by the
+ * group's n_g = num_heads / num_groups query heads.  This route caches the
+ * latent expanded into per-group keys and values (2 g d_h values per token)
+ * plus the shared RoPE key, and decodes with ordinary grouped-query
+ * attention over them.  Over the same weights it is algebraically equal to
+ * the absorbed route (qkn_decode_up with W^UV_h = W^UV_{g(h)}, and W^K_g made
+ * of n_g copies of W^UK_g): it trades cache bytes for FLOPs per byte.
+ * bf16 storage only; (d_h, d_rope, d_v) = (128, 64, 128) or (64, 32, 64).
+ * ------------------------------------------------------------------------- */
+
+/* The GQA route's cache, caller-allocated device memory, bf16, 16-byte aligned:
+ *   k      [num_blocks, num_groups, block_size, d_h]   normalised keys
+ *   v      [num_blocks, num_groups, block_size, d_v]   values
+ *   k_rope [num_blocks, block_size, d_rope]            as qkn_cache.k_rope
+ * Slot s of the pool is token s % block_size of block s / block_size.  Slots
+ * that no qkn_gqa_append has written may hold anything; the decode reads no
+ * slot past a sequence's length. */
+typedef struct {
+  void* k;
+  void* v;
+  void* k_rope;
+  int32_t num_blocks;
+  int32_t d_v;
+} qkn_gqa_cache;
+
+/* qkn_gqa_append — expand n_tok new tokens into the GQA route's cache.
+ * For token i with slot s = slot[i], position p = pos[i] and every group g:
+ *   k[s, g] = gamma_k[g] * z / S(z),  z = c_new[i] W^UK_g   (S over the d_h columns)
+ *   v[s, g] = c_new[i] W^UV_g
+ *   k_rope[s] = RoPE_p(gamma_kr * k_rope_raw[i] / S(k_rope_raw[i]))
+ * (GQLA summary, section 2, "Ruta GQA": the latent expanded into g groups of
+ * keys and values; the key RMS-normalised after its up-projection as in the
+ * QK-Normed summary, "Planteamiento del Problema").  fp32 products.
+ *   c_new      [n_tok, r_kv] bf16, 16-byte aligned;  k_rope_raw [n_tok, d_rope] bf16, 16-byte aligned
+ *   slot, pos  [n_tok] int32 device arrays; a token whose slot is outside
+ *              [0, num_blocks * block_size) is skipped
+ *   w_uk       [num_groups, r_kv, d_h] fp32, 16-byte aligned;  gamma_k [num_groups, d_h] fp32
+ *   w_uv       [num_groups, r_kv, d_v] bf16, 16-byte aligned;  gamma_kr [d_rope] fp32
+ * n_tok == 0 is a no-op.  Returns QKN_ERR_UNSUPPORTED for fp32 storage,
+ * other head widths, r_kv not a multiple of 32 or more than 65535 groups,
+ * QKN_ERR_INVALID_ARG for bad dims or a missing or misaligned pointer. */
+QKN_EXPORT qkn_status qkn_gqa_append(const qkn_dims* dims, const qkn_gqa_cache* cache, const void* c_new,
+                      const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                      const float* w_uk, const float* gamma_k, const void* w_uv, const float* gamma_kr,
+                      void* stream);
+
+/* Bytes of device workspace qkn_gqa_decode needs for `batch` sequences of
+ * s_q query tokens on a GPU of num_sms SMs (0 = the current device's).  The
+ * sparse form needs only its first 256 bytes (the status word).  Initialise
+ * it with qkn_workspace_init. */
+QKN_EXPORT qkn_status qkn_gqa_workspace_size(const qkn_dims* dims, int32_t d_v, int32_t batch, int32_t s_q,
+                      int32_t num_sms, size_t* bytes);
+
+/* qkn_gqa_decode — one decode step of the GQA route.  Query row (j, h) of
+ * sequence b, head h in group g = h / n_g, sits at position L_b - s_q + j and
+ * gets
+ *   l[t] = sigma (RMSNorm(q_jh) gamma_q[h] . k[t, g]
+ *                 + RoPE_pos(RMSNorm(q^R_jh) gamma_qr[h]) . k_rope[t]),
+ *   o_v[b, j, h] = sum_t softmax(l)[t] v[t, g],  lse[b, j, h] = log sum_t exp(l[t]),
+ * over the tokens t <= L_b - s_q + j of the sequence (dense), or, with a
+ * selection, over the tokens selection[b, j, g, :] lists among them (sparse
+ * GQLA: the n_g heads of a group share the query token's list).  sigma is
+ * dims->softmax_scale (0 = 1/sqrt(d_h + d_rope)); the queries are normalised
+ * and rotated inside the call.
+ *   q          [batch, s_q, num_heads, d_h] bf16 (raw queries)
+ *   q_rope     [batch, s_q, num_heads, d_rope] bf16 (raw)
+ *   gamma_q    [num_heads, d_h] fp32;  gamma_qr [num_heads, d_rope] fp32
+ *   block_table [batch, max_blocks] int32, seq_lens [batch] int32 (device)
+ *   selection  NULL (dense) or [batch, s_q, num_groups, sel_k] int32 token
+ *              positions, -1 for none; a listed position after the query's
+ *              is not attended; the positions of one list should be distinct
+ *   out_v      [batch, s_q, num_heads, d_v] bf16, 16-byte aligned;  lse [batch, s_q, num_heads] fp32
+ *   max_ctas   cap on the dense decode's CTAs (0 = one per SM)
+ * Dense: a split-KV decode on a device schedule, then the merge of the
+ * splits, on `stream`.  Sparse: one CTA per (sequence, query token, group).
+ * A sequence whose length is below s_q or past its block table, and a block
+ * id outside the pool, are recorded in the workspace status word
+ * (QKN_ERR_BOUNDS); the former's rows come out as zeros with lse = -inf, the
+ * latter reads block 0 instead.  A row with no token (an empty selection)
+ * gets zeros and lse = -inf.  Returns QKN_ERR_UNSUPPORTED for fp32 storage or
+ * other head widths, QKN_ERR_INVALID_ARG for bad arguments or a workspace
+ * smaller than qkn_gqa_workspace_size says; batch == 0 is a no-op. */
+QKN_EXPORT qkn_status qkn_gqa_decode(const qkn_dims* dims, const qkn_gqa_cache* cache, const void* q,
+                      const void* q_rope, const float* gamma_q, const float* gamma_qr,
+                      const int32_t* block_table, int32_t max_blocks, const int32_t* seq_lens, int32_t batch,
+                      int32_t s_q, const int32_t* selection, int32_t sel_k, void* workspace, size_t ws_bytes,
+                      void* out_v, float* lse, int32_t max_ctas, void* stream);
+
 /* Synchronise `stream`, then read the workspace status word into *device_status
  * (a qkn_status value; QKN_OK if no kernel recorded an error).  The word is
  * sticky until qkn_workspace_init clears it. */

@@ -27,7 +27,7 @@ KERNEL_AUTO, KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1, 2
 EXPORTED = ["qkn_append", "qkn_absorb_query", "qkn_decode_workspace_size", "qkn_workspace_init",
             "qkn_decode", "qkn_read_device_status", "qkn_decode_kernel_for", "qkn_status_string",
             "qkn_version", "qkn_decode_noalloc", "qkn_append_absorb", "qkn_key_gram", "qkn_decode_up",
-            "qkn_merge_partials"]
+            "qkn_merge_partials", "qkn_gqa_append", "qkn_gqa_workspace_size", "qkn_gqa_decode"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -49,6 +49,11 @@ class _Cache(ctypes.Structure):
                 ("num_blocks", ctypes.c_int32), ("ak_scratch", ctypes.c_void_p)]
 
 
+class _GqaCache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("k_rope", ctypes.c_void_p),
+                ("num_blocks", ctypes.c_int32), ("d_v", ctypes.c_int32)]
+
+
 class _Opts(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("max_ctas", ctypes.c_int32), ("head_tile", ctypes.c_int32),
                 ("wait_limit", ctypes.c_int64), ("split_event", ctypes.c_void_p),
@@ -62,6 +67,7 @@ def _load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     PD, PC, PO = ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), ctypes.POINTER(_Opts)
+    PG = ctypes.POINTER(_GqaCache)
     sig = {
         "qkn_append": (I32, [PD, PC, P, P, P, P, I32, P, P, P, P]),
         "qkn_key_gram": (I32, [PD, P, P, P]),
@@ -77,6 +83,9 @@ def _load() -> ctypes.CDLL:
         "qkn_version": (I32, []),
         "qkn_decode_noalloc": (I32, [PD, PC, I32, P, P, P, P, I32, P, I32, I32, P, P, P, PO, P]),
         "qkn_append_absorb": (I32, [PD, PC, P, P, P, P, I32, P, P, P, I32, P, P, P, P, P, P, P, P, P, P]),
+        "qkn_gqa_append": (I32, [PD, PG, P, P, P, P, I32, P, P, P, P, P]),
+        "qkn_gqa_workspace_size": (I32, [PD, I32, I32, I32, I32, ctypes.POINTER(SZ)]),
+        "qkn_gqa_decode": (I32, [PD, PG, P, P, P, P, P, I32, P, I32, I32, P, I32, P, SZ, P, P, I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -140,6 +149,22 @@ class Cache:
     def c(self) -> _Cache:
         return _Cache(self.latent.data_ptr(), self.k_rope.data_ptr(), self.a_k.data_ptr(), self.num_blocks,
                       None if self.ak_scratch is None else self.ak_scratch.data_ptr())
+
+
+class GqaCache:
+    """The GQA route's paged cache: per-group normalised keys and values, and the shared RoPE key."""
+
+    def __init__(self, dims: Dims, num_blocks: int, d_v: int, device="cuda"):
+        bs = dims.block_size
+        self.dims = dims
+        self.num_blocks = num_blocks
+        self.d_v = d_v
+        self.k = torch.empty((num_blocks, dims.num_groups, bs, dims.d_h), dtype=dims.torch_dtype, device=device)
+        self.v = torch.empty((num_blocks, dims.num_groups, bs, d_v), dtype=dims.torch_dtype, device=device)
+        self.k_rope = torch.empty((num_blocks, bs, dims.d_rope), dtype=dims.torch_dtype, device=device)
+
+    def c(self) -> _GqaCache:
+        return _GqaCache(self.k.data_ptr(), self.v.data_ptr(), self.k_rope.data_ptr(), self.num_blocks, self.d_v)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -263,6 +288,35 @@ def merge_partials(dims: Dims, parts, lse_parts, out, lse, stream=None) -> None:
     rows = int(lse_parts[0].numel())
     _check(_lib.qkn_merge_partials(ctypes.byref(dims.c()), n_parts, rows, _ptr(parts), _ptr(lse_parts), _ptr(out),
                                    _ptr(lse), _stream(stream)), "qkn_merge_partials")
+
+
+def gqa_append(dims: Dims, cache: GqaCache, c_new, k_rope_raw, slot, pos, w_uk, gamma_k, w_uv, gamma_kr,
+               stream=None) -> None:
+    """qkn_gqa_append: expand tokens into the GQA route's cache (per-group keys and values, RoPE key)."""
+    n_tok = int(c_new.shape[0])
+    _check(_lib.qkn_gqa_append(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(c_new), _ptr(k_rope_raw),
+                               _ptr(slot), _ptr(pos), n_tok, _ptr(w_uk), _ptr(gamma_k), _ptr(w_uv), _ptr(gamma_kr),
+                               _stream(stream)), "qkn_gqa_append")
+
+
+def gqa_workspace_size(dims: Dims, d_v: int, batch: int, s_q: int, num_sms: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.qkn_gqa_workspace_size(ctypes.byref(dims.c()), d_v, batch, s_q, num_sms, ctypes.byref(out)),
+           "qkn_gqa_workspace_size")
+    return int(out.value)
+
+
+def gqa_decode(dims: Dims, cache: GqaCache, q, q_rope, gamma_q, gamma_qr, block_table, seq_lens, s_q: int,
+               workspace, out_v, lse, selection=None, max_ctas: int = 0, stream=None) -> None:
+    """qkn_gqa_decode: grouped-query attention over the GQA route's cache (dense), or over each query token's
+    listed tokens per group (``selection`` [batch, s_q, groups, k] int32, sparse)."""
+    batch = int(block_table.shape[0])
+    max_blocks = int(block_table.shape[1])
+    sel_k = 0 if selection is None else int(selection.shape[-1])
+    _check(_lib.qkn_gqa_decode(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(q), _ptr(q_rope), _ptr(gamma_q),
+                               _ptr(gamma_qr), _ptr(block_table), max_blocks, _ptr(seq_lens), batch, s_q,
+                               _ptr(selection), sel_k, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _ptr(out_v), _ptr(lse), max_ctas, _stream(stream)), "qkn_gqa_decode")
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:

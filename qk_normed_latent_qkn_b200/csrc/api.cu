@@ -484,3 +484,194 @@ qkn_status qkn_read_device_status(const void* workspace, void* stream, int32_t* 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- the GQA route
+
+namespace {
+
+qkn_status check_gqa_cache(const qkn_gqa_cache* c) {
+  if (!c || !c->k || !c->v || !c->k_rope || c->num_blocks <= 0 || c->d_v <= 0) return QKN_ERR_INVALID_ARG;
+  if (!aligned(c->k, 16) || !aligned(c->v, 16) || !aligned(c->k_rope, 16)) return QKN_ERR_INVALID_ARG;
+  if ((int64_t)c->num_blocks * kBlockSize > INT32_MAX) return QKN_ERR_INVALID_ARG;
+  return QKN_OK;
+}
+
+// Query rows per tile and tiles per group: a dense tile holds the group's rows of every query token
+// of the step (s_q n_g of them), a sparse one those of one query token (n_g), in tiles of 16 or 32.
+void gqa_tiling(const qkn_dims* d, int s_q, bool sparse, int* rows, int* tpg) {
+  const int ng = d->num_heads / d->num_groups;
+  const int span = sparse ? ng : s_q * ng;
+  *rows = span <= 16 ? 16 : 32;
+  *tpg = ceil_div(span, *rows);
+}
+
+// Dense decode CTAs: one per SM (capped), whole groups of the schedule's row tiles where they fit.
+int gqa_ncta(int nsm, int ht, int max_ctas) {
+  int n = nsm;
+  if (max_ctas > 0 && max_ctas < n) n = max_ctas;
+  if (n >= ht) n = n / ht * ht;
+  return n;
+}
+
+struct GqaWs {
+  size_t lse_off, o_off, total;   // status word | split lse | split outputs
+};
+
+GqaWs gqa_ws_layout(const qkn_dims* d, int d_v, int batch, int s_q, int nsm) {
+  int rows = 0, tpg = 0;
+  gqa_tiling(d, s_q, false, &rows, &tpg);
+  const int64_t ht = (int64_t)d->num_groups * tpg;
+  // any CTA cap gives at most nsm CTAs, so nsm bounds the slots
+  const int64_t slot_rows = sched_slots(batch, ht, nsm) * rows;
+  GqaWs w;
+  w.lse_off = kStatusBytes;
+  w.o_off = w.lse_off + ((size_t)slot_rows * 4 + 255) / 256 * 256;
+  w.total = w.o_off + (size_t)slot_rows * d_v * 4;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+qkn_status qkn_gqa_append(const qkn_dims* dims, const qkn_gqa_cache* cache, const void* c_new,
+                          const void* k_rope_raw, const int32_t* slot, const int32_t* pos, int32_t n_tok,
+                          const float* w_uk, const float* gamma_k, const void* w_uv, const float* gamma_kr,
+                          void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (n_tok < 0) return QKN_ERR_INVALID_ARG;
+  if ((st = check_gqa_cache(cache)) != QKN_OK) return st;
+  if (dims->dtype != QKN_BF16 || !gqa_supported(dims->d_h, dims->d_rope, cache->d_v)) return QKN_ERR_UNSUPPORTED;
+  // the expansion stages the latent 32 columns at a time; one grid row per group
+  if (dims->r_kv % 32 || dims->num_groups > 65535) return QKN_ERR_UNSUPPORTED;
+  if (n_tok == 0) return QKN_OK;
+  if (!c_new || !k_rope_raw || !slot || !pos || !w_uk || !gamma_k || !w_uv || !gamma_kr) return QKN_ERR_INVALID_ARG;
+  if (!aligned(c_new, 16) || !aligned(k_rope_raw, 16) || !aligned(w_uk, 16) || !aligned(w_uv, 16) ||
+      !aligned(gamma_k, 4) || !aligned(gamma_kr, 4))
+    return QKN_ERR_INVALID_ARG;
+  GqaAppendArgs a;
+  a.k_cache = cache->k;
+  a.v_cache = cache->v;
+  a.k_rope = cache->k_rope;
+  a.c_new = c_new;
+  a.k_rope_raw = k_rope_raw;
+  a.slot = slot;
+  a.pos = pos;
+  a.w_uk = w_uk;
+  a.gamma_k = gamma_k;
+  a.w_uv = w_uv;
+  a.gamma_kr = gamma_kr;
+  a.n_tok = n_tok;
+  a.r = dims->r_kv;
+  a.d_h = dims->d_h;
+  a.d_v = cache->d_v;
+  a.d_rope = dims->d_rope;
+  a.groups = dims->num_groups;
+  a.n_slots = (int64_t)cache->num_blocks * kBlockSize;
+  a.eps = dims->eps;
+  a.freq = rope_freqs(dims);
+  cudaError_t e = launch_gqa_append(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+qkn_status qkn_gqa_workspace_size(const qkn_dims* dims, int32_t d_v, int32_t batch, int32_t s_q, int32_t num_sms,
+                                  size_t* bytes) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if (!bytes || d_v <= 0 || batch < 0 || s_q < 1 || num_sms < 0) return QKN_ERR_INVALID_ARG;
+  int n = num_sms;
+  if (n == 0 && sm_count(&n) != 0) return QKN_ERR_CUDA;
+  *bytes = gqa_ws_layout(dims, d_v, batch, s_q, n).total;
+  return QKN_OK;
+}
+
+qkn_status qkn_gqa_decode(const qkn_dims* dims, const qkn_gqa_cache* cache, const void* q, const void* q_rope,
+                          const float* gamma_q, const float* gamma_qr, const int32_t* block_table,
+                          int32_t max_blocks, const int32_t* seq_lens, int32_t batch, int32_t s_q,
+                          const int32_t* selection, int32_t sel_k, void* workspace, size_t ws_bytes, void* out_v,
+                          float* lse, int32_t max_ctas, void* stream) {
+  qkn_status st = check_dims(dims);
+  if (st != QKN_OK) return st;
+  if ((st = check_gqa_cache(cache)) != QKN_OK) return st;
+  if (dims->dtype != QKN_BF16 || !gqa_supported(dims->d_h, dims->d_rope, cache->d_v)) return QKN_ERR_UNSUPPORTED;
+  if (batch < 0 || s_q < 1 || max_blocks < 1 || max_ctas < 0 || (selection && sel_k < 1)) return QKN_ERR_INVALID_ARG;
+  if (batch == 0) return QKN_OK;
+  if (!q || !q_rope || !gamma_q || !gamma_qr || !block_table || !seq_lens || !workspace || !out_v || !lse)
+    return QKN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(q_rope, 16) || !aligned(out_v, 16) || !aligned(workspace, 256) ||
+      !aligned(gamma_q, 4) || !aligned(gamma_qr, 4))
+    return QKN_ERR_INVALID_ARG;
+  int nsm = 0;
+  if (sm_count(&nsm) != 0) return QKN_ERR_CUDA;
+  const bool sparse = selection != nullptr;
+  const GqaWs w = gqa_ws_layout(dims, cache->d_v, batch, s_q, nsm);
+  if (ws_bytes < (sparse ? (size_t)kStatusBytes : w.total)) return QKN_ERR_INVALID_ARG;
+
+  char* ws = static_cast<char*>(workspace);
+  GqaDecodeArgs a;
+  a.k_cache = cache->k;
+  a.v_cache = cache->v;
+  a.k_rope = cache->k_rope;
+  a.num_blocks = cache->num_blocks;
+  a.q = q;
+  a.q_rope = q_rope;
+  a.gamma_q = gamma_q;
+  a.gamma_qr = gamma_qr;
+  a.block_table = block_table;
+  a.max_blocks = max_blocks;
+  a.seq_lens = seq_lens;
+  a.batch = batch;
+  a.s_q = s_q;
+  a.heads = dims->num_heads;
+  a.groups = dims->num_groups;
+  a.d_h = dims->d_h;
+  a.d_rope = dims->d_rope;
+  a.d_v = cache->d_v;
+  gqa_tiling(dims, s_q, sparse, &a.rows, &a.tpg);
+  a.ht_count = dims->num_groups * a.tpg;
+  a.ncta = gqa_ncta(nsm, a.ht_count, max_ctas);
+  // starting an item (the tile's queries, the ring's first pages) costs about two pages of time
+  a.item_cost = 2;
+  a.selection = selection;
+  a.sel_k = sparse ? sel_k : 0;
+  a.part_o = reinterpret_cast<float*>(ws + w.o_off);
+  a.part_lse = reinterpret_cast<float*>(ws + w.lse_off);
+  a.out = out_v;
+  a.lse = lse;
+  a.status = reinterpret_cast<int32_t*>(ws);
+  a.eps = dims->eps;
+  a.score_scale = softmax_scale_of(dims) * 1.4426950408889634f;   // sigma * log2(e)
+  a.freq = rope_freqs(dims);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_gqa_decode(a, cs);
+  if (e == cudaErrorNotSupported) return QKN_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return QKN_ERR_CUDA;
+  if (sparse) return QKN_OK;
+
+  CombineArgs c;
+  c.seq_lens = seq_lens;
+  c.batch = batch;
+  c.s_q = s_q;
+  c.heads = dims->num_heads;
+  c.r = cache->d_v;
+  c.rows = a.rows;
+  c.ht_count = a.ht_count;
+  c.ncta = a.ncta;
+  c.item_cost = a.item_cost;
+  c.max_blocks = max_blocks;
+  c.max_items = a.ncta + 1;
+  c.nslots = sched_slots(batch, a.ht_count, a.ncta);
+  c.part_o = a.part_o;
+  c.part_lse = a.part_lse;
+  c.out = out_v;
+  c.lse = lse;
+  c.status = a.status;
+  c.seg_desc = nullptr;
+  c.group_heads = dims->num_heads / dims->num_groups;
+  c.tiles_per_group = a.tpg;
+  e = launch_combine_grouped(c, cs);
+  return e == cudaSuccess ? QKN_OK : QKN_ERR_CUDA;
+}
+
+}  // extern "C"

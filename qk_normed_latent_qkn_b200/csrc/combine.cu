@@ -37,7 +37,10 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4
 // per CTA; every thread owns the same 16 bytes of each of them, and the rows' loads are issued
 // together, so that a CTA keeps RPC times as many loads in flight and the grid fits in fewer waves.
 // The RPC rows of a CTA lie in one segment (RPC divides the tile's row count).
-template <typename T, bool kDesc, int RPC>
+// kGroup: the GQA route's row tiles, each holding one KV group's query rows (CombineArgs.group_heads);
+// the RPC rows of a CTA then belong to one query token (RPC divides n_g), so that they are
+// consecutive rows of the output as well.
+template <typename T, bool kDesc, int RPC, bool kGroup = false>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   __shared__ int64_t first_s;
   __shared__ int nitems_s;
@@ -47,9 +50,20 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   const int seg = grow0 / a.rows, row0 = grow0 - seg * a.rows;
   const int b = seg / a.ht_count, ht = seg - b * a.ht_count;
   const int qrows = a.s_q * a.heads;
-  const int rho0 = ht * a.rows + row0;
-  if (b >= a.batch || rho0 >= qrows) return;
-  const int nrows = min(RPC, qrows - rho0);               // rows of this CTA inside the sequence
+  int rho0, nrows;                                        // first query row, rows of this CTA
+  if constexpr (kGroup) {
+    const int g = ht / a.tiles_per_group, rb = ht - g * a.tiles_per_group;
+    const int u = rb * a.rows + row0;                     // u = j * n_g + m
+    const int span = a.s_q * a.group_heads;
+    if (b >= a.batch || u >= span) return;
+    const int j = u / a.group_heads, m = u - j * a.group_heads;
+    rho0 = j * a.heads + g * a.group_heads + m;
+    nrows = min(RPC, span - u);
+  } else {
+    rho0 = ht * a.rows + row0;
+    if (b >= a.batch || rho0 >= qrows) return;
+    nrows = min(RPC, qrows - rho0);                       // rows of this CTA inside the sequence
+  }
   const int64_t orow0 = (int64_t)b * qrows + rho0;
   const int nvec = a.r / 4;
   // the splits of the segment: from the descriptor the tcgen05 decode wrote, else from the
@@ -175,6 +189,15 @@ cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t st) {
                 : launch_chained(combine_kernel<float, true, 1>, grid, block, smem, st, a);
   return bf16 ? launch_chained(combine_kernel<__nv_bfloat16, false, 1>, grid, block, smem, st, a)
               : launch_chained(combine_kernel<float, false, 1>, grid, block, smem, st, a);
+}
+
+cudaError_t launch_combine_grouped(const CombineArgs& a, cudaStream_t st) {
+  // four rows per CTA when they never straddle two query tokens (n_g and the tile's rows multiples of 4)
+  const int64_t rows = (int64_t)a.batch * a.ht_count * a.rows;
+  const dim3 block(kCombThreads);
+  if (a.rows % 4 == 0 && a.group_heads % 4 == 0 && rows >= 4096)
+    return launch_chained(combine_kernel<__nv_bfloat16, false, 4, true>, dim3((unsigned)(rows / 4)), block, 0, st, a);
+  return launch_chained(combine_kernel<__nv_bfloat16, false, 1, true>, dim3((unsigned)rows), block, 0, st, a);
 }
 
 }  // namespace qkn

@@ -94,6 +94,11 @@ struct CombineArgs {
   float* lse;                // [batch, s_q, H]
   int32_t* status;           // workspace status word
   const int2* seg_desc;      // per-segment (first slot, splits) from the tcgen05 kernel, or null
+  // GQA route (gqa.cu) only; 0 elsewhere.  Row tiles hold one KV group's query rows: tile ht is
+  // row block ht % tiles_per_group of group ht / tiles_per_group, whose rows u = (j, m), u = j * n_g + m
+  // (query token j, head g * n_g + m) are laid out u = block * rows + row.
+  int32_t group_heads = 0;   // n_g
+  int32_t tiles_per_group = 0;
 };
 
 // Merge fused with the per-head value up-projection (combine_up.cu): c.out is not used; the merged
@@ -105,6 +110,62 @@ struct CombineUpArgs {
   void* out_v;               // [batch, s_q, H, d_v] in the storage type
   int32_t col_groups;        // output column groups per (head, row block); set by the launcher
 };
+
+// GQA route of GQLA (gqa.cu): keys and values expanded per KV group, one key head and one value
+// head per group.  bf16 storage.
+struct GqaAppendArgs {
+  void* k_cache;           // [num_blocks, groups, 64, d_h]   normalised keys
+  void* v_cache;           // [num_blocks, groups, 64, d_v]
+  void* k_rope;            // [num_blocks, 64, d_rope]        normalised, rotated RoPE keys
+  const void* c_new;       // [n_tok, r]
+  const void* k_rope_raw;  // [n_tok, d_rope]
+  const int32_t* slot;
+  const int32_t* pos;
+  const float* w_uk;       // [groups, r, d_h] fp32
+  const float* gamma_k;    // [groups, d_h]
+  const void* w_uv;        // [groups, r, d_v] storage type
+  const float* gamma_kr;   // [d_rope]
+  int32_t n_tok, r, d_h, d_v, d_rope, groups;
+  int64_t n_slots;         // a token whose slot is outside [0, n_slots) is skipped
+  float eps;
+  RopeFreqs freq;
+};
+
+struct GqaDecodeArgs {
+  const void* k_cache;       // as in GqaAppendArgs
+  const void* v_cache;
+  const void* k_rope;
+  int32_t num_blocks;
+  const void* q;             // [batch, s_q, H, d_h]     raw queries
+  const void* q_rope;        // [batch, s_q, H, d_rope]
+  const float* gamma_q;      // [H, d_h]
+  const float* gamma_qr;     // [H, d_rope]
+  const int32_t* block_table;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  int32_t batch, s_q, heads, groups;
+  int32_t d_h, d_rope, d_v;
+  int32_t rows;              // query rows per tile: 16 or 32
+  int32_t tpg;               // tiles per group (dense) or per (query token, group) (sparse)
+  int32_t ht_count;          // dense: tiles per sequence (groups * tpg)
+  int32_t ncta, item_cost;   // dense: the device schedule's CTAs and item start cost
+  const int32_t* selection;  // sparse: [batch, s_q, groups, sel_k] token positions (-1: none); null = dense
+  int32_t sel_k;
+  float* part_o;             // dense: [slots, rows, d_v] normalised partial outputs
+  float* part_lse;           // dense: [slots, rows]
+  void* out;                 // sparse: [batch, s_q, H, d_v]
+  float* lse;                // sparse: [batch, s_q, H]
+  int32_t* status;
+  float eps;
+  float score_scale;         // sigma * log2(e): logits in base-2 units
+  RopeFreqs freq;
+};
+
+bool gqa_supported(int d_h, int d_rope, int d_v);
+cudaError_t launch_gqa_append(const GqaAppendArgs& a, cudaStream_t st);
+cudaError_t launch_gqa_decode(const GqaDecodeArgs& a, cudaStream_t st);
+// The merge of the GQA route's split partials (combine.cu, grouped row tiles).
+cudaError_t launch_combine_grouped(const CombineArgs& a, cudaStream_t st);
 
 cudaError_t launch_append(const AppendArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_key_gram(const float* w_k, float* gram, int groups, int r, int width, cudaStream_t st);

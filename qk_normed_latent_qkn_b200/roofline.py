@@ -58,6 +58,33 @@ def decode_step_cost(seq_lens: Sequence[int], s_q: int, heads: int, groups: int,
     )
 
 
+# ----------------------------------------------------------------- the GQA route
+def gqa_bytes_per_token(groups: int, d_h: int, d_rope: int, d_v: int, elem: int = 2) -> int:
+    """Cache bytes per token of the GQA route: one key and one value head per group plus the shared
+    RoPE key ("GQLA", section 2, Ruta GQA: 2 g d_h values plus the RoPE key when d_v = d_h)."""
+    return elem * (groups * (d_h + d_v) + d_rope)
+
+
+def gqa_flops_per_token_row(d_h: int, d_rope: int, d_v: int) -> int:
+    """A query row's FLOPs on one visible token: its logit over d_h + d_R, its share of the values."""
+    return 2 * (d_h + d_rope) + 2 * d_v
+
+
+def gqa_step_cost(seq_lens: Sequence[int], s_q: int, heads: int, groups: int, d_h: int, d_rope: int, d_v: int,
+                  elem: int = 2) -> StepCost:
+    """Cost of one GQA-route decode step: the expanded cache read once, the raw queries read, o_v and lse
+    written; FLOPs over the causal (query token, key) pairs of every head."""
+    tokens = sum(int(L) for L in seq_lens)
+    pairs = sum(int(L) - s_q + j + 1 for L in seq_lens for j in range(s_q))
+    rows = len(seq_lens) * s_q * heads
+    return StepCost(
+        cache_bytes=tokens * gqa_bytes_per_token(groups, d_h, d_rope, d_v, elem),
+        query_bytes=rows * elem * (d_h + d_rope),
+        output_bytes=rows * (elem * d_v + 4),
+        flops=pairs * heads * gqa_flops_per_token_row(d_h, d_rope, d_v),
+    )
+
+
 # ----------------------------------------------------------------- the merge of the split-KV partials
 def split_counts(seq_lens: Sequence[int], s_q: int, max_blocks: int, ht_count: int, ncta: int,
                  item_cost: int, block: int = 64) -> list:

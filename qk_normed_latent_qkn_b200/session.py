@@ -1,5 +1,9 @@
 """Device-resident decode state on top of the C ABI.
 
+A ``GqaSession`` does the same for the GQA route (qkn_gqa_append,
+qkn_gqa_decode): the per-group expanded cache, the group weights, the raw
+queries and a workspace.
+
 A ``DecodeSession`` owns a paged cache, the key up-projection and norm
 weights, the value up-projection (optional), the absorbed queries and a
 decode workspace, and forwards to ``qkn_append``, ``qkn_absorb_query``,
@@ -13,8 +17,9 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, absorb_query, append, append_absorb, decode, decode_up,
-               key_gram, decode_workspace_size, read_device_status, workspace_init)
+from . import (AK_CACHE, KERNEL_AUTO, Cache, Dims, GqaCache, absorb_query, append, append_absorb, decode, decode_up,
+               gqa_append, gqa_decode, gqa_workspace_size, key_gram, decode_workspace_size, read_device_status,
+               workspace_init)
 
 
 def to_device(x, dtype: torch.dtype, device) -> torch.Tensor:
@@ -159,3 +164,87 @@ def session_from_inputs(inp, device="cuda", dtype=None) -> DecodeSession:
     s.absorb(inp.q.reshape(B * s_q, wl.heads, wl.d_h), inp.q_rope.reshape(B * s_q, wl.heads, wl.d_rope),
              inp.query_positions().reshape(-1))
     return s
+
+
+class GqaSession:
+    """Device state of the GQA route: per-group keys and values expanded from the latent, the group weights
+    W^UK_g, gamma_k[g], W^UV_g, the norm weights of the queries and RoPE key, the step's raw queries and a
+    workspace."""
+
+    def __init__(self, dims: Dims, num_blocks: int, d_v: int, device="cuda"):
+        self.dims = dims
+        self.device = torch.device(device)
+        self.cache = GqaCache(dims, num_blocks, d_v, device=self.device)
+        self.w_uk = self.gamma_k = self.w_uv = self.gamma_q = self.gamma_qr = self.gamma_kr = None
+        self.q = self.q_rope = None
+        self.workspace: Optional[torch.Tensor] = None
+
+    def load_weights(self, w_uk, gamma_k, w_uv, gamma_q, gamma_qr, gamma_kr) -> None:
+        """W^UK [g, r, d_h] and the gammas in fp32, W^UV [g, r, d_v] in the storage dtype."""
+        f32, dev = torch.float32, self.device
+        self.w_uk = to_device(w_uk, f32, dev)
+        self.gamma_k = to_device(gamma_k, f32, dev)
+        self.w_uv = to_device(w_uv, self.dims.torch_dtype, dev)
+        self.gamma_q = to_device(gamma_q, f32, dev)
+        self.gamma_qr = to_device(gamma_qr, f32, dev)
+        self.gamma_kr = to_device(gamma_kr, f32, dev)
+
+    def append(self, c, k_rope_raw, slot, pos, chunk: int = 1 << 16) -> None:
+        dt, dev = self.dims.torch_dtype, self.device
+        n = int(c.shape[0])
+        for t0 in range(0, n, chunk):
+            sl = slice(t0, min(n, t0 + chunk))
+            gqa_append(self.dims, self.cache, to_device(c[sl], dt, dev), to_device(k_rope_raw[sl], dt, dev),
+                       to_device(slot[sl], torch.int32, dev), to_device(pos[sl], torch.int32, dev), self.w_uk,
+                       self.gamma_k, self.w_uv, self.gamma_kr)
+
+    def set_queries(self, q, q_rope) -> None:
+        """The step's raw queries: q [batch, s_q, H, d_h], q_rope [batch, s_q, H, d_R]."""
+        dt, dev = self.dims.torch_dtype, self.device
+        self.q = to_device(q, dt, dev)
+        self.q_rope = to_device(q_rope, dt, dev)
+
+    def ensure_workspace(self, batch: int, s_q: int) -> torch.Tensor:
+        need = gqa_workspace_size(self.dims, self.cache.d_v, batch, s_q)
+        if self.workspace is None or self.workspace.numel() < need:
+            self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            workspace_init(self.workspace)
+        return self.workspace
+
+    def decode(self, block_table, seq_lens, s_q: int, selection=None, max_ctas: int = 0, out_v=None, lse=None):
+        """o_v [batch, s_q, H, d_v] and lse [batch, s_q, H]; ``selection`` [batch, s_q, g, k] for sparse."""
+        d, dev = self.dims, self.device
+        bt = to_device(block_table, torch.int32, dev)
+        sl = to_device(seq_lens, torch.int32, dev)
+        batch = bt.shape[0]
+        ws = self.ensure_workspace(batch, s_q)
+        if out_v is None:
+            out_v = torch.empty((batch, s_q, d.num_heads, self.cache.d_v), dtype=d.torch_dtype, device=dev)
+        if lse is None:
+            lse = torch.empty((batch, s_q, d.num_heads), dtype=torch.float32, device=dev)
+        sel = None if selection is None else to_device(selection, torch.int32, dev)
+        gqa_decode(d, self.cache, self.q, self.q_rope, self.gamma_q, self.gamma_qr, bt, sl, s_q, ws, out_v, lse,
+                   selection=sel, max_ctas=max_ctas)
+        return out_v, lse
+
+    def device_status(self) -> int:
+        return read_device_status(self.workspace)
+
+    def clear_status(self) -> None:
+        workspace_init(self.workspace)
+
+
+def gqa_session_from_inputs(inp, device="cuda") -> GqaSession:
+    """A GQA-route session from a seeded problem of a tied-groups workload: group weights loaded, every
+    context token expanded into the cache, the step's queries set."""
+    wl = inp.wl
+    dims = Dims(num_heads=wl.heads, num_groups=wl.groups, r_kv=wl.r_kv, d_h=wl.d_h, d_rope=wl.d_rope,
+                eps=wl.eps, softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta,
+                dtype=1 if wl.dtype == "bf16" else 0, block_size=wl.block_size)
+    s = GqaSession(dims, inp.num_blocks, wl.d_v, device=device)
+    w_uk, gamma_k, w_uv = inp.group_weights()
+    s.load_weights(w_uk, gamma_k, w_uv, inp.gamma_q, inp.gamma_qr, inp.gamma_kr)
+    s.append(inp.c, inp.k_rope, inp.token_slots(), inp.token_positions())
+    s.set_queries(inp.q, inp.q_rope)
+    return s
+

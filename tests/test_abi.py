@@ -170,3 +170,55 @@ def test_decode_up_validates_the_value_projection_before_any_launch():
     import dataclasses
     wide = dataclasses.replace(DIMS, r_kv=1024).c()
     assert _decode_up(lib, wide, 0x100, 64, 0x100) == qkn.ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- the GQA route
+GQA_DIMS = qkn.Dims(num_heads=128, num_groups=8, r_kv=512, d_h=128, d_rope=64)
+
+
+def _gqa_decode(lib, dims, cache, selection=None, sel_k=0, batch=1, q=0x100, out_v=0x100, ws=0x100):
+    return lib.qkn_gqa_decode(ctypes.byref(dims), ctypes.byref(cache), q, 0x100, 0x100, 0x100, 0x100, 1, 0x100,
+                              batch, 1, selection, sel_k, ws, 1 << 30, out_v, 0x100, 0, None)
+
+
+def _gqa_append(lib, dims, cache, n_tok=4, c_new=0x100, w_uk=0x100):
+    return lib.qkn_gqa_append(ctypes.byref(dims), ctypes.byref(cache), c_new, 0x100, 0x100, 0x100, n_tok, w_uk,
+                              0x100, 0x100, 0x100, None)
+
+
+def test_gqa_route_validates_before_any_launch():
+    lib = qkn.raw_library()
+    dims = GQA_DIMS.c()
+    cache = qkn._GqaCache(0x1000, 0x2000, 0x3000, 4, 128)
+    # widths the kernels take: (d_h, d_rope, d_v) = (128, 64, 128) or (64, 32, 64), bf16 only
+    assert _gqa_decode(lib, dims, qkn._GqaCache(0x1000, 0x2000, 0x3000, 4, 96)) == qkn.ERR_UNSUPPORTED
+    import dataclasses
+    f32 = dataclasses.replace(GQA_DIMS, dtype=qkn.F32).c()
+    assert _gqa_decode(lib, f32, cache) == qkn.ERR_UNSUPPORTED
+    assert _gqa_append(lib, f32, cache) == qkn.ERR_UNSUPPORTED
+    narrow = dataclasses.replace(GQA_DIMS, d_h=64, d_rope=32).c()
+    assert _gqa_decode(lib, narrow, qkn._GqaCache(0x1000, 0x2000, 0x3000, 4, 64), batch=0) == qkn.OK
+    # missing cache arrays, misaligned pointers, a selection without a length
+    assert _gqa_decode(lib, dims, qkn._GqaCache(0x1000, None, 0x3000, 4, 128)) == qkn.ERR_INVALID_ARG
+    assert _gqa_decode(lib, dims, qkn._GqaCache(0x1008, 0x2000, 0x3000, 4, 128)) == qkn.ERR_INVALID_ARG
+    assert _gqa_decode(lib, dims, cache, q=None) == qkn.ERR_INVALID_ARG
+    assert _gqa_decode(lib, dims, cache, q=0x104) == qkn.ERR_INVALID_ARG
+    assert _gqa_decode(lib, dims, cache, out_v=0x108) == qkn.ERR_INVALID_ARG
+    assert _gqa_decode(lib, dims, cache, ws=0x180) == qkn.ERR_INVALID_ARG       # workspace 256-byte aligned
+    assert _gqa_decode(lib, dims, cache, selection=0x100, sel_k=0) == qkn.ERR_INVALID_ARG
+    assert _gqa_decode(lib, dims, cache, batch=0) == qkn.OK                     # empty batch: no-op
+    assert _gqa_append(lib, dims, cache, n_tok=-1) == qkn.ERR_INVALID_ARG
+    assert _gqa_append(lib, dims, cache, n_tok=0) == qkn.OK
+    assert _gqa_append(lib, dims, cache, c_new=None) == qkn.ERR_INVALID_ARG
+    assert _gqa_append(lib, dims, cache, w_uk=0x104) == qkn.ERR_INVALID_ARG
+    odd_r = dataclasses.replace(GQA_DIMS, r_kv=520).c()       # the expansion stages 32 latent columns at a time
+    assert _gqa_append(lib, odd_r, cache) == qkn.ERR_UNSUPPORTED
+
+
+def test_gqa_workspace_holds_one_partial_per_slot():
+    # dense: 32 query rows per tile (s_q = 2, 16 heads per group), one tile per group, a partial
+    # (rows x d_v fp32 + lse) per (sequence, tile) pair and per CTA of the schedule
+    ws = qkn.gqa_workspace_size(GQA_DIMS, 128, 32, 2, num_sms=148)
+    assert ws >= 256 + (32 * 8 + 148) * 32 * (128 * 4 + 4)
+    assert qkn.gqa_workspace_size(GQA_DIMS, 128, 64, 2, num_sms=148) > ws
+

@@ -2,7 +2,8 @@
 import json
 import os
 
-from qk_normed_latent_qkn_b200.roofline import cache_bytes_per_token, decode_step_cost, flops_per_token_row
+from qk_normed_latent_qkn_b200.roofline import (cache_bytes_per_token, decode_step_cost, flops_per_token_row,
+                                                gqa_step_cost)
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_figures.json")))
 
@@ -35,3 +36,22 @@ def test_step_cost_counts_causal_pairs():
     assert c2.flops == (9 + 10) * 2 * flops_per_token_row(8, 4)
     assert c1.flops == 10 * 2 * flops_per_token_row(8, 4)
     assert c1.cache_bytes == 10 * (2 * 12 + 4)
+
+
+def test_gqa_route_intensity_sits_at_the_printed_ridge():
+    # the GQA route's g and s_q put a long-context step's intensity at about 37 FLOP/byte for both
+    # configurations the page names
+    fig = GOLDEN["gqa_route_intensity_h20_ridge_flop_per_byte"]
+    sh = fig["shape"]
+    for cfg in fig["configs"]:
+        L = 1 << 18
+        c = gqa_step_cost([L], cfg["s_q"], cfg["heads"], cfg["groups"], sh["d_h"], sh["d_rope"], sh["d_v"],
+                          elem=sh["elem_bytes"])
+        assert abs(c.intensity - fig["value"]) < 2.5, (cfg, c.intensity)
+
+
+def test_gqa_step_cost_counts_causal_pairs_and_group_bytes():
+    c = gqa_step_cost([10], 2, 4, 2, 8, 4, 6)
+    assert c.cache_bytes == 10 * 2 * (2 * (8 + 6) + 4)
+    assert c.flops == (9 + 10) * 4 * (2 * (8 + 4) + 2 * 6)
+
