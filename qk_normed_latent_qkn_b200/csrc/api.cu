@@ -631,7 +631,8 @@ qkn_status qkn_gqa_decode(const qkn_dims* dims, const qkn_gqa_cache* cache, cons
   gqa_tiling(dims, s_q, sparse, &a.rows, &a.tpg);
   a.ht_count = dims->num_groups * a.tpg;
   a.ncta = gqa_ncta(nsm, a.ht_count, max_ctas);
-  // starting an item (the tile's queries, the ring's first pages) costs about two pages of time
+  // starting an item (the tile's queries, filling the ring) is taken as two pages of time, an
+  // estimate from the ring's depth that no measurement has tuned yet
   a.item_cost = 2;
   a.selection = selection;
   a.sel_k = sparse ? sel_k : 0;
