@@ -44,7 +44,11 @@ rational arithmetic; invariance of the logits to rescaling c_t; softmax rows
 summing to 1; closed forms (one token, zero queries, identical tokens); a
 library softmax-attention routine on materialised keys; brute-force loops for
 the causal mask; RoPE's relative-position property; permutation invariance.
-The absolute outputs on the five workloads are parity unpinned beyond those
+The GQA route's pins: equality with the absorbed route over group-tied
+weights; torch's grouped-query attention on keys and values the check forms;
+a one-token closed form; a full selection equal to dense and an empty one
+giving zeros; a brute-force loop over a sparse selection.
+The absolute outputs on the workloads are parity unpinned beyond those
 properties: the pages print no worked example.
 """
 from __future__ import annotations
